@@ -1,0 +1,147 @@
+"""ctypes binding of the fp64 CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path never does.
+
+Every function takes numpy arrays (any float dtype is upcast to float64,
+which is exact for fp32 and bf16 values) and returns numpy arrays.  The
+arithmetic lives in ``lsh_oracle.cpp``; this file only marshals arguments and
+builds that file with the host C++ compiler when its library is missing or
+older than the source.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lsh_oracle.cpp")
+_LIB = os.path.join(_HERE, "liblsh_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile lsh_oracle.cpp into liblsh_oracle.so (plain -O2, no fast-math)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-fno-fast-math",
+                               _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_lsh_hash.argtypes = [I, I, I, I, I, I, P, P, P, P, P]
+        lib.oracle_lsh_sort.argtypes = [I, I, P, P]
+        lib.oracle_lsh_attend_fwd.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P]
+        lib.oracle_lsh_combine.argtypes = [I, I, I, I, I, P, P, P, P]
+        lib.oracle_lsh_attend_bwd.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P]
+        for f in (lib.oracle_lsh_hash, lib.oracle_lsh_sort, lib.oracle_lsh_attend_fwd,
+                  lib.oracle_lsh_combine, lib.oracle_lsh_attend_bwd):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, name: str):
+    if rc != 0:
+        raise ValueError(f"{name}: invalid argument (status {rc})")
+
+
+def lsh_hash(Q, rot, n_buckets: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Q [B,H,L,d], rot [R,d,nb/2] -> keys u32, buckets i32, near_tie u8, each [R,B,H,L]."""
+    Q = _f64(Q)
+    rot = _f64(rot)
+    B, H, L, d = Q.shape
+    R = rot.shape[0]
+    keys = np.zeros((R, B, H, L), np.uint32)
+    buckets = np.zeros((R, B, H, L), np.int32)
+    tie = np.zeros((R, B, H, L), np.uint8)
+    rc = _load().oracle_lsh_hash(B, H, L, d, n_buckets, R, _ptr(Q), _ptr(rot), _ptr(keys),
+                                 _ptr(buckets), _ptr(tie))
+    _check(rc, "oracle_lsh_hash")
+    return keys, buckets, tie
+
+
+def lsh_sort(keys: np.ndarray) -> np.ndarray:
+    """keys [..., L] u32 (bucket*L + position) -> perm [..., L] i32."""
+    keys = np.ascontiguousarray(keys, dtype=np.uint32)
+    L = keys.shape[-1]
+    rows = keys.size // L if L else 0
+    perm = np.zeros(keys.shape, np.int32)
+    _check(_load().oracle_lsh_sort(rows, L, _ptr(keys), _ptr(perm)), "oracle_lsh_sort")
+    return perm
+
+
+def lsh_attend_fwd(Q, V, keys, perm, chunk: int, causal: bool):
+    """-> o_part [R,B,H,L,d] and lse_r [R,B,H,L], both float64."""
+    Q = _f64(Q)
+    V = _f64(V)
+    keys = np.ascontiguousarray(keys, dtype=np.uint32)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    B, H, L, d = Q.shape
+    R = keys.shape[0]
+    o_part = np.zeros((R, B, H, L, d))
+    lse_r = np.zeros((R, B, H, L))
+    rc = _load().oracle_lsh_attend_fwd(B, H, L, d, R, chunk, int(bool(causal)), _ptr(Q), _ptr(V),
+                                       _ptr(keys), _ptr(perm), _ptr(o_part), _ptr(lse_r))
+    _check(rc, "oracle_lsh_attend_fwd")
+    return o_part, lse_r
+
+
+def lsh_combine(o_part, lse_r):
+    """o_part [R,B,H,L,d], lse_r [R,B,H,L] -> O [B,H,L,d], lse [B,H,L]."""
+    o_part = _f64(o_part)
+    lse_r = _f64(lse_r)
+    R, B, H, L, d = o_part.shape
+    O = np.zeros((B, H, L, d))
+    lse = np.zeros((B, H, L))
+    rc = _load().oracle_lsh_combine(R, B, H, L, d, _ptr(o_part), _ptr(lse_r), _ptr(O), _ptr(lse))
+    _check(rc, "oracle_lsh_combine")
+    return O, lse
+
+
+def lsh_attend_bwd(Q, V, dO, keys, perm, chunk: int, causal: bool):
+    """Gradients of sum(dO * O) with buckets frozen -> dQ, dV [B,H,L,d] float64."""
+    Q = _f64(Q)
+    V = _f64(V)
+    dO = _f64(dO)
+    keys = np.ascontiguousarray(keys, dtype=np.uint32)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    B, H, L, d = Q.shape
+    R = keys.shape[0]
+    dQ = np.zeros_like(Q)
+    dV = np.zeros_like(V)
+    rc = _load().oracle_lsh_attend_bwd(B, H, L, d, R, chunk, int(bool(causal)), _ptr(Q), _ptr(V),
+                                       _ptr(dO), _ptr(keys), _ptr(perm), _ptr(dQ), _ptr(dV))
+    _check(rc, "oracle_lsh_attend_bwd")
+    return dQ, dV
+
+
+def lsh_forward(Q, V, rot, n_buckets: int, chunk: int, causal: bool):
+    """The whole forward: hash -> sort -> attend -> combine.  Returns a dict of arrays."""
+    keys, buckets, tie = lsh_hash(Q, rot, n_buckets)
+    perm = lsh_sort(keys)
+    o_part, lse_r = lsh_attend_fwd(Q, V, keys, perm, chunk, causal)
+    O, lse = lsh_combine(o_part, lse_r)
+    return {"keys": keys, "buckets": buckets, "near_tie": tie, "perm": perm,
+            "o_part": o_part, "lse_r": lse_r, "O": O, "lse": lse}

@@ -1,0 +1,363 @@
+"""Pins of the fp64 CPU oracle against facts fixed outside the oracle itself.
+
+Each test checks the oracle against something it does not compute by its own
+code path: a probability the Reformer explainer states (collision rate
+1 - theta/pi for angular LSH), exact symmetries of the hash, library routines
+on special cases that reduce to dense attention, brute-force enumeration of
+bucket-mates on tiny inputs, closed forms (constant values, lone tokens,
+repeated rounds) and finite differences of the forward.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------------------
+# hash
+# ---------------------------------------------------------------------------
+
+def test_collision_probability_matches_one_minus_theta_over_pi(oracle):
+    """Reformer explainer, angular LSH: two vectors at angle theta share a
+    bucket with probability 1 - theta/pi (hyperplane case, n_buckets = 2)."""
+    d = 64
+    rounds = 100_000
+    thetas = np.linspace(0.15, math.pi - 0.15, 12)
+    rng = _rng(11)
+    basis, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    e0, e1 = basis[:, 0], basis[:, 1]
+    vecs = []
+    for th in thetas:
+        vecs.append(3.0 * e0)
+        vecs.append(0.5 * (math.cos(th) * e0 + math.sin(th) * e1))
+    Q = np.stack(vecs)[None, None]  # [1, 1, 24, d]
+    rot = rng.standard_normal((rounds, d, 1))
+    _, buckets, _ = oracle.lsh_hash(Q, rot, 2)
+    b = buckets[:, 0, 0, :]  # [rounds, 24]
+    for a, th in enumerate(thetas):
+        rate = np.mean(b[:, 2 * a] == b[:, 2 * a + 1])
+        assert abs(rate - (1.0 - th / math.pi)) < 0.01, (th, rate)
+
+
+@pytest.mark.parametrize("nb", [4, 16, 64, 1024])
+def test_hash_antipodal_symmetry(oracle, nb):
+    """Negating x negates every projection, so its sector is the opposite one:
+    bucket(-x) = (bucket(x) + nb/2) mod nb whenever there is no near tie."""
+    rng = _rng(nb)
+    x = rng.standard_normal((1, 1, 200, 64))
+    Q = np.concatenate([x, -x], axis=2)
+    rot = rng.standard_normal((3, 64, nb // 2))
+    _, b, tie = oracle.lsh_hash(Q, rot, nb)
+    bp, bn = b[..., :200], b[..., 200:]
+    ok = (tie[..., :200] == 0) & (tie[..., 200:] == 0)
+    assert ok.mean() > 0.95
+    assert np.array_equal(bn[ok], (bp[ok] + nb // 2) % nb)
+
+
+@pytest.mark.parametrize("nb", [2, 6, 32, 256])
+def test_hash_brute_force_over_sector_directions(oracle, nb):
+    """Brute force: enumerate the nb directions +R_j and -R_j as explicit
+    vectors and take the first direction of largest projection."""
+    rng = _rng(100 + nb)
+    Q = rng.standard_normal((2, 3, 50, 64))
+    rot = rng.standard_normal((2, 64, nb // 2))
+    keys, b, tie = oracle.lsh_hash(Q, rot, nb)
+    for r in range(2):
+        dirs = np.concatenate([rot[r], -rot[r]], axis=1)  # [d, nb] sector directions
+        proj = np.einsum("bhld,dn->bhln", Q, dirs)
+        expect = np.argmax(proj, axis=-1)  # first index of the maximum
+        ok = tie[r] == 0
+        assert np.array_equal(b[r][ok], expect[ok])
+    L = Q.shape[2]
+    pos = np.arange(L, dtype=np.uint64)
+    assert np.array_equal(keys.astype(np.uint64), b.astype(np.uint64) * L + pos)
+
+
+def test_hash_exact_ties_take_the_lowest_index(oracle):
+    """Duplicated or negated rotation columns make exact ties; the first index
+    of [p ; -p] wins and the tie is flagged."""
+    rng = _rng(5)
+    Q = rng.standard_normal((1, 1, 40, 16))
+    # columns 0 and 1 identical, column 2 much shorter: max |p| sits at 0 == 1
+    r = rng.standard_normal((16, 1))
+    rot = np.concatenate([r, r, 1e-3 * rng.standard_normal((16, 1))], axis=1)[None]
+    _, b, tie = oracle.lsh_hash(Q, rot, 6)
+    p0 = Q[0, 0] @ r[:, 0]
+    expect = np.where(p0 >= 0, 0, 3)
+    assert np.array_equal(b[0, 0, 0], expect)
+    assert np.all(tie == 1)
+    # column 1 = -column 0: z = (p, -p, -p, p); the first half wins the tie
+    rot2 = np.concatenate([r, -r], axis=1)[None]
+    _, b2, tie2 = oracle.lsh_hash(Q, rot2, 4)
+    assert np.array_equal(b2[0, 0, 0], np.where(p0 >= 0, 0, 1))
+    assert np.all(tie2 == 1)
+
+
+def test_hash_one_bucket_ignores_rotation(oracle):
+    rng = _rng(6)
+    Q = rng.standard_normal((2, 2, 32, 64))
+    keys, b, tie = oracle.lsh_hash(Q, np.zeros((3, 64, 0)), 1)
+    assert np.all(b == 0) and np.all(tie == 0)
+    assert np.array_equal(keys, np.broadcast_to(np.arange(32, dtype=np.uint32), keys.shape))
+
+
+# ---------------------------------------------------------------------------
+# sort
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("nb,L", [(2, 64), (8, 256), (64, 1000), (1024, 4096)])
+def test_sort_is_stable_bucket_order(oracle, nb, L):
+    rng = _rng(L)
+    buckets = rng.integers(0, nb, size=(3, L)).astype(np.uint64)
+    keys = (buckets * L + np.arange(L, dtype=np.uint64)).astype(np.uint32)
+    perm = oracle.lsh_sort(keys)
+    for row in range(3):
+        p = perm[row]
+        assert np.array_equal(np.sort(p), np.arange(L))
+        assert np.all(np.diff(keys[row][p].astype(np.int64)) > 0)
+        assert np.array_equal(p, np.lexsort((np.arange(L), buckets[row])))
+
+
+# ---------------------------------------------------------------------------
+# attention and combine
+# ---------------------------------------------------------------------------
+
+def _dense_reference(Q, V, causal, same_bucket=None):
+    """Dense shared-QK attention through torch's SDPA in float64: keys are the
+    unit queries, the diagonal gets -1e5, future positions -inf."""
+    q = torch.from_numpy(Q)
+    v = torch.from_numpy(V)
+    k = q / q.norm(dim=-1, keepdim=True)
+    L = q.shape[-2]
+    mask = torch.zeros(L, L, dtype=torch.float64)
+    if causal:
+        mask = mask.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), float("-inf"))
+    mask = mask.expand(q.shape[0], q.shape[1], L, L).clone()
+    if same_bucket is not None:
+        mask = mask.masked_fill(~torch.from_numpy(same_bucket), float("-inf"))
+    mask = mask + torch.diag(torch.full((L,), -1e5, dtype=torch.float64))
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=1.0 / math.sqrt(Q.shape[-1]))
+    return o.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_one_bucket_one_chunk_is_full_attention(oracle, causal):
+    """With one bucket and c = L, LSH attention is dense shared-QK attention
+    with the self mask."""
+    rng = _rng(7 + causal)
+    Q = rng.standard_normal((2, 3, 48, 64))
+    V = rng.standard_normal((2, 3, 48, 64))
+    out = oracle.lsh_forward(Q, V, np.zeros((1, 64, 0)), 1, 48, causal)
+    ref = _dense_reference(Q, V, causal)
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+    # lse: the library logsumexp of the scores with the diagonal replaced
+    q = torch.from_numpy(Q)
+    s = q @ (q / q.norm(dim=-1, keepdim=True)).transpose(-1, -2) / 8.0
+    s = s.clone()
+    s.diagonal(dim1=-2, dim2=-1).fill_(-1e5)
+    if causal:
+        s = s.masked_fill(torch.ones(48, 48, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(out["lse"], torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_two_chunks_see_the_whole_row(oracle, causal):
+    """With two chunks, chunk 0's previous chunk is chunk 1 and vice versa, so
+    every query sees every same-bucket key: dense attention under a
+    bucket-equality mask."""
+    rng = _rng(17 + causal)
+    Q = rng.standard_normal((1, 2, 64, 64))
+    V = rng.standard_normal((1, 2, 64, 64))
+    rot = rng.standard_normal((1, 64, 2))
+    out = oracle.lsh_forward(Q, V, rot, 4, 32, causal)
+    b = out["buckets"][0]
+    same = b[..., :, None] == b[..., None, :]
+    ref = _dense_reference(Q, V, causal, same_bucket=same)
+    np.testing.assert_allclose(out["O"], ref, rtol=0, atol=1e-12)
+
+
+def _brute_force(Q, V, buckets, chunk, causal):
+    """Per query, enumerate the same-bucket keys whose sorted chunk is the
+    query's own or the one before it (a set, wrapping), then take one
+    softmax per round and one over all rounds together."""
+    R = buckets.shape[0]
+    B, H, L, d = Q.shape
+    n_c = L // chunk
+    o_r = np.zeros((R, B, H, L, d))
+    lse_r = np.zeros((R, B, H, L))
+    O = np.zeros((B, H, L, d))
+    lse = np.zeros((B, H, L))
+    for b in range(B):
+        for h in range(H):
+            q = Q[b, h]
+            nrm = np.linalg.norm(q, axis=1)
+            all_s = [[] for _ in range(L)]
+            all_v = [[] for _ in range(L)]
+            for r in range(R):
+                bk = buckets[r, b, h]
+                order = np.lexsort((np.arange(L), bk))
+                slot = np.empty(L, int)
+                slot[order] = np.arange(L)
+                ch = slot // chunk
+                for i in range(L):
+                    allowed = {ch[i], (ch[i] - 1) % n_c}
+                    s, vs = [], []
+                    for j in range(L):
+                        if bk[j] != bk[i] or ch[j] not in allowed:
+                            continue
+                        if causal and j > i:
+                            continue
+                        sc = -1e5 if j == i else float(q[i] @ q[j]) / (nrm[j] * math.sqrt(d))
+                        s.append(sc)
+                        vs.append(V[b, h, j])
+                    s = np.array(s)
+                    m = s.max()
+                    l = m + math.log(np.exp(s - m).sum())
+                    lse_r[r, b, h, i] = l
+                    o_r[r, b, h, i] = (np.exp(s - l)[:, None] * np.array(vs)).sum(0)
+                    all_s[i].extend(s)
+                    all_v[i].extend(vs)
+            for i in range(L):
+                s = np.array(all_s[i])
+                m = s.max()
+                l = m + math.log(np.exp(s - m).sum())
+                lse[b, h, i] = l
+                O[b, h, i] = (np.exp(s - l)[:, None] * np.array(all_v[i])).sum(0)
+    return o_r, lse_r, O, lse
+
+
+@pytest.mark.parametrize("L,chunk,nb,R,causal", [
+    (8, 4, 2, 1, False), (16, 4, 4, 2, True), (32, 8, 8, 3, False),
+    (48, 16, 4, 2, True), (24, 8, 2, 2, True), (40, 8, 6, 1, False),
+])
+def test_brute_force_bucket_mates(oracle, L, chunk, nb, R, causal):
+    rng = _rng(L * 31 + nb)
+    Q = rng.standard_normal((1, 2, L, 16))
+    V = rng.standard_normal((1, 2, L, 16))
+    rot = rng.standard_normal((R, 16, nb // 2))
+    out = oracle.lsh_forward(Q, V, rot, nb, chunk, causal)
+    o_r, lse_r, O, lse = _brute_force(Q, V, out["buckets"], chunk, causal)
+    np.testing.assert_allclose(out["o_part"], o_r, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["lse_r"], lse_r, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(out["O"], O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], lse, rtol=1e-12, atol=1e-9)
+
+
+def test_constant_values_give_constant_output(oracle):
+    rng = _rng(9)
+    Q = rng.standard_normal((1, 2, 64, 64))
+    V = np.full((1, 2, 64, 64), 3.25)
+    out = oracle.lsh_forward(Q, V, rng.standard_normal((3, 64, 4)), 8, 16, True)
+    np.testing.assert_allclose(out["O"], 3.25, rtol=0, atol=1e-12)
+
+
+def test_lone_token_returns_its_own_value(oracle):
+    """A token with no bucket-mate in its window attends only to itself:
+    o_r = v and lse_r = -1e5 exactly."""
+    rng = _rng(10)
+    L, c = 32, 4
+    Q = rng.standard_normal((1, 1, L, 64))
+    V = rng.standard_normal((1, 1, L, 64))
+    out = oracle.lsh_forward(Q, V, rng.standard_normal((1, 64, 32)), 64, c, False)
+    bk = out["buckets"][0, 0, 0]
+    perm = out["perm"][0, 0, 0]
+    slot = np.empty(L, int)
+    slot[perm] = np.arange(L)
+    n_c = L // c
+    lone = 0
+    for i in range(L):
+        chs = {slot[i] // c, (slot[i] // c - 1) % n_c}
+        mates = [j for j in range(L) if j != i and bk[j] == bk[i] and slot[j] // c in chs]
+        if not mates:
+            lone += 1
+            assert out["lse_r"][0, 0, 0, i] == -1e5
+            np.testing.assert_array_equal(out["o_part"][0, 0, 0, i], V[0, 0, i])
+    assert lone > 5
+
+
+def test_identical_rounds_equal_one_round(oracle):
+    """R copies of one rotation: the combine averages R equal results, so O is
+    the one-round output and lse grows by ln R."""
+    rng = _rng(12)
+    Q = rng.standard_normal((1, 2, 64, 64))
+    V = rng.standard_normal((1, 2, 64, 64))
+    r1 = rng.standard_normal((1, 64, 8))
+    one = oracle.lsh_forward(Q, V, r1, 16, 16, True)
+    four = oracle.lsh_forward(Q, V, np.repeat(r1, 4, axis=0), 16, 16, True)
+    np.testing.assert_allclose(four["O"], one["O"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(four["lse"], one["lse"] + math.log(4), rtol=1e-12, atol=1e-9)
+
+
+def test_combine_of_one_round_is_identity(oracle):
+    rng = _rng(13)
+    o = rng.standard_normal((1, 2, 3, 8, 16))
+    l = rng.standard_normal((1, 2, 3, 8))
+    O, lse = oracle.lsh_combine(o, l)
+    np.testing.assert_allclose(O, o[0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, l[0], rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,chunk,nb,R,causal", [(16, 4, 4, 2, True), (32, 8, 2, 3, False),
+                                                  (24, 8, 4, 1, True)])
+def test_backward_matches_finite_differences(oracle, L, chunk, nb, R, causal):
+    """Central differences of sum(dO * O) in fp64 with buckets frozen."""
+    rng = _rng(L + 1000 * R)
+    d = 8
+    Q = rng.standard_normal((1, 2, L, d))
+    V = rng.standard_normal((1, 2, L, d))
+    dO = rng.standard_normal((1, 2, L, d))
+    rot = rng.standard_normal((R, d, nb // 2))
+    keys, _, _ = oracle.lsh_hash(Q, rot, nb)
+    perm = oracle.lsh_sort(keys)
+    dQ, dV = oracle.lsh_attend_bwd(Q, V, dO, keys, perm, chunk, causal)
+
+    def loss(Qx, Vx):
+        o_part, lse_r = oracle.lsh_attend_fwd(Qx, Vx, keys, perm, chunk, causal)
+        O, _ = oracle.lsh_combine(o_part, lse_r)
+        return float((dO * O).sum())
+
+    h = 1e-5
+    idx = [tuple(rng.integers(0, s) for s in Q.shape) for _ in range(40)]
+    for ix in idx:
+        for X, G, name in ((Q, dQ, "dQ"), (V, dV, "dV")):
+            Xp = X.copy(); Xp[ix] += h
+            Xm = X.copy(); Xm[ix] -= h
+            fd = (loss(Xp, V) - loss(Xm, V)) / (2 * h) if name == "dQ" else \
+                 (loss(Q, Xp) - loss(Q, Xm)) / (2 * h)
+            assert abs(fd - G[ix]) <= 1e-6 * max(1.0, abs(fd)), (name, ix, fd, G[ix])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_one_bucket_matches_autograd(oracle, causal):
+    """nb = 1 and c = L: dense shared-QK attention, differentiated by torch
+    autograd in float64 (key normalisation included)."""
+    rng = _rng(21 + causal)
+    L, d = 32, 16
+    Q = rng.standard_normal((1, 2, L, d))
+    V = rng.standard_normal((1, 2, L, d))
+    dO = rng.standard_normal((1, 2, L, d))
+    keys, _, _ = oracle.lsh_hash(Q, np.zeros((1, d, 0)), 1)
+    perm = oracle.lsh_sort(keys)
+    dQ, dV = oracle.lsh_attend_bwd(Q, V, dO, keys, perm, L, causal)
+    q = torch.from_numpy(Q).requires_grad_(True)
+    v = torch.from_numpy(V).requires_grad_(True)
+    k = q / q.norm(dim=-1, keepdim=True)
+    mask = torch.zeros(L, L, dtype=torch.float64)
+    if causal:
+        mask = mask.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), float("-inf"))
+    mask = mask + torch.diag(torch.full((L,), -1e5, dtype=torch.float64))
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=1.0 / math.sqrt(d))
+    (o * torch.from_numpy(dO)).sum().backward()
+    np.testing.assert_allclose(dQ, q.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dV, v.grad.numpy(), rtol=0, atol=1e-10)
