@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Benchmark of the LSH-attention hot path on B200.
+
+Headline: forward tokens/s (B*L per second, all heads and 8 hash rounds) on
+the L=65536 workload (B=1, H=8, d=64, n_buckets=1024, n_rounds=8, chunk=64,
+causal, bf16), one step = hash -> sort -> chunk attention with the fused
+round combine, inputs resident in HBM, L2 flushed (256 MB memset) between
+timed steps.  Also reported: fwd+bwd tokens/s (L=16384 workload and an
+L=65536 variant), the same forward end to end from pinned host buffers, per
+stage times, the roofline of the dominant kernel, clocks, and the CPU
+oracle timed on the host cores.
+
+``--impl reference`` times the CPU oracle (the reference arm) on a bounded
+sample of the same workload.  Under torchrun every rank runs the full
+workload on its own GPU (weak scaling, no data-path collective); timings are
+max-reduced over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from lsh_attention_long_b200 import workloads as W  # noqa: E402
+
+METRIC = "LSH-attention tokens/s (fwd, fwd+bwd) at L=65536, 8 rounds; % of roofline"
+HEADLINE = "fwd_bf16_L65536"
+BWD_WORKLOAD = "fwdbwd_bf16_L16384"
+FLUSH_BYTES = 256 << 20
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=HEADLINE)
+    p.add_argument("--no-extras", action="store_true",
+                   help="headline only: skip fwd+bwd, e2e and the CPU baseline")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# process group (one rank per GPU; collectives only for barriers and timing)
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed regions
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML every
+    10 ms on a background thread while the timed region runs."""
+
+    REASONS = (("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
+               ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
+               ("nvmlClocksEventReasonSwThermalSlowdown", "sw_thermal_slowdown"),
+               ("nvmlClocksEventReasonSwPowerCap", "sw_power_cap"),
+               ("nvmlClocksEventReasonHwPowerBrakeSlowdown", "hw_power_brake_slowdown"))
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.err = None
+        self._stop = None
+        self._thread = None
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = int(vis.split(",")[self.index]) if vis and vis.split(",")[0].isdigit() \
+                else self.index
+            h = nv.nvmlDeviceGetHandleByIndex(phys)
+            self.smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                      nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                      nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.01)
+
+        self._nv = nv
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+        nv = self._nv
+        reasons = []
+        for attr, name in self.REASONS:
+            bit = getattr(nv, attr, 0)
+            if any(r[2] & bit for r in self.rows):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.smax,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": round(max(r[1] for r in self.rows), 1), "source": "nvml 10 ms"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per stage (per call of the stage on workload w)
+# ---------------------------------------------------------------------------
+
+def stage_work(w: W.Workload):
+    s = 2 if w.dtype == "bf16" else 4
+    d, R = w.d, w.n_rounds
+    n_tok = w.B * w.H * w.L
+    tr = n_tok * R
+    return {
+        # Q read once for all rounds, one u32 key written per token-round
+        "hash": {"bytes": n_tok * d * s + tr * 4, "flops": tr * d * w.n_buckets},
+        # read a key, write a permutation entry
+        "sort": {"bytes": tr * 8, "flops": 0},
+        # gather q and v rows, the perm entry and the packed key per
+        # token-round; fp32 partial (o_r, lse_r) written for rounds < R-1 and
+        # read back by the combine; O and lse written once
+        "attend": {"bytes": tr * (2 * d * s + 8) + 2 * n_tok * (R - 1) * (4 * d + 4)
+                   + n_tok * (d * s + 4),
+                   "flops": tr * 8 * w.chunk * d},
+    }
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def device_inputs(w: W.Workload, dev):
+    inp = W.make_inputs(w)
+    return {k: v.to(dev) for k, v in inp.items()}
+
+
+def run_ours(args, world, rank):
+    import lsh_attention_long_b200 as L
+    L.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.WORKLOADS[args.workload]
+    t = device_inputs(w, dev)
+    Q, V, rot = t["Q"], t["V"], t["rot"]
+    R, B, H, Lx = w.n_rounds, w.B, w.H, w.L
+    shape = L.make_shape(B, H, Lx, w.d, w.n_buckets, R, w.chunk, w.causal, Q.dtype)
+    ws = L.workspace(shape, dev)
+    keys = torch.empty((R, B, H, Lx), dtype=torch.int32, device=dev)
+    perm = torch.empty_like(keys)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, H, Lx), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        L.lsh_hash(Q, rot, w.n_buckets, keys=keys, want_buckets=False)
+        ev[1].record(stream)
+        L.lsh_sort(keys, w.n_buckets, perm=perm)
+        ev[2].record(stream)
+        L.lsh_attend_fwd(Q, V, keys, perm, w.n_buckets, w.chunk, w.causal, O=O, lse=lse, ws=ws)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    stage_ms = {"hash": 0.0, "sort": 0.0, "attend": 0.0}
+    total_ms = 0.0
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for _ in range(args.steps):
+            flush.zero_()
+            ev[0].record(stream)
+            step()
+            ev[3].record(stream)
+            ev[3].synchronize()
+            a, b, c = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3])
+            stage_ms["hash"] += a
+            stage_ms["sort"] += b
+            stage_ms["attend"] += c
+            total_ms += a + b + c
+        torch.cuda.synchronize()
+    barrier(world)
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    launches_per_step = 1 + 1 + (2 if R > 1 else 1)
+    value = world * B * Lx * args.steps / (total_ms / 1e3)
+
+    peaks, peak_kind = load_peaks()
+    work = stage_work(w)
+    stages = {}
+    for name, ms in stage_ms.items():
+        sec = ms / args.steps / 1e3
+        gbs = work[name]["bytes"] / sec / 1e9
+        tfs = work[name]["flops"] / sec / 1e12
+        stages[name] = {"ms": round(ms / args.steps, 4), "GB_s": round(gbs, 1),
+                        "TFLOP_s": round(tfs, 2),
+                        "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                        "tensor_frac": round(tfs / peaks["bf16_tflops"], 4)}
+    dom = max(stage_ms, key=stage_ms.get)
+    bound = "tensor" if dom == "hash" and w.dtype == "bf16" and w.n_buckets >= 256 else "hbm"
+    traffic = TRAFFIC.get((dom, w.name))
+    if bound == "hbm":
+        roof = {"bound": "hbm", "kernel": dom, "achieved": stages[dom]["GB_s"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": stages[dom]["hbm_frac"],
+                "traffic": traffic, "peak_source": peak_kind}
+    else:
+        roof = {"bound": "tensor", "kernel": dom, "achieved": stages[dom]["TFLOP_s"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": stages[dom]["tensor_frac"], "traffic": traffic,
+                "peak_source": peak_kind}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian Q, V, rotations)",
+        "config": {"workload": w.name, "B": B, "H": H, "L": Lx, "d": w.d,
+                   "n_buckets": w.n_buckets, "n_rounds": R, "chunk": w.chunk,
+                   "causal": w.causal, "l2": "flushed between timed steps (256 MB memset)",
+                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "roofline": roof, "stages": stages,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_extras:
+        result["e2e"] = run_e2e(args, w, world)
+        result["fwd_bwd"] = {BWD_WORKLOAD: run_fwd_bwd(args, W.WORKLOADS[BWD_WORKLOAD], world),
+                             "fwd_bf16_L65536+bwd": run_fwd_bwd(args, w, world)}
+    del flush, ws
+    return result
+
+
+def run_e2e(args, w, world):
+    """The same forward through the public API with host buffers: pinned
+    host -> device copies of Q, V and rotations, one lsh_forward call, and
+    the device -> pinned host copy of O, all inside the timed region."""
+    import lsh_attention_long_b200 as L
+    dev = torch.device("cuda", torch.cuda.current_device())
+    host = {k: v.pin_memory() for k, v in W.make_inputs(w).items()}
+    dq = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    shape = L.make_shape(w.B, w.H, w.L, w.d, w.n_buckets, w.n_rounds, w.chunk, w.causal,
+                         host["Q"].dtype)
+    ws = L.workspace(shape, dev)
+    out = {"keys": torch.empty((w.n_rounds, w.B, w.H, w.L), dtype=torch.int32, device=dev)}
+    out["perm"] = torch.empty_like(out["keys"])
+    out["O"] = torch.empty_like(dq["Q"])
+    out["lse"] = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    O_host = torch.empty_like(host["Q"]).pin_memory()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(3, args.steps // 4)
+
+    def step():
+        for k in ("Q", "V", "rot"):
+            dq[k].copy_(host[k], non_blocking=True)
+        L.lsh_forward(dq["Q"], dq["V"], dq["rot"], w.n_buckets, w.chunk, w.causal, out=out, ws=ws)
+        O_host.copy_(out["O"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = 0.0
+    for _ in range(steps):
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    bi = sum(host[k].numel() * host[k].element_size() for k in ("Q", "V", "rot"))
+    bo = O_host.numel() * O_host.element_size()
+    return {"value": round(world * w.B * w.L * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": steps,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+def run_fwd_bwd(args, w, world):
+    """Forward + backward (dQ, dV with buckets frozen) tokens/s, device-resident."""
+    import lsh_attention_long_b200 as L
+    dev = torch.device("cuda", torch.cuda.current_device())
+    t = device_inputs(w, dev)
+    if "dO" not in t:
+        t["dO"] = W.gaussian(tuple(t["Q"].shape), 2, t["Q"].dtype).to(dev)
+    shape = L.make_shape(w.B, w.H, w.L, w.d, w.n_buckets, w.n_rounds, w.chunk, w.causal,
+                         t["Q"].dtype)
+    ws = L.workspace(shape, dev)
+    out = {"keys": torch.empty((w.n_rounds, w.B, w.H, w.L), dtype=torch.int32, device=dev)}
+    out["perm"] = torch.empty_like(out["keys"])
+    out["O"] = torch.empty_like(t["Q"])
+    out["lse"] = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    dQ, dV = torch.empty_like(t["Q"]), torch.empty_like(t["V"])
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    steps = max(3, args.steps // 4)
+
+    def step():
+        e[0].record(stream)
+        L.lsh_forward(t["Q"], t["V"], t["rot"], w.n_buckets, w.chunk, w.causal, out=out, ws=ws)
+        e[1].record(stream)
+        L.lsh_attend_bwd(t["Q"], t["V"], out["O"], t["dO"], out["keys"], out["perm"], out["lse"],
+                         w.n_buckets, w.chunk, w.causal, dQ=dQ, dV=dV, ws=ws)
+        e[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    fwd = bwd = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        step()
+        e[2].synchronize()
+        fwd += e[0].elapsed_time(e[1])
+        bwd += e[1].elapsed_time(e[2])
+    barrier(world)
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error in fwd+bwd")
+    tot = max_over_ranks(fwd + bwd, world)
+    return {"value": round(world * w.B * w.L * steps / (tot / 1e3), 1), "unit": "tokens/s",
+            "ms_fwd": round(fwd / steps, 4), "ms_bwd": round(bwd / steps, 4), "steps": steps,
+            "config": {"B": w.B, "H": w.H, "L": w.L, "n_buckets": w.n_buckets,
+                       "n_rounds": w.n_rounds, "chunk": w.chunk, "causal": w.causal}}
+
+
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the kernel as it stands, keyed by (stage, workload); None until taken.
+TRAFFIC = {}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------
+
+class OracleSampler:
+    """Times the fp64 CPU oracle (single thread, as it stands) on a bounded
+    sample of a workload and scales each stage to the whole step.
+
+    Setup (untimed): the oracle hashes one full row (head 0, round 0) so that
+    the sort and attention samples have real keys.  A timed sample is then:
+    the oracle's hash of `n_tok` tokens of head 0 for round 0, its sort of
+    that row, its attention for the queries of `n_chunks` chunks of that row,
+    and its combine over `n_tok` tokens.  Each stage's time is scaled by the
+    number of such units in the whole step (B*H*L*R tokens hashed, B*H*R rows
+    sorted, B*H*R*L/c chunks attended, B*H*L tokens combined)."""
+
+    def __init__(self, w: W.Workload):
+        from oracle import oracle as cpu_oracle
+        import numpy as np
+        cpu_oracle.build()
+        self.o, self.np, self.w = cpu_oracle, np, w
+        inp = W.make_inputs(w)
+        self.Q = inp["Q"][:1, :1].float().numpy()
+        self.V = inp["V"][:1, :1].float().numpy()
+        self.rot = inp["rot"][:1].float().numpy()
+        self.keys, _, _ = cpu_oracle.lsh_hash(self.Q, self.rot, w.n_buckets)
+        self.perm = cpu_oracle.lsh_sort(self.keys)
+
+    def step(self, n_tok: int, n_chunks: int):
+        w, o, np = self.w, self.o, self.np
+        t0 = time.perf_counter()
+        o.lsh_hash(self.Q[:, :, :n_tok], self.rot, w.n_buckets)
+        t1 = time.perf_counter()
+        o.lsh_sort(self.keys)
+        t2 = time.perf_counter()
+        o.lsh_attend_fwd_range(self.Q, self.V, self.keys, self.perm, w.chunk, w.causal, 0,
+                               n_chunks)
+        t3 = time.perf_counter()
+        part = np.zeros((w.n_rounds, 1, 1, n_tok, w.d))
+        o.lsh_combine(part, np.zeros((w.n_rounds, 1, 1, n_tok)))
+        t4 = time.perf_counter()
+        rows = w.B * w.H * w.n_rounds
+        full = ((t1 - t0) / n_tok * w.B * w.H * w.L * w.n_rounds
+                + (t2 - t1) * rows
+                + (t3 - t2) / n_chunks * rows * (w.L // w.chunk)
+                + (t4 - t3) / n_tok * w.B * w.H * w.L)
+        return t4 - t0, full
+
+    def describe(self, n_tok, n_chunks):
+        w = self.w
+        return (f"{w.name}: oracle hash of {n_tok} tokens (head 0, round 0), sort of one "
+                f"{w.L}-token row, attention for {n_chunks} chunks of that row, combine of "
+                f"{n_tok} tokens; each stage scaled by its unit count to the whole step "
+                f"(B*H*L*R hashes, B*H*R rows, B*H*R*L/c chunks); single-threaded fp64")
+
+
+def run_cpu_baseline(w):
+    s = OracleSampler(w)
+    n_tok, n_chunks = 8192, 128
+    sec, full = s.step(n_tok, n_chunks)
+    return {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle", "sample": s.describe(n_tok, n_chunks) + f"; sample took {sec:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    w = W.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    s = OracleSampler(w)
+    # a few minutes in all: about 150 s of sampling over warm-up + timed steps
+    per_step = 150.0 / (args.warmup + args.steps)
+    probe, _ = s.step(256, 4)
+    scale = max(1.0, min(32.0, per_step / max(probe, 1e-3)))
+    n_tok, n_chunks = int(256 * scale), max(1, int(4 * scale))
+    full = []
+    for i in range(args.warmup + args.steps):
+        _, f = s.step(n_tok, n_chunks)
+        if i >= args.warmup:
+            full.append(f)
+    per = sum(full) / len(full)
+    value = w.B * w.L / per
+    sample = s.describe(n_tok, n_chunks)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "n_buckets": w.n_buckets, "n_rounds": w.n_rounds, "chunk": w.chunk,
+                   "causal": w.causal},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 only; other ranks exit without work
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        res = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), 0)
+        print(json.dumps(res), flush=True)
+        return
+    world, rank, _ = dist_setup(args.gpus)
+    try:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device for --impl ours")
+        res = run_ours(args, world, rank)
+        if rank == 0 and not args.no_extras and world == 1:
+            res["cpu_baseline"] = run_cpu_baseline(W.WORKLOADS[args.workload])
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

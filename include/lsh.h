@@ -1,0 +1,162 @@
+/*
+ * lsh.h -- C ABI of the B200 (sm_100a) shared-QK LSH attention library.
+ *
+ * The library implements Reformer's LSH attention as described in
+ * "Reformer explainer" (akshathtiwari.co.in/blog/reformer, its single
+ * section) and "Reformer: The Efficient Transformer" (codewithpapers.app
+ * listing, abstract): tokens are hashed by the angular sector they fall
+ * into after a random rotation, queries and keys are tied (shared-QK), tokens
+ * are sorted by bucket and cut into equal chunks that attend to their
+ * bucket-mates, and several hash rounds are unioned.  The exact arithmetic
+ * is the five-step definition below:
+ *
+ *   1. hash     bucket = argmax([q.R_r ; -q.R_r]), R_r of shape [d, nb/2]
+ *               (lowest index wins a tie), key = bucket*L + position;
+ *   2. sort     stable sort of every (round, batch, head) row by
+ *               (bucket, position);
+ *   3. attend   chunks of `chunk` sorted slots attend to themselves and to the
+ *               previous chunk (chunk 0 wraps to the last; a single chunk
+ *               attends to itself once); keys are q/|q|, scores are scaled by
+ *               1/sqrt(d); another bucket or (causal) a later position
+ *               scores -inf, the token itself scores -1e5 (replacing its
+ *               score), so it is used only when nothing else is left;
+ *   4. scatter  each round's output o_r and logsumexp lse_r land at the
+ *               token's original position;
+ *   5. combine  lse = logsumexp_r lse_r,  O = sum_r exp(lse_r - lse) o_r.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense, row-major DEVICE pointers owned by the caller.
+ *     The library allocates nothing; scratch memory comes from the caller's
+ *     workspace `ws` of `ws_bytes` bytes (see lsh_workspace_size).
+ *   - Layouts: Q, V, O, dO, dQ, dV are [B, H, L, d] in the shape's dtype;
+ *     rot is [n_rounds, d, n_buckets/2] in the same dtype; keys, buckets and
+ *     perm are [n_rounds, B, H, L]; o_part is [n_rounds, B, H, L, d] fp32;
+ *     lse_r is [n_rounds, B, H, L] fp32; lse is [B, H, L] fp32.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on it.  Argument errors are returned before any
+ *     launch; a launch failure returns LSH_ERR_CUDA.  Errors found by a
+ *     kernel (malformed keys) are recorded in a device status word that
+ *     lsh_device_status() reads.
+ *   - Supported: d == 64; dtype LSH_F32 or LSH_BF16; n_buckets == 1 or an
+ *     even number 2..32768; n_buckets * L < 2^31; B*H*L*n_rounds < 2^31;
+ *     n_rounds*B*H <= 65535; chunk >= 1 divides L; chunk <= 64.  B, H or L
+ *     equal to 0 is an empty call that returns LSH_OK without launching.
+ *   - Every buffer must be 16-byte aligned.
+ */
+#ifndef LSH_ATTENTION_LSH_H_
+#define LSH_ATTENTION_LSH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LSH_API __attribute__((visibility("default")))
+#else
+#define LSH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSH_OK = 0,
+  LSH_ERR_INVALID_ARG = 1, /* null pointer, negative size, chunk not dividing L, ... */
+  LSH_ERR_UNSUPPORTED = 2, /* valid but outside the supported set above */
+  LSH_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  LSH_ERR_WORKSPACE = 4,   /* ws is NULL or smaller than lsh_workspace_size() */
+  LSH_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+  LSH_ERR_BAD_KEYS = 6     /* keys not of the form bucket*L + position, bucket < n_buckets */
+} lsh_status;
+
+typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
+
+typedef struct lsh_shape {
+  int32_t B;         /* batch */
+  int32_t H;         /* heads */
+  int32_t L;         /* sequence length */
+  int32_t d;         /* head dimension (64) */
+  int32_t n_buckets; /* buckets per hash round */
+  int32_t n_rounds;  /* hash rounds R */
+  int32_t chunk;     /* chunk length c in sorted slots */
+  int32_t causal;    /* nonzero: a later original position is masked */
+  int32_t dtype;     /* lsh_dtype of Q, V, rot, O, dO, dQ, dV */
+} lsh_shape;
+
+/* Bytes of workspace that covers any call below for this shape (the largest
+ * need: the per-round partials of lsh_attend_fwd when the caller passes no
+ * o_part / lse_r, or the fp32 gradient accumulators of lsh_attend_bwd).
+ * Returns 0 for an invalid or empty shape. */
+LSH_API size_t lsh_workspace_size(const lsh_shape* shape);
+
+/* Step 1 (hash).  For every round r and token (b, h, i):
+ *   p = Q[b,h,i,:] . rot[r,:,:]   (fp32 accumulation of exact products for
+ *                                  bf16; fp32 FMA for f32),
+ *   bucket = first index of the maximum of [p ; -p],
+ *   keys[r,b,h,i] = bucket*L + i.
+ * Q: [B,H,L,d]; rot: [R,d,n_buckets/2] (ignored, may be NULL, when
+ * n_buckets == 1); keys: [R,B,H,L] u32 (required); buckets: [R,B,H,L] i32
+ * or NULL. */
+LSH_API lsh_status lsh_hash(const lsh_shape* shape, const void* Q, const void* rot, uint32_t* keys,
+                    int32_t* buckets, void* stream);
+
+/* Step 2 (sort).  For every row (r, b, h), perm[r,b,h,t] = original position
+ * at sorted slot t, with slots in ascending (bucket, position) order: a
+ * stable counting sort on the bucket.  keys must be as lsh_hash writes them;
+ * a malformed key records LSH_ERR_BAD_KEYS in the device status word.
+ * ws is not used by the current kernels (may be NULL). */
+LSH_API lsh_status lsh_sort(const lsh_shape* shape, const uint32_t* keys, int32_t* perm, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Steps 3-5 (gather -> chunk attention -> scatter, fused combine).
+ * Q, V: [B,H,L,d]; keys, perm: from lsh_hash / lsh_sort.
+ * o_part: [R,B,H,L,d] fp32 or NULL; lse_r: [R,B,H,L] fp32 or NULL.
+ * O: [B,H,L,d] in dtype, or NULL to skip the combine (then o_part and lse_r
+ * are required and receive every round).  lse: [B,H,L] fp32 or NULL.
+ * When O is given, the combine runs in the epilogue of the last round;
+ * partials of the earlier rounds go to o_part/lse_r when given, else to ws
+ * (then ws_bytes >= lsh_workspace_size()). */
+LSH_API lsh_status lsh_attend_fwd(const lsh_shape* shape, const void* Q, const void* V,
+                          const uint32_t* keys, const int32_t* perm, float* o_part,
+                          float* lse_r, void* O, float* lse, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Step 5 alone: O = sum_r exp(lse_r - lse) o_part[r], lse = logsumexp_r lse_r.
+ * o_part [R,B,H,L,d] fp32, lse_r [R,B,H,L] fp32 -> O [B,H,L,d] dtype,
+ * lse [B,H,L] fp32 (or NULL). */
+LSH_API lsh_status lsh_combine(const lsh_shape* shape, const float* o_part, const float* lse_r, void* O,
+                       float* lse, void* stream);
+
+/* Whole forward in one call: lsh_hash -> lsh_sort -> lsh_attend_fwd with the
+ * fused combine.  keys and perm are outputs (they are also what the backward
+ * needs); buckets may be NULL; lse [B,H,L] fp32 is required (the backward
+ * needs it).  ws_bytes >= lsh_workspace_size(). */
+LSH_API lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void* V, const void* rot,
+                       uint32_t* keys, int32_t* buckets, int32_t* perm, void* O, float* lse,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of steps 3-5 with buckets and permutations held constant.
+ * Given the forward's O [B,H,L,d] and lse [B,H,L] and the upstream gradient
+ * dO [B,H,L,d], writes dQ and dV [B,H,L,d] in dtype.  dQ includes the path
+ * through the key normalisation q/|q|.  Masked entries (another bucket, a
+ * later position, the token itself) carry no score gradient; the token's own
+ * value still receives the weight it was given.  ws_bytes >=
+ * lsh_workspace_size(). */
+LSH_API lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const void* V, const void* O,
+                          const void* dO, const uint32_t* keys, const int32_t* perm,
+                          const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Synchronises `stream`, returns the first error a kernel recorded since the
+ * last call (LSH_OK if none) and clears it.  LSH_ERR_CUDA if the
+ * synchronisation itself fails. */
+LSH_API lsh_status lsh_device_status(void* stream);
+
+/* Static text for a status code. */
+LSH_API const char* lsh_status_string(lsh_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSH_ATTENTION_LSH_H_ */

@@ -1,0 +1,11 @@
+"""B200-native shared-QK LSH attention (Reformer), forward and backward.
+
+The compute lives in ``liblsh.so`` (hand-written sm_100a CUDA kernels behind
+the C ABI of ``include/lsh.h``); :mod:`lsh_attention_long_b200.lsh` is its
+ctypes binding and :mod:`lsh_attention_long_b200.workloads` draws the seeded
+synthetic inputs.
+"""
+
+from .lsh import (LshError, Shape, load_library, lsh_attend_bwd, lsh_attend_fwd,  # noqa: F401
+                  lsh_combine, lsh_device_status, lsh_forward, lsh_hash, lsh_sort,
+                  lsh_workspace_size, make_shape, workspace)

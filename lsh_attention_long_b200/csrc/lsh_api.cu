@@ -1,0 +1,320 @@
+// C ABI of the LSH attention library (declared in include/lsh.h): argument
+// checks, workspace carve-up and kernel dispatch.  The whole library is this
+// one translation unit; the kernels live in the included headers.
+#include "lsh.h"
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "attend_simt.cuh"
+#include "common.cuh"
+#include "hash_simt.cuh"
+#include "sort.cuh"
+
+namespace {
+
+using lsh::kHeadDim;
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxBuckets = 32768;
+constexpr int kMaxChunk = 64;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+inline bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u); }
+
+struct Dims {
+  int B, H, L, d, nb, R, c, causal, dtype;
+  size_t n_tok;  // B*H*L
+  bool empty;
+};
+
+lsh_status check_shape(const lsh_shape* s, Dims* o) {
+  if (!s) return LSH_ERR_INVALID_ARG;
+  if (s->B < 0 || s->H < 0 || s->L < 0 || s->d <= 0 || s->n_rounds < 1 || s->chunk < 1)
+    return LSH_ERR_INVALID_ARG;
+  if (s->n_buckets < 1 || (s->n_buckets > 1 && (s->n_buckets & 1))) return LSH_ERR_INVALID_ARG;
+  if (s->dtype != LSH_F32 && s->dtype != LSH_BF16) return LSH_ERR_INVALID_ARG;
+  o->B = s->B; o->H = s->H; o->L = s->L; o->d = s->d; o->nb = s->n_buckets;
+  o->R = s->n_rounds; o->c = s->chunk; o->causal = s->causal ? 1 : 0; o->dtype = s->dtype;
+  o->n_tok = (size_t)s->B * s->H * s->L;
+  o->empty = o->n_tok == 0;
+  if (!o->empty && s->L % s->chunk) return LSH_ERR_INVALID_ARG;
+  if (s->d != kHeadDim) return LSH_ERR_UNSUPPORTED;
+  if (s->n_buckets > kMaxBuckets) return LSH_ERR_UNSUPPORTED;
+  if (s->chunk > kMaxChunk) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)s->n_buckets * s->L >= (int64_t(1) << 31)) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)o->n_tok * s->n_rounds >= (int64_t(1) << 31)) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)s->n_rounds * s->B * s->H > 65535) return LSH_ERR_UNSUPPORTED;  // grid.y
+  return LSH_OK;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline lsh_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory.
+template <typename K>
+lsh_status allow_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return LSH_OK;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+                 cudaSuccess
+             ? LSH_OK
+             : LSH_ERR_CUDA;
+}
+
+size_t fwd_ws_bytes(const Dims& D) {
+  const size_t prev = (size_t)(D.R - 1) * D.n_tok;
+  return align_up(prev * kHeadDim * sizeof(float)) + align_up(prev * sizeof(float));
+}
+
+size_t bwd_ws_bytes(const Dims& D) {
+  return align_up(D.n_tok * sizeof(float)) + 3 * align_up(D.n_tok * kHeadDim * sizeof(float));
+}
+
+lsh::AttnDims attn_dims(const Dims& D) {
+  lsh::AttnDims a;
+  a.B = D.B; a.H = D.H; a.L = D.L; a.chunk = D.c; a.n_chunks = D.L / D.c;
+  a.causal = D.causal;
+  a.W = a.n_chunks > 1 ? 2 * D.c : D.c;
+  a.BH = D.B * D.H;
+  return a;
+}
+
+template <typename T>
+lsh_status hash_launch(const Dims& D, const void* Q, const void* rot, uint32_t* keys,
+                       int32_t* buckets, cudaStream_t st) {
+  constexpr int TOK = 128;
+  const int half = D.nb / 2;
+  const dim3 grid((unsigned)((D.n_tok + TOK - 1) / TOK), (unsigned)D.R);
+  lsh::hash_simt_kernel<T, TOK><<<grid, TOK, 0, st>>>(
+      static_cast<const T*>(Q), static_cast<const T*>(rot), keys, buckets, (int)D.n_tok, D.L, half);
+  return last_launch();
+}
+
+lsh_status sort_launch(const Dims& D, const uint32_t* keys, int32_t* perm, cudaStream_t st) {
+  const size_t budget = 200 * 1024;
+  int nwarps = (int)(budget / ((size_t)D.nb * sizeof(uint32_t)));
+  nwarps = nwarps > 32 ? 32 : nwarps;
+  const int by_len = (D.L + 127) / 128;  // at least 4 steps of 32 per warp
+  nwarps = nwarps > by_len ? by_len : nwarps;
+  if (nwarps < 1) nwarps = 1;
+  const size_t smem = (size_t)nwarps * D.nb * sizeof(uint32_t);
+  lsh_status st0 = allow_smem(lsh::sort_rows_kernel, smem);
+  if (st0 != LSH_OK) return st0;
+  const unsigned rows = (unsigned)((size_t)D.R * D.B * D.H);
+  lsh::sort_rows_kernel<<<rows, nwarps * 32, smem, st>>>(keys, perm, D.L, D.nb);
+  return last_launch();
+}
+
+template <typename T>
+lsh_status attend_fwd_launch(const Dims& D, const void* Q, const void* V, const uint32_t* keys,
+                             const int32_t* perm, float* o_part, float* lse_r, void* O, float* lse,
+                             void* ws, size_t ws_bytes, cudaStream_t st) {
+  const lsh::AttnDims a = attn_dims(D);
+  const size_t smem = lsh::simt_fwd_smem_bytes(a.chunk, a.W);
+  lsh_status s0 = allow_smem(lsh::attend_fwd_simt_kernel<T>, smem);
+  if (s0 != LSH_OK) return s0;
+  const T* q = static_cast<const T*>(Q);
+  const T* v = static_cast<const T*>(V);
+  if (!O) {
+    const dim3 grid((unsigned)a.n_chunks, (unsigned)(D.R * a.BH));
+    lsh::attend_fwd_simt_kernel<T><<<grid, 256, smem, st>>>(
+        q, v, keys, perm, a, 0, o_part, lse_r, 0, D.R, nullptr, nullptr, nullptr, nullptr);
+    return last_launch();
+  }
+  // partial buffers for rounds 0..R-2
+  float* po = o_part;
+  float* pl = lse_r;
+  if (D.R > 1 && (!po || !pl)) {
+    if (!ws || ws_bytes < fwd_ws_bytes(D)) return LSH_ERR_WORKSPACE;
+    char* w = static_cast<char*>(ws);
+    const size_t prev = (size_t)(D.R - 1) * D.n_tok;
+    if (!po) po = reinterpret_cast<float*>(w);
+    if (!pl) pl = reinterpret_cast<float*>(w + align_up(prev * kHeadDim * sizeof(float)));
+  }
+  if (D.R > 1) {
+    const dim3 grid((unsigned)a.n_chunks, (unsigned)((D.R - 1) * a.BH));
+    lsh::attend_fwd_simt_kernel<T><<<grid, 256, smem, st>>>(
+        q, v, keys, perm, a, 0, po, pl, 0, D.R, nullptr, nullptr, nullptr, nullptr);
+    if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)a.n_chunks, (unsigned)a.BH);
+  lsh::attend_fwd_simt_kernel<T><<<grid, 256, smem, st>>>(
+      q, v, keys, perm, a, D.R - 1, o_part, lse_r, 1, D.R, po, pl, static_cast<T*>(O), lse);
+  return last_launch();
+}
+
+template <typename T>
+lsh_status combine_launch(const Dims& D, const float* o_part, const float* lse_r, void* O,
+                          float* lse, cudaStream_t st) {
+  const size_t n = D.n_tok * 8;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  lsh::combine_kernel<T><<<blocks, 256, 0, st>>>(o_part, lse_r, D.R, D.n_tok,
+                                                 static_cast<T*>(O), lse);
+  return last_launch();
+}
+
+template <typename T>
+lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const void* O,
+                             const void* dO, const uint32_t* keys, const int32_t* perm,
+                             const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,
+                             cudaStream_t st) {
+  if (!ws || ws_bytes < bwd_ws_bytes(D)) return LSH_ERR_WORKSPACE;
+  const lsh::AttnDims a = attn_dims(D);
+  char* w = static_cast<char*>(ws);
+  float* G = reinterpret_cast<float*>(w);
+  const size_t acc_bytes = align_up(D.n_tok * kHeadDim * sizeof(float));
+  float* dq = reinterpret_cast<float*>(w + align_up(D.n_tok * sizeof(float)));
+  float* dk = reinterpret_cast<float*>(reinterpret_cast<char*>(dq) + acc_bytes);
+  float* dv = reinterpret_cast<float*>(reinterpret_cast<char*>(dk) + acc_bytes);
+  if (cudaMemsetAsync(dq, 0, 3 * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
+  const T* q = static_cast<const T*>(Q);
+  const unsigned tb = (unsigned)((D.n_tok + 255) / 256);
+  lsh::bwd_dot_kernel<T><<<tb, 256, 0, st>>>(static_cast<const T*>(O), static_cast<const T*>(dO),
+                                             D.n_tok, G);
+  if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+  const size_t smem = lsh::simt_bwd_smem_bytes(a.chunk, a.W);
+  lsh_status s0 = allow_smem(lsh::attend_bwd_simt_kernel<T>, smem);
+  if (s0 != LSH_OK) return s0;
+  const dim3 grid((unsigned)a.n_chunks, (unsigned)(D.R * a.BH));
+  lsh::attend_bwd_simt_kernel<T><<<grid, 256, smem, st>>>(
+      q, static_cast<const T*>(V), static_cast<const T*>(dO), keys, perm, lse, G, a, dq, dk, dv);
+  if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+  lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok, static_cast<T*>(dQ),
+                                                  static_cast<T*>(dV));
+  return last_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lsh_workspace_size(const lsh_shape* shape) {
+  Dims D;
+  if (check_shape(shape, &D) != LSH_OK || D.empty) return 0;
+  const size_t f = fwd_ws_bytes(D), b = bwd_ws_bytes(D);
+  return f > b ? f : b;
+}
+
+lsh_status lsh_hash(const lsh_shape* shape, const void* Q, const void* rot, uint32_t* keys,
+                    int32_t* buckets, void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Q || !keys || (D.nb > 1 && !rot)) return LSH_ERR_INVALID_ARG;
+  if (misaligned(Q) || misaligned(rot) || misaligned(keys) || misaligned(buckets))
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D.dtype == LSH_BF16 ? hash_launch<__nv_bfloat16>(D, Q, rot, keys, buckets, st)
+                             : hash_launch<float>(D, Q, rot, keys, buckets, st);
+}
+
+lsh_status lsh_sort(const lsh_shape* shape, const uint32_t* keys, int32_t* perm, void* ws,
+                    size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!keys || !perm || misaligned(keys) || misaligned(perm)) return LSH_ERR_INVALID_ARG;
+  return sort_launch(D, keys, perm, as_stream(stream));
+}
+
+lsh_status lsh_attend_fwd(const lsh_shape* shape, const void* Q, const void* V,
+                          const uint32_t* keys, const int32_t* perm, float* o_part, float* lse_r,
+                          void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Q || !V || !keys || !perm) return LSH_ERR_INVALID_ARG;
+  if (!O && (!o_part || !lse_r)) return LSH_ERR_INVALID_ARG;
+  if (misaligned(Q) || misaligned(V) || misaligned(keys) || misaligned(perm) ||
+      misaligned(o_part) || misaligned(lse_r) || misaligned(O) || misaligned(lse) ||
+      misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D.dtype == LSH_BF16
+             ? attend_fwd_launch<__nv_bfloat16>(D, Q, V, keys, perm, o_part, lse_r, O, lse, ws,
+                                                ws_bytes, st)
+             : attend_fwd_launch<float>(D, Q, V, keys, perm, o_part, lse_r, O, lse, ws, ws_bytes,
+                                        st);
+}
+
+lsh_status lsh_combine(const lsh_shape* shape, const float* o_part, const float* lse_r, void* O,
+                       float* lse, void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!o_part || !lse_r || !O) return LSH_ERR_INVALID_ARG;
+  if (misaligned(o_part) || misaligned(lse_r) || misaligned(O) || misaligned(lse))
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D.dtype == LSH_BF16 ? combine_launch<__nv_bfloat16>(D, o_part, lse_r, O, lse, st)
+                             : combine_launch<float>(D, o_part, lse_r, O, lse, st);
+}
+
+lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void* V, const void* rot,
+                       uint32_t* keys, int32_t* buckets, int32_t* perm, void* O, float* lse,
+                       void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!O || !lse || !perm) return LSH_ERR_INVALID_ARG;
+  s = lsh_hash(shape, Q, rot, keys, buckets, stream);
+  if (s != LSH_OK) return s;
+  s = lsh_sort(shape, keys, perm, ws, ws_bytes, stream);
+  if (s != LSH_OK) return s;
+  return lsh_attend_fwd(shape, Q, V, keys, perm, nullptr, nullptr, O, lse, ws, ws_bytes, stream);
+}
+
+lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const void* V, const void* O,
+                          const void* dO, const uint32_t* keys, const int32_t* perm,
+                          const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Q || !V || !O || !dO || !keys || !perm || !lse || !dQ || !dV) return LSH_ERR_INVALID_ARG;
+  if (misaligned(Q) || misaligned(V) || misaligned(O) || misaligned(dO) || misaligned(keys) ||
+      misaligned(perm) || misaligned(lse) || misaligned(dQ) || misaligned(dV) || misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D.dtype == LSH_BF16
+             ? attend_bwd_launch<__nv_bfloat16>(D, Q, V, O, dO, keys, perm, lse, dQ, dV, ws,
+                                                ws_bytes, st)
+             : attend_bwd_launch<float>(D, Q, V, O, dO, keys, perm, lse, dQ, dV, ws, ws_bytes,
+                                        st);
+}
+
+lsh_status lsh_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return LSH_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lsh::g_status, sizeof(int)) != cudaSuccess) return LSH_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(lsh::g_status, &zero, sizeof(int)) != cudaSuccess) return LSH_ERR_CUDA;
+  return static_cast<lsh_status>(v);
+}
+
+const char* lsh_status_string(lsh_status status) {
+  switch (status) {
+    case LSH_OK: return "ok";
+    case LSH_ERR_INVALID_ARG: return "invalid argument";
+    case LSH_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case LSH_ERR_CUDA: return "CUDA error";
+    case LSH_ERR_WORKSPACE: return "workspace missing or too small";
+    case LSH_ERR_TIMEOUT: return "device wait timed out";
+    case LSH_ERR_BAD_KEYS: return "keys are not bucket*L + position";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

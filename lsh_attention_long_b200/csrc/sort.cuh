@@ -1,0 +1,113 @@
+// Per-row stable counting sort of packed LSH keys.
+//
+// "Reformer explainer" (akshathtiwari.co.in/blog/reformer): after hashing,
+// tokens are sorted by bucket.  Within every (round, batch, head) row the
+// order is (bucket, position); since a row's keys arrive in position order,
+// a stable counting sort on the bucket produces it.
+//
+// One CTA per row.  Each warp owns a contiguous segment of the row and a
+// private histogram in shared memory, so counting needs no atomics:
+//   pass 1  per 32-token step, __match_any_sync groups equal buckets and the
+//           group leader adds the group size to the warp's histogram;
+//   scan    bucket-major, warp-minor exclusive prefix sums turn the
+//           histograms into each warp's first output slot per bucket;
+//   pass 2  the same walk again; a token's slot is its warp's offset for the
+//           bucket plus its rank among equal-bucket lanes of lower index.
+// Warps, steps and lanes visit positions in increasing order, so equal
+// buckets keep position order: the sort is stable.
+#pragma once
+
+#include "common.cuh"
+
+namespace lsh {
+
+constexpr uint32_t kNoBucket = 0xffffffffu;
+
+__device__ __forceinline__ uint32_t checked_bucket(const uint32_t* k, int t, int L, int nb,
+                                                   bool& bad) {
+  const uint32_t key = k[t];
+  const uint32_t b = key / (uint32_t)L;
+  if (b >= (uint32_t)nb || key - b * (uint32_t)L != (uint32_t)t) {
+    bad = true;
+    return kNoBucket;
+  }
+  return b;
+}
+
+__global__ void __launch_bounds__(1024)
+sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, int L, int nb) {
+  extern __shared__ uint32_t cnt[];  // [nwarps][nb]
+  __shared__ uint32_t warp_sums[32];
+  const int nwarps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t* k = keys + (size_t)blockIdx.x * L;
+  int32_t* out = perm + (size_t)blockIdx.x * L;
+
+  for (int e = threadIdx.x; e < nwarps * nb; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+
+  const int seg = (((L + nwarps - 1) / nwarps) + 31) & ~31;
+  const int begin = min(L, w * seg), end = min(L, begin + seg);
+  uint32_t* my = cnt + (size_t)w * nb;
+  bool bad = false;
+
+  // pass 1: per-warp histograms
+  for (int base = begin; base < end; base += 32) {
+    const int t = base + lane;
+    const uint32_t b = (t < end) ? checked_bucket(k, t, L, nb, bad) : kNoBucket;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    if (b != kNoBucket && lane == __ffs(peers) - 1) my[b] += __popc(peers);
+  }
+  if (bad) record_status(kErrBadKeys);
+  __syncthreads();
+
+  // scan: each thread owns a contiguous run of buckets
+  const int per = (nb + blockDim.x - 1) / blockDim.x;
+  const int b0 = min(nb, threadIdx.x * per), b1 = min(nb, b0 + per);
+  uint32_t local = 0;
+  for (int b = b0; b < b1; ++b)
+    for (int ww = 0; ww < nwarps; ++ww) local += cnt[ww * nb + b];
+  uint32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    uint32_t v = lane < nwarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += x;
+    }
+    if (lane < nwarps) warp_sums[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  uint32_t running = incl - local + (w > 0 ? warp_sums[w - 1] : 0);
+  for (int b = b0; b < b1; ++b)
+    for (int ww = 0; ww < nwarps; ++ww) {
+      const uint32_t c = cnt[ww * nb + b];
+      cnt[ww * nb + b] = running;
+      running += c;
+    }
+  __syncthreads();
+
+  // pass 2: stable scatter of positions
+  for (int base = begin; base < end; base += 32) {
+    const int t = base + lane;
+    bool dummy = false;
+    const uint32_t b = (t < end) ? checked_bucket(k, t, L, nb, dummy) : kNoBucket;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    if (b != kNoBucket) {
+      const uint32_t rank = __popc(peers & ((1u << lane) - 1u));
+      out[my[b] + rank] = t;
+    }
+    __syncwarp();
+    if (b != kNoBucket && lane == __ffs(peers) - 1) my[b] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+}  // namespace lsh

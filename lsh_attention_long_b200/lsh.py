@@ -1,0 +1,227 @@
+"""Python binding of the C ABI in include/lsh.h (argument marshalling only).
+
+Every function here checks tensor shapes, allocates missing outputs with
+torch on the inputs' device, and calls the same-named entry point of
+``liblsh.so`` through ctypes on the current CUDA stream.  All arithmetic runs
+in the library's CUDA kernels; there is no CPU path.  Importing works without
+a GPU, and a missing library raises instead of falling back.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsh.so")
+
+LSH_F32, LSH_BF16 = 0, 1
+STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "LSH_ERR_CUDA",
+          4: "LSH_ERR_WORKSPACE", 5: "LSH_ERR_TIMEOUT", 6: "LSH_ERR_BAD_KEYS"}
+
+EXPORTS = ("lsh_workspace_size", "lsh_hash", "lsh_sort", "lsh_attend_fwd", "lsh_combine",
+           "lsh_forward", "lsh_attend_bwd", "lsh_device_status", "lsh_status_string")
+
+
+class LshError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "L", "d", "n_buckets", "n_rounds", "chunk", "causal", "dtype")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblsh.so (built by ``python -m lsh_attention_long_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing; build it with "
+                           "`python -m lsh_attention_long_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, S = ctypes.c_void_p, ctypes.POINTER(Shape)
+    sz = ctypes.c_size_t
+    sig = {
+        "lsh_workspace_size": ([S], sz),
+        "lsh_hash": ([S, P, P, P, P, P], ctypes.c_int),
+        "lsh_sort": ([S, P, P, P, sz, P], ctypes.c_int),
+        "lsh_attend_fwd": ([S, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "lsh_combine": ([S, P, P, P, P, P], ctypes.c_int),
+        "lsh_forward": ([S, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "lsh_attend_bwd": ([S, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "lsh_device_status": ([P], ctypes.c_int),
+        "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return LSH_F32
+    if t == torch.bfloat16:
+        return LSH_BF16
+    raise TypeError(f"unsupported dtype {t}; use float32 or bfloat16")
+
+
+def make_shape(B, H, L, d, n_buckets, n_rounds, chunk, causal, dtype: torch.dtype) -> Shape:
+    return Shape(B, H, L, d, n_buckets, n_rounds, chunk, int(bool(causal)), _dtype_code(dtype))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the LSH library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _call(name: str, *args):
+    rc = getattr(load_library(), name)(*args)
+    if rc != 0:
+        raise LshError(name, rc)
+
+
+def _qshape(Q: torch.Tensor):
+    if Q.dim() != 4:
+        raise ValueError("Q must be [B, H, L, d]")
+    return tuple(Q.shape)
+
+
+def lsh_workspace_size(shape: Shape) -> int:
+    return int(load_library().lsh_workspace_size(ctypes.byref(shape)))
+
+
+def workspace(shape: Shape, device) -> torch.Tensor:
+    """A byte tensor large enough for any call on this shape."""
+    return torch.empty(max(lsh_workspace_size(shape), 16), dtype=torch.uint8, device=device)
+
+
+def lsh_hash(Q, rot, n_buckets: int, *, keys=None, buckets=None, want_buckets=True, stream=None):
+    """Step 1: keys [R,B,H,L] u32 (as int32 storage) and bucket ids [R,B,H,L] i32."""
+    B, H, L, d = _qshape(Q)
+    R = rot.shape[0]
+    shape = make_shape(B, H, L, d, n_buckets, R, 1, False, Q.dtype)
+    if keys is None:
+        keys = torch.empty((R, B, H, L), dtype=torch.int32, device=Q.device)
+    if buckets is None and want_buckets:
+        buckets = torch.empty((R, B, H, L), dtype=torch.int32, device=Q.device)
+    _call("lsh_hash", ctypes.byref(shape), _ptr(Q), _ptr(rot) if n_buckets > 1 else None,
+          _ptr(keys), _ptr(buckets), _stream(stream))
+    return keys, buckets
+
+
+def lsh_sort(keys, n_buckets: int, *, perm=None, stream=None):
+    """Step 2: perm [R,B,H,L] i32 (original position at each sorted slot)."""
+    R, B, H, L = keys.shape
+    shape = make_shape(B, H, L, 64, n_buckets, R, 1, False, torch.float32)
+    if perm is None:
+        perm = torch.empty_like(keys, dtype=torch.int32)
+    _call("lsh_sort", ctypes.byref(shape), _ptr(keys), _ptr(perm), None, 0, _stream(stream))
+    return perm
+
+
+def lsh_attend_fwd(Q, V, keys, perm, n_buckets: int, chunk: int, causal: bool, *,
+                   o_part=None, lse_r=None, O=None, lse=None, combine=True, ws=None,
+                   stream=None):
+    """Steps 3-5.  Returns (O, lse, o_part, lse_r); O/lse are None when combine=False."""
+    B, H, L, d = _qshape(Q)
+    R = keys.shape[0]
+    shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    if combine:
+        if O is None:
+            O = torch.empty_like(Q)
+        if lse is None:
+            lse = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
+        if ws is None and (o_part is None or lse_r is None):
+            ws = workspace(shape, Q.device)
+    else:
+        if o_part is None:
+            o_part = torch.empty((R, B, H, L, d), dtype=torch.float32, device=Q.device)
+        if lse_r is None:
+            lse_r = torch.empty((R, B, H, L), dtype=torch.float32, device=Q.device)
+    _call("lsh_attend_fwd", ctypes.byref(shape), _ptr(Q), _ptr(V), _ptr(keys), _ptr(perm),
+          _ptr(o_part), _ptr(lse_r), _ptr(O) if combine else None,
+          _ptr(lse) if combine else None, _ptr(ws), 0 if ws is None else ws.numel(),
+          _stream(stream))
+    return O, lse, o_part, lse_r
+
+
+def lsh_combine(o_part, lse_r, dtype: torch.dtype, *, O=None, lse=None, stream=None):
+    """Step 5 alone: O [B,H,L,d] in dtype and lse [B,H,L] fp32."""
+    R, B, H, L, d = o_part.shape
+    shape = make_shape(B, H, L, d, 2, R, 1, False, dtype)
+    if O is None:
+        O = torch.empty((B, H, L, d), dtype=dtype, device=o_part.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=o_part.device)
+    _call("lsh_combine", ctypes.byref(shape), _ptr(o_part), _ptr(lse_r), _ptr(O), _ptr(lse),
+          _stream(stream))
+    return O, lse
+
+
+def lsh_forward(Q, V, rot, n_buckets: int, chunk: int, causal: bool, *, out=None, ws=None,
+                want_buckets=False, stream=None) -> Dict[str, torch.Tensor]:
+    """Whole forward (hash -> sort -> attend with fused combine) in one C call.
+
+    ``out`` may hold preallocated tensors under the keys returned."""
+    B, H, L, d = _qshape(Q)
+    R = rot.shape[0]
+    shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    o = dict(out or {})
+    dev = Q.device
+    o.setdefault("keys", torch.empty((R, B, H, L), dtype=torch.int32, device=dev))
+    o.setdefault("perm", torch.empty((R, B, H, L), dtype=torch.int32, device=dev))
+    o.setdefault("O", torch.empty_like(Q))
+    o.setdefault("lse", torch.empty((B, H, L), dtype=torch.float32, device=dev))
+    if want_buckets:
+        o.setdefault("buckets", torch.empty((R, B, H, L), dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(shape, dev)
+    _call("lsh_forward", ctypes.byref(shape), _ptr(Q), _ptr(V),
+          _ptr(rot) if n_buckets > 1 else None, _ptr(o["keys"]), _ptr(o.get("buckets")),
+          _ptr(o["perm"]), _ptr(o["O"]), _ptr(o["lse"]), _ptr(ws), ws.numel(), _stream(stream))
+    return o
+
+
+def lsh_attend_bwd(Q, V, O, dO, keys, perm, lse, n_buckets: int, chunk: int, causal: bool, *,
+                   dQ=None, dV=None, ws=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Backward with buckets frozen: (dQ, dV) in Q's dtype."""
+    B, H, L, d = _qshape(Q)
+    R = keys.shape[0]
+    shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    if dQ is None:
+        dQ = torch.empty_like(Q)
+    if dV is None:
+        dV = torch.empty_like(V)
+    if ws is None:
+        ws = workspace(shape, Q.device)
+    _call("lsh_attend_bwd", ctypes.byref(shape), _ptr(Q), _ptr(V), _ptr(O), _ptr(dO),
+          _ptr(keys), _ptr(perm), _ptr(lse), _ptr(dQ), _ptr(dV), _ptr(ws), ws.numel(),
+          _stream(stream))
+    return dQ, dV
+
+
+def lsh_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the first device-side error code."""
+    return int(load_library().lsh_device_status(_stream(stream)))

@@ -132,12 +132,17 @@ int oracle_lsh_sort(int rows, int L, const uint32_t* keys, int32_t* perm) {
 // Steps 3-4 -- chunked shared-QK attention for every round, scattered back to
 // original positions.  o_part is [R, B, H, L, d], lse_r is [R, B, H, L].
 // The bucket of position j in row (r, b, h) is keys[r,b,h,j] / L.
-int oracle_lsh_attend_fwd(int B, int H, int L, int d, int n_rounds, int chunk, int causal,
-                          const double* Q, const double* V, const uint32_t* keys,
-                          const int32_t* perm, double* o_part, double* lse_r) {
+// Only the queries of chunks [chunk_begin, chunk_end) of every row are
+// computed (their outputs land at those queries' positions); the plain
+// entry point below takes every chunk.
+int oracle_lsh_attend_fwd_range(int B, int H, int L, int d, int n_rounds, int chunk, int causal,
+                                const double* Q, const double* V, const uint32_t* keys,
+                                const int32_t* perm, int chunk_begin, int chunk_end,
+                                double* o_part, double* lse_r) {
   if (B < 0 || H < 0 || L < 0 || d <= 0 || n_rounds < 0 || chunk <= 0) return 1;
   if (L % chunk != 0) return 1;
   const int n_chunks = L / chunk;
+  if (chunk_begin < 0 || chunk_end > n_chunks || chunk_begin > chunk_end) return 1;
   const double scale = 1.0 / std::sqrt((double)d);
   const double neg_inf = -std::numeric_limits<double>::infinity();
   std::vector<double> khat((size_t)L * d);
@@ -159,7 +164,7 @@ int oracle_lsh_attend_fwd(int B, int H, int L, int d, int n_rounds, int chunk, i
           for (int k = 0; k < d; ++k)
             khat[(size_t)j * d + k] = nrm > 0.0 ? q[(size_t)j * d + k] / nrm : 0.0;
         }
-        for (int c = 0; c < n_chunks; ++c) {
+        for (int c = chunk_begin; c < chunk_end; ++c) {
           // window: the previous chunk (wrapping) then this chunk; one chunk
           // only once when the row is a single chunk
           int nw = 0;
@@ -205,6 +210,14 @@ int oracle_lsh_attend_fwd(int B, int H, int L, int d, int n_rounds, int chunk, i
         }
       }
   return 0;
+}
+
+int oracle_lsh_attend_fwd(int B, int H, int L, int d, int n_rounds, int chunk, int causal,
+                          const double* Q, const double* V, const uint32_t* keys,
+                          const int32_t* perm, double* o_part, double* lse_r) {
+  if (chunk <= 0 || L < 0) return 1;
+  return oracle_lsh_attend_fwd_range(B, H, L, d, n_rounds, chunk, causal, Q, V, keys, perm, 0,
+                                     L / chunk, o_part, lse_r);
 }
 
 // Step 5 -- combine rounds: lse = logsumexp_r lse_r, o = sum_r exp(lse_r - lse) o_r.

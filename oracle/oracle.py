@@ -45,9 +45,11 @@ def _load():
         lib.oracle_lsh_hash.argtypes = [I, I, I, I, I, I, P, P, P, P, P]
         lib.oracle_lsh_sort.argtypes = [I, I, P, P]
         lib.oracle_lsh_attend_fwd.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P]
+        lib.oracle_lsh_attend_fwd_range.argtypes = [I, I, I, I, I, I, I, P, P, P, P, I, I, P, P]
         lib.oracle_lsh_combine.argtypes = [I, I, I, I, I, P, P, P, P]
         lib.oracle_lsh_attend_bwd.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P]
         for f in (lib.oracle_lsh_hash, lib.oracle_lsh_sort, lib.oracle_lsh_attend_fwd,
+                  lib.oracle_lsh_attend_fwd_range,
                   lib.oracle_lsh_combine, lib.oracle_lsh_attend_bwd):
             f.restype = ctypes.c_int
         _lib = lib
@@ -105,6 +107,25 @@ def lsh_attend_fwd(Q, V, keys, perm, chunk: int, causal: bool):
     rc = _load().oracle_lsh_attend_fwd(B, H, L, d, R, chunk, int(bool(causal)), _ptr(Q), _ptr(V),
                                        _ptr(keys), _ptr(perm), _ptr(o_part), _ptr(lse_r))
     _check(rc, "oracle_lsh_attend_fwd")
+    return o_part, lse_r
+
+
+def lsh_attend_fwd_range(Q, V, keys, perm, chunk: int, causal: bool, chunk_begin: int,
+                         chunk_end: int):
+    """lsh_attend_fwd restricted to the queries of chunks [chunk_begin, chunk_end)
+    of every row; other positions of the outputs stay zero."""
+    Q = _f64(Q)
+    V = _f64(V)
+    keys = np.ascontiguousarray(keys, dtype=np.uint32)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    B, H, L, d = Q.shape
+    R = keys.shape[0]
+    o_part = np.zeros((R, B, H, L, d))
+    lse_r = np.zeros((R, B, H, L))
+    rc = _load().oracle_lsh_attend_fwd_range(B, H, L, d, R, chunk, int(bool(causal)), _ptr(Q),
+                                             _ptr(V), _ptr(keys), _ptr(perm), chunk_begin,
+                                             chunk_end, _ptr(o_part), _ptr(lse_r))
+    _check(rc, "oracle_lsh_attend_fwd_range")
     return o_part, lse_r
 
 

@@ -1,0 +1,234 @@
+"""GPU parity: every step of the CUDA path against the fp64 CPU oracle.
+
+Bit-exact for integers (bucket ids away from near ties, keys, permutations);
+max-abs 2e-3 (f32 inputs) or 2e-2 (bf16 inputs, fp32 accumulation) for
+outputs, logsumexps and gradients.  The oracle is fed the GPU's own keys and
+permutations so that a legitimate near-tie flip cannot cause a tolerance
+failure; near ties (top two rotated projections within 1e-5 relative) are
+counted and reported.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import lsh_attention_long_b200 as L
+from lsh_attention_long_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 2e-3, torch.bfloat16: 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from lsh_attention_long_b200 import build
+    build.build()
+    L.load_library()
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def _check_status():
+    assert L.lsh_device_status() == 0
+
+
+def check_hash(oracle, Q, rot, nb, keys, buckets, sample=None):
+    """Bucket ids bit-exact except near ties; keys = bucket*L + position."""
+    Qn = _np(Q)
+    Ln = Q.shape[2]
+    kb = buckets.cpu().numpy()
+    kk = keys.cpu().numpy().view(np.uint32)
+    pos = np.arange(Ln, dtype=np.uint64)
+    assert np.array_equal(kk.astype(np.uint64), kb.astype(np.uint64) * Ln + pos)
+    if sample is not None:
+        flat = Qn.reshape(-1, Qn.shape[-1])
+        idx = np.random.default_rng(0).choice(flat.shape[0], size=min(sample, flat.shape[0]),
+                                              replace=False)
+        _, ob, tie = oracle.lsh_hash(flat[idx][None, None], _np(rot), nb)
+        gb = kb.reshape(kb.shape[0], -1)[:, idx]
+        ob, tie = ob[:, 0, 0], tie[:, 0, 0]
+    else:
+        _, ob, tie = oracle.lsh_hash(Qn, _np(rot), nb)
+        gb = kb
+    bad = (gb != ob) & (tie == 0)
+    assert not bad.any(), f"{int(bad.sum())} bucket mismatches outside near ties"
+    return int(tie.sum())
+
+
+def run_steps(inp, nb, chunk, causal):
+    Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
+    keys, buckets = L.lsh_hash(Q, rot, nb)
+    perm = L.lsh_sort(keys, nb)
+    _, _, o_part, lse_r = L.lsh_attend_fwd(Q, V, keys, perm, nb, chunk, causal, combine=False)
+    O, lse, _, _ = L.lsh_attend_fwd(Q, V, keys, perm, nb, chunk, causal)
+    torch.cuda.synchronize()
+    _check_status()
+    return dict(Q=Q, V=V, rot=rot, keys=keys, buckets=buckets, perm=perm, o_part=o_part,
+                lse_r=lse_r, O=O, lse=lse)
+
+
+def check_all(oracle, inp, nb, chunk, causal, heads=None):
+    g = run_steps(inp, nb, chunk, causal)
+    tol = TOL[inp["Q"].dtype]
+    check_hash(oracle, g["Q"], g["rot"], nb, g["keys"], g["buckets"])
+    keys_np = g["keys"].cpu().numpy().view(np.uint32)
+    assert np.array_equal(g["perm"].cpu().numpy(), oracle.lsh_sort(keys_np))
+    Qn, Vn = _np(g["Q"]), _np(g["V"])
+    perm_np = g["perm"].cpu().numpy()
+    if heads is not None:  # restrict the attention comparison to some (b, h)
+        b, h = heads
+        Qn, Vn = Qn[b:b + 1, h:h + 1], Vn[b:b + 1, h:h + 1]
+        keys_np = keys_np[:, b:b + 1, h:h + 1]
+        perm_np = perm_np[:, b:b + 1, h:h + 1]
+        sl = (slice(b, b + 1), slice(h, h + 1))
+    else:
+        sl = (slice(None), slice(None))
+    o_part, lse_r = oracle.lsh_attend_fwd(Qn, Vn, keys_np, perm_np, chunk, causal)
+    O, lse = oracle.lsh_combine(o_part, lse_r)
+    np.testing.assert_allclose(_np(g["o_part"])[:, sl[0], sl[1]], o_part, rtol=0, atol=tol)
+    np.testing.assert_allclose(_np(g["lse_r"])[:, sl[0], sl[1]], lse_r, rtol=1e-6, atol=tol)
+    np.testing.assert_allclose(_np(g["O"])[sl], O, rtol=0, atol=tol)
+    np.testing.assert_allclose(_np(g["lse"])[sl], lse, rtol=1e-6, atol=tol)
+    # standalone combine of the GPU partials equals the fused epilogue
+    Oc, lsec = L.lsh_combine(g["o_part"], g["lse_r"], g["Q"].dtype)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(_np(Oc), _np(g["O"]), rtol=0, atol=tol / 4)
+    np.testing.assert_allclose(_np(lsec), _np(g["lse"]), rtol=1e-6, atol=1e-5)
+    return g
+
+
+CASES = [
+    # B, H, L, nb, R, chunk, causal
+    (1, 3, 320, 16, 2, 64, True),     # 5 chunks (odd), ragged hash tiles
+    (2, 1, 96, 6, 3, 32, False),      # nb/2 = 3, three chunks
+    (1, 2, 64, 8, 2, 64, True),       # one chunk: window is the chunk once
+    (1, 2, 128, 4, 2, 64, False),     # two chunks: each sees the whole row
+    (1, 1, 256, 1, 2, 64, True),      # one bucket
+    (1, 2, 256, 2, 3, 16, False),     # hyperplane hash, small chunks
+    (1, 1, 256, 1024, 1, 64, False),  # more buckets than tokens: lone tokens
+    (1, 2, 64, 4, 1, 4, True),        # tiny chunks
+    (1, 1, 512, 32768, 1, 64, True),  # the largest bucket count
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,Lx,nb,R,chunk,causal", CASES)
+def test_small_shapes(oracle, dtype, B, H, Lx, nb, R, chunk, causal):
+    inp = W.make_random(B, H, Lx, 64, nb, R, dtype, seed=Lx + nb + R)
+    check_all(oracle, inp, nb, chunk, causal)
+
+
+def test_workload_fwd_f32_L1024(oracle):
+    w = W.WORKLOADS["fwd_f32_L1024"]
+    check_all(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal)
+
+
+@pytest.mark.parametrize("name,head", [("fwd_bf16_L4096", (5, 3)),
+                                       ("fwd_bf16_L16384_clustered", (1, 6))])
+def test_workload_bf16(oracle, name, head):
+    w = W.WORKLOADS[name]
+    check_all(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal, heads=head)
+
+
+def test_workload_L65536_as_benchmarked(oracle):
+    """The benchmarked forward (one lsh_forward call) at full size; hash on a
+    sample of tokens, sort on every row, attention on one sampled head."""
+    w = W.WORKLOADS["fwd_bf16_L65536"]
+    inp = W.make_inputs(w)
+    Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
+    out = L.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal, want_buckets=True)
+    torch.cuda.synchronize()
+    _check_status()
+    ties = check_hash(oracle, Q, rot, w.n_buckets, out["keys"], out["buckets"], sample=4096)
+    keys_np = out["keys"].cpu().numpy().view(np.uint32)
+    assert np.array_equal(out["perm"].cpu().numpy(), oracle.lsh_sort(keys_np))
+    h = 3
+    o_part, lse_r = oracle.lsh_attend_fwd(_np(Q)[:, h:h + 1], _np(V)[:, h:h + 1],
+                                          keys_np[:, :, h:h + 1],
+                                          out["perm"].cpu().numpy()[:, :, h:h + 1],
+                                          w.chunk, w.causal)
+    O, lse = oracle.lsh_combine(o_part, lse_r)
+    np.testing.assert_allclose(_np(out["O"])[:, h:h + 1], O, rtol=0, atol=2e-2)
+    np.testing.assert_allclose(_np(out["lse"])[:, h:h + 1], lse, rtol=1e-6, atol=2e-2)
+    print(f"near ties in the 4096-token sample: {ties}")
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def check_bwd(oracle, inp, nb, chunk, causal, heads=None):
+    dtype = inp["Q"].dtype
+    Q, V, rot, dO = (inp[k].cuda() for k in ("Q", "V", "rot", "dO"))
+    out = L.lsh_forward(Q, V, rot, nb, chunk, causal)
+    dQ, dV = L.lsh_attend_bwd(Q, V, out["O"], dO, out["keys"], out["perm"], out["lse"], nb,
+                              chunk, causal)
+    torch.cuda.synchronize()
+    _check_status()
+    keys_np = out["keys"].cpu().numpy().view(np.uint32)
+    perm_np = out["perm"].cpu().numpy()
+    Qn, Vn, dOn = _np(Q), _np(V), _np(dO)
+    gQ, gV = _np(dQ), _np(dV)
+    if heads is not None:
+        b, h = heads
+        Qn, Vn, dOn = (x[b:b + 1, h:h + 1] for x in (Qn, Vn, dOn))
+        keys_np, perm_np = keys_np[:, b:b + 1, h:h + 1], perm_np[:, b:b + 1, h:h + 1]
+        gQ, gV = gQ[b:b + 1, h:h + 1], gV[b:b + 1, h:h + 1]
+    rQ, rV = oracle.lsh_attend_bwd(Qn, Vn, dOn, keys_np, perm_np, chunk, causal)
+    tol = TOL[dtype]
+    np.testing.assert_allclose(gV, rV, rtol=0, atol=tol)
+    np.testing.assert_allclose(gQ, rQ, rtol=0, atol=tol)
+
+
+BWD_CASES = [
+    (1, 3, 320, 16, 2, 64, True),
+    (2, 1, 96, 6, 3, 32, False),
+    (1, 2, 64, 8, 2, 64, True),
+    (1, 2, 128, 4, 2, 64, False),
+    (1, 1, 256, 1, 2, 64, True),
+    (1, 1, 256, 1024, 2, 64, False),
+    (1, 2, 64, 4, 1, 4, True),
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,Lx,nb,R,chunk,causal", BWD_CASES)
+def test_backward_small_shapes(oracle, dtype, B, H, Lx, nb, R, chunk, causal):
+    inp = W.make_random(B, H, Lx, 64, nb, R, dtype, seed=7 * Lx + nb, backward=True)
+    check_bwd(oracle, inp, nb, chunk, causal)
+
+
+def test_backward_workload_L16384(oracle):
+    w = W.WORKLOADS["fwdbwd_bf16_L16384"]
+    check_bwd(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal, heads=(1, 2))
+
+
+# ---------------------------------------------------------------------------
+# edge cases of the ABI on the device
+# ---------------------------------------------------------------------------
+
+def test_malformed_keys_are_reported():
+    """Keys that are not bucket*L + position (here two rows swapped) are
+    detected by the sort kernel's own check; every access stays in bounds."""
+    inp = W.make_random(1, 1, 256, 64, 16, 1, torch.bfloat16, seed=3)
+    Q, rot = inp["Q"].cuda(), inp["rot"].cuda()
+    keys, _ = L.lsh_hash(Q, rot, 16)
+    bad = keys.clone()
+    bad[0, 0, 0, 0], bad[0, 0, 0, 1] = keys[0, 0, 0, 1], keys[0, 0, 0, 0]
+    L.lsh_sort(bad, 16)
+    assert L.lsh_device_status() == 6
+    L.lsh_sort(keys, 16)
+    assert L.lsh_device_status() == 0
+
+
+def test_empty_batch_is_a_no_op():
+    Q = torch.empty((0, 2, 64, 64), dtype=torch.bfloat16, device="cuda")
+    rot = torch.randn(1, 64, 4, device="cuda").to(torch.bfloat16)
+    out = L.lsh_forward(Q, Q, rot, 8, 64, True)
+    assert out["O"].numel() == 0
+    assert L.lsh_device_status() == 0

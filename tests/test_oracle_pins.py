@@ -361,3 +361,23 @@ def test_backward_one_bucket_matches_autograd(oracle, causal):
     (o * torch.from_numpy(dO)).sum().backward()
     np.testing.assert_allclose(dQ, q.grad.numpy(), rtol=0, atol=1e-10)
     np.testing.assert_allclose(dV, v.grad.numpy(), rtol=0, atol=1e-10)
+
+
+def test_chunk_range_restricts_the_full_computation(oracle):
+    """The chunk-range entry point (used to time bounded samples) computes the
+    same values as the full call on the queries of those chunks, nothing else."""
+    rng = _rng(31)
+    Q = rng.standard_normal((1, 2, 128, 16))
+    V = rng.standard_normal((1, 2, 128, 16))
+    keys, _, _ = oracle.lsh_hash(Q, rng.standard_normal((2, 16, 4)), 8)
+    perm = oracle.lsh_sort(keys)
+    full_o, full_l = oracle.lsh_attend_fwd(Q, V, keys, perm, 16, True)
+    o, l = oracle.lsh_attend_fwd_range(Q, V, keys, perm, 16, True, 2, 5)
+    slots = perm[..., 32:80]  # queries of chunks 2..4
+    mask = np.zeros(l.shape, bool)
+    for r in range(2):
+        for h in range(2):
+            mask[r, 0, h, slots[r, 0, h]] = True
+    np.testing.assert_array_equal(l[mask], full_l[mask])
+    np.testing.assert_array_equal(o[mask], full_o[mask])
+    assert np.all(l[~mask] == 0) and np.all(o[~mask] == 0)
