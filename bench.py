@@ -464,11 +464,23 @@ class OracleSampler:
 
 
 def run_cpu_baseline(w):
-    s = OracleSampler(w)
-    n_tok, n_chunks = 8192, 128
-    sec, full = s.step(n_tok, n_chunks)
+    """The oracle as it stands on one whole head (b=0, h=0) of the workload:
+    hash, sort, attention and combine for all rounds, scaled by B*H."""
+    from oracle import oracle as cpu_oracle
+    cpu_oracle.build()
+    inp = W.make_inputs(w)
+    Q = inp["Q"][:1, :1].float().numpy()
+    V = inp["V"][:1, :1].float().numpy()
+    rot = inp["rot"].float().numpy()
+    t0 = time.perf_counter()
+    cpu_oracle.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal)
+    sec = time.perf_counter() - t0
+    full = sec * w.B * w.H
     return {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": 1,
-            "kind": "oracle", "sample": s.describe(n_tok, n_chunks) + f"; sample took {sec:.1f} s"}
+            "kind": "oracle",
+            "sample": f"one head (b=0, h=0) of {w.name}, all {w.n_rounds} rounds, full "
+                      f"L={w.L}: hash, sort, attention, combine in {sec:.1f} s single-threaded "
+                      f"fp64; scaled by B*H={w.B * w.H} to the whole step"}
 
 
 def run_reference(args, world, rank):

@@ -190,13 +190,16 @@ attend_fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V,
       for (int rr = 0; rr < n_rounds - 1; ++rr) mx = fmaxf(mx, prev_lse[(size_t)rr * n_tok + tok]);
       float z = expf(my_lse - mx);
       for (int rr = 0; rr < n_rounds - 1; ++rr) z += expf(prev_lse[(size_t)rr * n_tok + tok] - mx);
+      // weights relative to the maximum: near lse = -1e5 (a token alone in
+      // every round) mx + log(z) is not representable to the needed precision
+      const float rz = 1.f / z;
       const float tot = mx + logf(z);
-      const float wl = expf(my_lse - tot);
+      const float wl = expf(my_lse - mx) * rz;
       float o[16];
 #pragma unroll
       for (int x = 0; x < 16; ++x) o[x] = wl * acc[x];
       for (int rr = 0; rr < n_rounds - 1; ++rr) {
-        const float wr = expf(prev_lse[(size_t)rr * n_tok + tok] - tot);
+        const float wr = expf(prev_lse[(size_t)rr * n_tok + tok] - mx) * rz;
         const float* src = prev_o + ((size_t)rr * n_tok + tok) * kHeadDim + part * 16;
         float t8[8];
         load8(src, t8);
@@ -227,10 +230,11 @@ __global__ void combine_kernel(const float* __restrict__ o_part, const float* __
   for (int r = 0; r < n_rounds; ++r) mx = fmaxf(mx, lse_r[(size_t)r * n_tok + tok]);
   float z = 0.f;
   for (int r = 0; r < n_rounds; ++r) z += expf(lse_r[(size_t)r * n_tok + tok] - mx);
+  const float rz = 1.f / z;
   const float tot = mx + logf(z);
   float o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   for (int r = 0; r < n_rounds; ++r) {
-    const float w = expf(lse_r[(size_t)r * n_tok + tok] - tot);
+    const float w = expf(lse_r[(size_t)r * n_tok + tok] - mx) * rz;
     float t8[8];
     load8(o_part + ((size_t)r * n_tok + tok) * kHeadDim + k, t8);
 #pragma unroll
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(256)
 attend_bwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V, const T* __restrict__ dO,
                        const uint32_t* __restrict__ keys, const int32_t* __restrict__ perm,
                        const float* __restrict__ lse, const float* __restrict__ G, AttnDims a,
-                       float* __restrict__ dq_acc, float* __restrict__ dk_acc,
+                       float inv_rounds, float* __restrict__ dq_acc, float* __restrict__ dk_acc,
                        float* __restrict__ dv_acc) {
   extern __shared__ float smem[];
   const int W = a.W, c = a.chunk;
@@ -327,10 +331,13 @@ attend_bwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V, const T
     const uint32_t lo = ki - ki % (uint32_t)a.L;
     const uint32_t span = a.causal ? (ki - lo + 1) : (uint32_t)a.L;
     const float li = ls[qi], gi = gs[qi];
+    // A token alone in every round has lse = -1e5 + ln R, which fp32 stores
+    // only to ~4e-3; its self weight in each round is exactly 1/R.
+    const bool lone = li < kSelfScore + kLoneMargin;
     for (int u = part; u < W; u += 4) {
       bool live;
       const float s = masked_score(q, qs, sc, ks, u, ki, lo, span, &live);
-      const float p = expf(s - li);
+      const float p = (lone && ks[u] == ki) ? inv_rounds : expf(s - li);
       float ds = 0.f;
       if (live) {
         float dp = 0.f;

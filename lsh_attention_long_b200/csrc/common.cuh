@@ -9,7 +9,10 @@ namespace lsh {
 
 constexpr int kHeadDim = 64;           // the only head dimension the kernels take
 constexpr float kSelfScore = -1e5f;    // replaces the score of a token with itself
-constexpr int kMaxChunkSimt = 128;     // largest chunk of the general (SIMT) kernels
+// A combined logsumexp below kSelfScore + kLoneMargin can only come from a
+// token whose every round held nothing but itself: any other key scores at
+// least -|q|/sqrt(d), far above -1e5 for any finite-range input.
+constexpr float kLoneMargin = 64.f;
 
 constexpr int kErrBadKeys = 6;         // LSH_ERR_BAD_KEYS
 

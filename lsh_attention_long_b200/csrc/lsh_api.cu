@@ -181,7 +181,8 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   if (s0 != LSH_OK) return s0;
   const dim3 grid((unsigned)a.n_chunks, (unsigned)(D.R * a.BH));
   lsh::attend_bwd_simt_kernel<T><<<grid, 256, smem, st>>>(
-      q, static_cast<const T*>(V), static_cast<const T*>(dO), keys, perm, lse, G, a, dq, dk, dv);
+      q, static_cast<const T*>(V), static_cast<const T*>(dO), keys, perm, lse, G, a,
+      1.f / (float)D.R, dq, dk, dv);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
   lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok, static_cast<T*>(dQ),
                                                   static_cast<T*>(dV));
