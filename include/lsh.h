@@ -66,7 +66,8 @@ typedef enum {
   LSH_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
   LSH_ERR_WORKSPACE = 4,   /* ws is NULL or smaller than lsh_workspace_size() */
   LSH_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
-  LSH_ERR_BAD_KEYS = 6     /* keys not of the form bucket*L + position, bucket < n_buckets */
+  LSH_ERR_BAD_KEYS = 6,    /* keys not of the form bucket*L + position, bucket < n_buckets */
+  LSH_ERR_SCRATCH_LIMIT = 7 /* problem too large for the library's built-in scratch array */
 } lsh_status;
 
 typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
@@ -146,6 +147,38 @@ LSH_API lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const v
                           const void* dO, const uint32_t* keys, const int32_t* perm,
                           const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,
                           void* stream);
+
+/* lsh_attend_fwd with the combine, for callers that cannot allocate memory.
+ *
+ * No passage of the pages corresponds to this entry point; it exists for
+ * deployment.  Some callers may not call cudaMalloc at the moment they run
+ * attention: a host framework whose memory planner owns every device buffer,
+ * a plugin inside another runtime's execution phase, or a latency-critical
+ * loop where an allocation would synchronise the device.  This call takes
+ * the same inputs and outputs as lsh_attend_fwd with O given (Q, V, keys,
+ * perm -> O, lse) but no workspace: the per-round partials of rounds
+ * 0..R-2 live in a scratch array of LSH_STATIC_SCRATCH_BYTES (64 MiB) that
+ * the library defines at file scope in device memory.  Every GPU that loads
+ * the library holds that array until the process exits.  It allocates
+ * nothing itself: no cudaMalloc, no cudaFree, no allocating library call.
+ *   - Capacity: (n_rounds - 1) * B * H * L * (d + 1) * 4 bytes must not
+ *     exceed LSH_STATIC_SCRATCH_BYTES, else LSH_ERR_SCRATCH_LIMIT is
+ *     returned before any launch.  One round (n_rounds == 1) needs none.
+ *   - Set-up: the first call on a device, with that device current, looks up
+ *     the array's device address (cudaGetSymbolAddress) and caches it; make
+ *     that first call outside any stream capture.
+ *   - Sharing: all calls in the process on a device use the same array and
+ *     it keeps whatever the last call left there.  Every element a call reads
+ *     is written earlier in the same call, so nothing needs clearing, but
+ *     two calls whose kernels overlap on the GPU (different streams, no
+ *     ordering between them) race on the array and give wrong results.
+ *     Order such calls on one stream or with events.
+ * Results are those of lsh_attend_fwd(shape, Q, V, keys, perm, NULL, NULL,
+ * O, lse, ws, ws_bytes, stream). */
+#define LSH_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+LSH_API lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const void* V,
+                                         const uint32_t* keys, const int32_t* perm, void* O,
+                                         float* lse, void* stream);
 
 /* Synchronises `stream`, returns the first error a kernel recorded since the
  * last call (LSH_OK if none) and clears it.  LSH_ERR_CUDA if the

@@ -6,10 +6,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "attend_simt.cuh"
 #include "common.cuh"
 #include "hash_simt.cuh"
 #include "sort.cuh"
+
+// Scratch of lsh_attend_fwd_static: the per-round partials of rounds
+// 0..R-2 for callers that cannot hand the library a workspace.  It is sized
+// once, here, and shared by every call on the device.
+static __device__ __align__(256) unsigned char g_static_scratch[LSH_STATIC_SCRATCH_BYTES];
 
 namespace {
 
@@ -189,6 +196,25 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   return last_launch();
 }
 
+// Device address of g_static_scratch per device, looked up on first use.
+// In host code the symbol is only a handle; kernels must get this address.
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+lsh_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LSH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return LSH_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return LSH_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -296,6 +322,29 @@ lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const void* V, 
                                         st);
 }
 
+lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const void* V,
+                                 const uint32_t* keys, const int32_t* perm, void* O, float* lse,
+                                 void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Q || !V || !keys || !perm || !O) return LSH_ERR_INVALID_ARG;
+  if (misaligned(Q) || misaligned(V) || misaligned(keys) || misaligned(perm) || misaligned(O) ||
+      misaligned(lse))
+    return LSH_ERR_INVALID_ARG;
+  if (fwd_ws_bytes(D) > LSH_STATIC_SCRATCH_BYTES) return LSH_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  s = static_scratch(&scratch);
+  if (s != LSH_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  return D.dtype == LSH_BF16
+             ? attend_fwd_launch<__nv_bfloat16>(D, Q, V, keys, perm, nullptr, nullptr, O, lse,
+                                                scratch, LSH_STATIC_SCRATCH_BYTES, st)
+             : attend_fwd_launch<float>(D, Q, V, keys, perm, nullptr, nullptr, O, lse, scratch,
+                                        LSH_STATIC_SCRATCH_BYTES, st);
+}
+
 lsh_status lsh_device_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return LSH_ERR_CUDA;
   int v = 0;
@@ -314,6 +363,7 @@ const char* lsh_status_string(lsh_status status) {
     case LSH_ERR_WORKSPACE: return "workspace missing or too small";
     case LSH_ERR_TIMEOUT: return "device wait timed out";
     case LSH_ERR_BAD_KEYS: return "keys are not bucket*L + position";
+    case LSH_ERR_SCRATCH_LIMIT: return "problem exceeds the built-in scratch of lsh_attend_fwd_static";
   }
   return "unknown status";
 }

@@ -20,7 +20,8 @@ LIB_PATH = os.path.join(_HERE, "liblsh.so")
 
 LSH_F32, LSH_BF16 = 0, 1
 STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "LSH_ERR_CUDA",
-          4: "LSH_ERR_WORKSPACE", 5: "LSH_ERR_TIMEOUT", 6: "LSH_ERR_BAD_KEYS"}
+          4: "LSH_ERR_WORKSPACE", 5: "LSH_ERR_TIMEOUT", 6: "LSH_ERR_BAD_KEYS",
+          7: "LSH_ERR_SCRATCH_LIMIT"}
 
 EXPORTS = ("lsh_workspace_size", "lsh_hash", "lsh_sort", "lsh_attend_fwd", "lsh_combine",
            "lsh_forward", "lsh_attend_bwd", "lsh_device_status", "lsh_status_string")

@@ -57,7 +57,7 @@ def _shape(**kw):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert lib.lsh_status_string(code)
     assert lib.lsh_status_string(6) == b"keys are not bucket*L + position"
 
