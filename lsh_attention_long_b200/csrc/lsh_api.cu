@@ -11,6 +11,7 @@
 #include "attend_simt.cuh"
 #include "common.cuh"
 #include "hash_simt.cuh"
+#include "hash_tc.cuh"
 #include "sort.cuh"
 
 // Scratch of lsh_attend_fwd_static: the per-round partials of rounds
@@ -90,9 +91,61 @@ lsh::AttnDims attn_dims(const Dims& D) {
   return a;
 }
 
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+// Tensor-core hash: bf16, nb/2 a power of two in [16, 1024].
+bool hash_tc_supported(const Dims& D) {
+  const int half = D.nb / 2;
+  return D.dtype == LSH_BF16 && half >= 16 && half <= 1024 && (half & (half - 1)) == 0;
+}
+
+lsh_status hash_tc_launch(const Dims& D, const void* Q, const void* rot, uint32_t* keys,
+                          int32_t* buckets, cudaStream_t st) {
+  lsh::HashTcArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.rot = static_cast<const __nv_bfloat16*>(rot);
+  a.keys = keys;
+  a.buckets = buckets;
+  a.n_tok = (int)D.n_tok;
+  a.L = D.L;
+  a.half = D.nb / 2;
+  a.R = D.R;
+  // rounds whose rotation columns fit the shared-memory budget; when they
+  // span more than one 256-column N-tile they must fill whole N-tiles
+  int rg = lsh::kHashTcRotBytes / (a.half * 128);
+  if (rg > D.R) rg = D.R;
+  if (rg * a.half > 256) rg = (rg * a.half / 256) * 256 / a.half;
+  if (rg < 1) rg = 1;
+  a.rounds_per_group = rg;
+  a.n_groups = (D.R + rg - 1) / rg;
+  a.n_mtiles = (int)((D.n_tok + 127) / 128);
+  int per = num_sms() / a.n_groups;
+  if (per < 1) per = 1;
+  if (per > a.n_mtiles) per = a.n_mtiles;
+  a.ctas_per_group = per;
+  const size_t smem = lsh::hash_tc_smem_bytes(rg, a.half);
+  const unsigned grid = (unsigned)(a.n_groups * per);
+  if (a.half >= 32) {
+    lsh_status s0 = allow_smem(lsh::hash_tc_kernel<32>, smem);
+    if (s0 != LSH_OK) return s0;
+    lsh::hash_tc_kernel<32><<<grid, 128, smem, st>>>(a);
+  } else {
+    lsh_status s0 = allow_smem(lsh::hash_tc_kernel<16>, smem);
+    if (s0 != LSH_OK) return s0;
+    lsh::hash_tc_kernel<16><<<grid, 128, smem, st>>>(a);
+  }
+  return last_launch();
+}
+
 template <typename T>
 lsh_status hash_launch(const Dims& D, const void* Q, const void* rot, uint32_t* keys,
                        int32_t* buckets, cudaStream_t st) {
+  if (hash_tc_supported(D)) return hash_tc_launch(D, Q, rot, keys, buckets, st);
   constexpr int TOK = 128;
   const int half = D.nb / 2;
   const dim3 grid((unsigned)((D.n_tok + TOK - 1) / TOK), (unsigned)D.R);

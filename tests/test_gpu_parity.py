@@ -232,3 +232,42 @@ def test_empty_batch_is_a_no_op():
     out = L.lsh_forward(Q, Q, rot, 8, 64, True)
     assert out["O"].numel() == 0
     assert L.lsh_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# tensor-core hash: shapes that exercise its round grouping and N-tiling
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,Lx,nb,R", [
+    (1, 3, 320, 32, 3),     # nb/2 = 16: 16-column chunks, ragged token tiles
+    (2, 2, 256, 64, 5),     # five rounds in one group (5 * 32 = 160 columns)
+    (1, 2, 512, 256, 3),    # 3 * 128 columns: groups of two rounds, then one
+    (1, 1, 384, 512, 9),    # 9 * 256: one round per N-tile, two groups
+    (1, 1, 256, 2048, 2),   # nb/2 = 1024: four N-tiles per round
+])
+def test_tensor_core_hash_shapes(oracle, B, H, Lx, nb, R):
+    inp = W.make_random(B, H, Lx, 64, nb, R, torch.bfloat16, seed=nb + R)
+    Q, rot = inp["Q"].cuda(), inp["rot"].cuda()
+    keys, buckets = L.lsh_hash(Q, rot, nb)
+    torch.cuda.synchronize()
+    _check_status()
+    check_hash(oracle, Q, rot, nb, keys, buckets)
+
+
+def test_tensor_core_hash_exact_ties_take_lowest_index():
+    """Duplicated and negated rotation columns make exact ties in the GPU's own
+    arithmetic; the first index of [p ; -p] must win."""
+    nb, half = 64, 32
+    g = torch.Generator().manual_seed(5)
+    base = torch.randn(64, half, generator=g)
+    base[:, 1] = base[:, 0]        # p_1 == p_0
+    base[:, 3] = -base[:, 2]       # p_3 == -p_2
+    rot = base[None].to(torch.bfloat16).cuda()
+    Q = torch.randn(1, 1, 1024, 64, generator=g).to(torch.bfloat16).cuda()
+    _, b = L.lsh_hash(Q, rot, nb)
+    torch.cuda.synchronize()
+    b = b.cpu().numpy().ravel()
+    assert not np.isin(b, [1, half + 1]).any()       # column 0 always beats its copy
+    # p_3 == -p_2: z_3 ties z_{half+2} and z_2 ties z_{half+3}; the lower index wins
+    assert not np.isin(b, [half + 2, half + 3]).any()
+    assert np.isin(b, [0, half, 2, 3]).any()
