@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attend_simt.cuh"
+#include "attend_tc.cuh"
 #include "common.cuh"
 #include "hash_simt.cuh"
 #include "hash_tc.cuh"
@@ -73,9 +74,37 @@ lsh_status allow_smem(K kernel, size_t bytes) {
              : LSH_ERR_CUDA;
 }
 
-size_t fwd_ws_bytes(const Dims& D) {
+// Tensor-core attention: bf16, d = 64, chunk = 64.
+bool attend_tc_supported(const Dims& D) { return D.dtype == LSH_BF16 && D.c == 64; }
+
+size_t counters_bytes(const Dims& D) {
+  return align_up(((size_t)D.B * D.H * D.R + 1) * sizeof(unsigned));
+}
+
+// Workspace of one lsh_attend_fwd call, given which optional outputs the
+// caller supplies.
+size_t attend_fwd_ws_bytes(const Dims& D, bool has_o_part, bool has_lse_r, bool has_O) {
+  if (attend_tc_supported(D)) {
+    if (has_O && !has_o_part && !has_lse_r)  // online combine: running state per token
+      return counters_bytes(D) + align_up(D.n_tok * kHeadDim * sizeof(float)) +
+             align_up(D.n_tok * sizeof(float2));
+    const size_t all = (size_t)D.R * D.n_tok;  // every round's partials
+    return counters_bytes(D) + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
+           (has_lse_r ? 0 : align_up(all * sizeof(float)));
+  }
+  if (!has_O) return 0;
   const size_t prev = (size_t)(D.R - 1) * D.n_tok;
-  return align_up(prev * kHeadDim * sizeof(float)) + align_up(prev * sizeof(float));
+  return (has_o_part ? 0 : align_up(prev * kHeadDim * sizeof(float))) +
+         (has_lse_r ? 0 : align_up(prev * sizeof(float)));
+}
+
+size_t fwd_ws_bytes(const Dims& D) {
+  size_t m = 0;
+  for (int i = 0; i < 8; ++i) {
+    const size_t b = attend_fwd_ws_bytes(D, i & 1, i & 2, i & 4);
+    m = b > m ? b : m;
+  }
+  return m;
 }
 
 size_t bwd_ws_bytes(const Dims& D) {
@@ -169,10 +198,81 @@ lsh_status sort_launch(const Dims& D, const uint32_t* keys, int32_t* perm, cudaS
   return last_launch();
 }
 
+lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const uint32_t* keys,
+                            const int32_t* perm, float* o_part, float* lse_r, void* O,
+                            float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const bool online = O && !o_part && !lse_r;
+  if (ws_bytes < attend_fwd_ws_bytes(D, o_part != nullptr, lse_r != nullptr, O != nullptr) ||
+      !ws)
+    return LSH_ERR_WORKSPACE;
+  lsh::AttnTcArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.keys = keys;
+  a.perm = perm;
+  a.L = D.L;
+  a.R = D.R;
+  a.BH = D.B * D.H;
+  a.n_chunks = D.L / 64;
+  a.causal = D.causal;
+  a.n_tiles = (a.n_chunks + 1) / 2;
+  a.tpi = a.n_tiles < 4 ? a.n_tiles : 4;
+  a.ipr = (a.n_tiles + a.tpi - 1) / a.tpi;
+  // heads whose running state and q, v rows share L2 while their rounds
+  // run: enough items between dependent rounds to cover one wave of CTAs
+  const size_t per_head = (size_t)D.L * (kHeadDim * 4 + 8 + 2 * kHeadDim * 2);
+  const int sms = num_sms();
+  long long hpb = (long long)((96ull << 20) / per_head);
+  const long long want = (2LL * sms + a.ipr - 1) / a.ipr;
+  if (hpb > want) hpb = want;
+  if (hpb < 1) hpb = 1;
+  if (hpb > a.BH) hpb = a.BH;
+  a.heads_per_block = (int)hpb;
+  a.n_items = (long long)a.R * a.BH * a.ipr;
+  a.online = online ? 1 : 0;
+  char* w = static_cast<char*>(ws);
+  a.counters = reinterpret_cast<unsigned*>(w);
+  w += counters_bytes(D);
+  a.acc_o = nullptr;
+  a.acc_ml = nullptr;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.o_part = o_part;
+  a.lse_r = lse_r;
+  if (online) {
+    a.acc_o = reinterpret_cast<float*>(w);
+    w += align_up(D.n_tok * kHeadDim * sizeof(float));
+    a.acc_ml = reinterpret_cast<float2*>(w);
+  } else {
+    const size_t all = (size_t)D.R * D.n_tok;
+    if (!a.o_part) {
+      a.o_part = reinterpret_cast<float*>(w);
+      w += align_up(all * kHeadDim * sizeof(float));
+    }
+    if (!a.lse_r) a.lse_r = reinterpret_cast<float*>(w);
+  }
+  if (cudaMemsetAsync(a.counters, 0, counters_bytes(D), st) != cudaSuccess) return LSH_ERR_CUDA;
+  const size_t smem = lsh::attend_tc_smem_bytes();
+  lsh_status s0 = allow_smem(lsh::attend_tc_kernel, smem);
+  if (s0 != LSH_OK) return s0;
+  const long long grid = a.n_items < sms ? a.n_items : sms;
+  lsh::attend_tc_kernel<<<(unsigned)grid, lsh::kAtThreads, smem, st>>>(a);
+  if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+  if (!online && O) {
+    const size_t n = D.n_tok * 8;
+    lsh::combine_kernel<__nv_bfloat16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        a.o_part, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
+    return last_launch();
+  }
+  return LSH_OK;
+}
+
 template <typename T>
 lsh_status attend_fwd_launch(const Dims& D, const void* Q, const void* V, const uint32_t* keys,
                              const int32_t* perm, float* o_part, float* lse_r, void* O, float* lse,
                              void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (attend_tc_supported(D))
+    return attend_tc_launch(D, Q, V, keys, perm, o_part, lse_r, O, lse, ws, ws_bytes, st);
   const lsh::AttnDims a = attn_dims(D);
   const size_t smem = lsh::simt_fwd_smem_bytes(a.chunk, a.W);
   lsh_status s0 = allow_smem(lsh::attend_fwd_simt_kernel<T>, smem);
@@ -189,7 +289,8 @@ lsh_status attend_fwd_launch(const Dims& D, const void* Q, const void* V, const 
   float* po = o_part;
   float* pl = lse_r;
   if (D.R > 1 && (!po || !pl)) {
-    if (!ws || ws_bytes < fwd_ws_bytes(D)) return LSH_ERR_WORKSPACE;
+    if (!ws || ws_bytes < attend_fwd_ws_bytes(D, po != nullptr, pl != nullptr, true))
+      return LSH_ERR_WORKSPACE;
     char* w = static_cast<char*>(ws);
     const size_t prev = (size_t)(D.R - 1) * D.n_tok;
     if (!po) po = reinterpret_cast<float*>(w);
@@ -386,7 +487,8 @@ lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const vo
   if (misaligned(Q) || misaligned(V) || misaligned(keys) || misaligned(perm) || misaligned(O) ||
       misaligned(lse))
     return LSH_ERR_INVALID_ARG;
-  if (fwd_ws_bytes(D) > LSH_STATIC_SCRATCH_BYTES) return LSH_ERR_SCRATCH_LIMIT;
+  if (attend_fwd_ws_bytes(D, false, false, true) > LSH_STATIC_SCRATCH_BYTES)
+    return LSH_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   s = static_scratch(&scratch);
   if (s != LSH_OK) return s;
