@@ -154,13 +154,13 @@ def lsh_attend_fwd(Q, V, keys, perm, n_buckets: int, chunk: int, causal: bool, *
             O = torch.empty_like(Q)
         if lse is None:
             lse = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
-        if ws is None and (o_part is None or lse_r is None):
-            ws = workspace(shape, Q.device)
     else:
         if o_part is None:
             o_part = torch.empty((R, B, H, L, d), dtype=torch.float32, device=Q.device)
         if lse_r is None:
             lse_r = torch.empty((R, B, H, L), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(shape, Q.device)
     _call("lsh_attend_fwd", ctypes.byref(shape), _ptr(Q), _ptr(V), _ptr(keys), _ptr(perm),
           _ptr(o_part), _ptr(lse_r), _ptr(O) if combine else None,
           _ptr(lse) if combine else None, _ptr(ws), 0 if ws is None else ws.numel(),
