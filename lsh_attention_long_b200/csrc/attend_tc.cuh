@@ -12,40 +12,46 @@
 // Tile = two consecutive chunks (128 query rows, one TMEM lane each); its
 // window is three chunks (k-1, k, k+1), 192 keys, of which each query chunk
 // uses two.  Per tile:
-//   S  = Q[128 x 64] . K[192 x 64]^T   tcgen05.mma, three N=64 MMAs -> TMEM
-//   P  = masked softmax numerators      CUDA cores, bf16 into shared memory
-//   O  = P[128 x 192] . V[192 x 64]     tcgen05.mma -> TMEM
-// The raw (unnormalised) queries serve as keys in the MMA; the key
-// normalisation 1/|q_j| and 1/sqrt(d) scale the scores in the softmax, so
-// the MMA multiplies exact bf16 inputs.
+//   S  = Q[128 x 64] . K[192 x 64]^T   tcgen05.mma (three N=64 MMAs) -> TMEM
+//   P  = masked softmax numerators      CUDA cores, bf16, written over S in TMEM
+//   O  = P[128 x 192] . V[192 x 64]     tcgen05.mma with A = P from TMEM
+// The raw queries serve as keys in the MMA; 1/|q_j| (precomputed per token)
+// and 1/sqrt(d) scale the scores in the softmax, so the MMA multiplies exact
+// bf16 inputs.
 //
 // Mask on packed keys (key = bucket*L + position, ascending within a bucket
 // in position order): key_j is in the query's bucket and allowed iff
 // (key_j - bucket_i*L) < span as unsigned, with span = key_i - bucket_i*L
 // (causal: strictly earlier positions, which also drops the token itself) or
 // L (non-causal, where key_j == key_i is dropped separately).  The token's
-// own entry enters only when a row has no other key in any of its round's
-// chunks: then the round's output is its own value and lse = -1e5.
+// own entry enters only when a row has no other key in its round's window:
+// then the round's output is its own value and lse = -1e5.
 //
-// Warp roles: warps 0-7 (256 threads) compute; thread (wg, m) owns query row
-// m and the window chunk kc = m/64 + wg, i.e. 64 of the row's 128 window
-// columns; the two halves of a row meet through shared memory for the row
-// max and sum.  Warp 8 gathers: row indices (perm), packed keys, and q, v
-// rows (cp.async, 128B-swizzled) of the next tiles into a ring of 3 slots,
-// signalling full/empty mbarriers.  Work comes from a global ticket
-// (dynamic scheduling) in items of up to 4 tiles of one (round, head) row.
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  two softmax/epilogue warpgroups; warpgroup w takes the
+//                   CTA's tiles w, w+2, w+4, ... so one warpgroup's softmax
+//                   overlaps the other's MMAs and epilogue.  Each owns half of
+//                   tensor memory: S/P in columns [256w, 256w+192), O in
+//                   [256w+192, 256w+256).
+//   warp 8          producer: takes work tickets, gathers perm, packed keys,
+//                   key scales and q, v rows (cp.async, 128B-swizzled) into a
+//                   ring of 4 shared-memory slots (full/empty mbarriers).
+//   warp 9          tensor-core issue: one thread polls the barriers and
+//                   issues S for tile n+1 as soon as its data and TMEM half
+//                   are free, and P.V for tile n as soon as P is written.
 //
 // Two output modes:
 //   partial  every round's normalised o_r (fp32) and lse_r go to o_part /
 //            lse_r at original positions (the combine runs afterwards);
-//   online   rounds of a head are taken in order; each round's tile folds its
+//   online   rounds of a head are taken in order; each round folds its
 //            result into a running (max, sum, unnormalised output) per token
 //            kept in the workspace, and the last round writes O (bf16) and
-//            lse.  Items of round r of a head wait (bounded spin) until all
-//            items of round r-1 of that head are done; tickets are taken in
-//            an order where that dependency always points to earlier
-//            tickets, so the scheme cannot deadlock.  Heads are processed in
-//            blocks sized so that a block's accumulators and q, v rows stay
+//            lse.  A tile of round r of a head waits (bounded spin) until
+//            every tile of round r-1 of that head is done (per-head tile
+//            counters); tickets are handed out in an order where that
+//            dependency always points to earlier tickets, so the scheme
+//            cannot deadlock.  Heads are taken in
+//            blocks sized so that a block's running state and q, v rows stay
 //            resident in L2 while its rounds run.
 #pragma once
 
@@ -53,14 +59,16 @@
 
 namespace lsh {
 
-constexpr int kAtSlots = 3;
-constexpr int kAtConsumers = 256;
-constexpr int kAtThreads = kAtConsumers + 32;
-constexpr int kAtChunkBytes = 64 * 128;              // 64 rows of 128 B
-constexpr int kAtSlotBytes = 6 * kAtChunkBytes;      // q then v of 3 chunks
-constexpr int kAtPBytes = 3 * 128 * 128;             // P: 3 key blocks of 128 rows
-constexpr uint32_t kAtNoKey = 0xffffffffu;           // never inside a bucket range
+constexpr int kAtSlots = 4;
+constexpr int kAtThreads = 320;
+constexpr int kAtChunkBytes = 64 * 128;          // 64 rows of 128 B
+constexpr int kAtSlotBytes = 6 * kAtChunkBytes;  // q then v of 3 chunks
+constexpr uint32_t kAtNoKey = 0xffffffffu;       // never inside a bucket range
 constexpr float kLog2e = 1.4426950408889634f;
+// Largest score bound |q_i|/sqrt(d) used directly as the softmax reference:
+// every allowed score s >= -bound, so exp(s - bound) >= exp(-2 * 30), far
+// from fp32 / bf16 underflow.
+constexpr float kRefLimit = 30.f;
 
 struct AtInfo {
   int r, bh, t;
@@ -75,6 +83,7 @@ struct AttnTcArgs {
   const __nv_bfloat16* V;
   const uint32_t* keys;
   const int32_t* perm;
+  const float* rn;   // [n_tok] log2(e) / (|q| sqrt(d)), 0 for a zero row
   int L, R, BH, n_chunks, causal;
   int n_tiles;       // tiles per row: ceil(n_chunks / 2)
   int tpi;           // tiles per item
@@ -88,45 +97,44 @@ struct AttnTcArgs {
   float2* acc_ml;    // online mode: [n_tok] (running max, running sum)
   __nv_bfloat16* O;  // online mode, last round
   float* lse;
-  unsigned* counters;  // [BH][R] items done; then one ticket counter
+  unsigned* counters;  // [BH][R] tiles done; then one ticket counter
 };
 
-// Shared memory beyond the 1024-aligned base.
 struct AtSmem {
   uint32_t pos[kAtSlots][192];
   uint32_t key[kAtSlots][192];
+  float rn[kAtSlots][192];
   AtInfo info[kAtSlots];
-  float rn[192];
-  float red_max[2][128];
-  float red_sum[2][128];
-  uint64_t full[kAtSlots], empty[kAtSlots], bar_s, bar_o;
+  uint64_t full[kAtSlots], empty[kAtSlots];
+  uint64_t s_full[2], p_full[2], o_full[2], tm_free[2];
   uint32_t tmem_base;
   int abort;
+  int dep_bh, dep_r;  // last (head, round) whose previous round was seen complete
 };
 
 __host__ __device__ inline size_t attend_tc_smem_bytes() {
-  return 1024 + (size_t)kAtSlots * kAtSlotBytes + kAtPBytes + sizeof(AtSmem);
+  return 1024 + (size_t)kAtSlots * kAtSlotBytes + sizeof(AtSmem);
 }
 
-// Named barrier over the 256 compute threads; returns the OR of `pred`.
-__device__ __forceinline__ bool consumers_or(bool pred) {
+// Named barrier (id 1 + w) over the 128 threads of warpgroup w; OR of pred.
+__device__ __forceinline__ bool wg_or(int w, bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred)
+      : "r"((uint32_t)pred), "r"(1 + w)
       : "memory");
   return r != 0;
-}
-__device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar))
                : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -137,6 +145,25 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Waits for a phase unless the CTA aborted; false on abort or timeout
+// (timeouts record LSH_ERR_TIMEOUT and set the abort flag).
+__device__ __forceinline__ bool at_wait(uint64_t* bar, uint32_t parity, int* abort) {
+  const long long t0 = clock64();
+  while (!tc::mbar_test(bar, parity)) {
+    if (*(volatile int*)abort) return false;
+    if (clock64() - t0 > tc::kSpinCycles) {
+      record_status(tc::kErrTimeout);
+      *(volatile int*)abort = 1;
+      return false;
+    }
+  }
+  return true;
 }
 
 // Item `ticket` -> (round, head row, first tile).  Order: blocks of heads;
@@ -155,36 +182,51 @@ __device__ __forceinline__ void at_decode(const AttnTcArgs& a, long long ticket,
   t0 = (rem % a.ipr) * a.tpi;
 }
 
+// log2(e) / (|q| sqrt(d)) per token (0 for a zero row): the key
+// normalisation and score scale, in the log2 units the softmax uses.
+__global__ void key_scale_kernel(const __nv_bfloat16* __restrict__ Q, size_t n_tok,
+                                 float* __restrict__ rn) {
+  const size_t tok = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tok >= n_tok) return;
+  float ssq = 0.f;
+#pragma unroll
+  for (int k = 0; k < kHeadDim; k += 8) {
+    float x[8];
+    load8(Q + tok * kHeadDim + k, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ssq = fmaf(x[e], x[e], ssq);
+  }
+  rn[tok] = ssq > 0.f ? rsqrtf(ssq) * (0.125f * kLog2e) : 0.f;
+}
+
 __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* slots = sm;
-  uint8_t* pbuf = sm + kAtSlots * kAtSlotBytes;
-  AtSmem& S = *reinterpret_cast<AtSmem*>(pbuf + kAtPBytes);
+  AtSmem& S = *reinterpret_cast<AtSmem*>(sm + kAtSlots * kAtSlotBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     for (int s = 0; s < kAtSlots; ++s) {
-      tc::mbar_init(&S.full[s], 64);  // 32 producer lanes x (cp.async arrive + arrive)
-      tc::mbar_init(&S.empty[s], 1);
+      tc::mbar_init(&S.full[s], 64);    // 32 producer lanes x (cp.async arrive + arrive)
+      tc::mbar_init(&S.empty[s], 128);  // every thread of the warpgroup that used it
     }
-    tc::mbar_init(&S.bar_s, 1);
-    tc::mbar_init(&S.bar_o, 1);
+    for (int w = 0; w < 2; ++w) {
+      tc::mbar_init(&S.s_full[w], 1);
+      tc::mbar_init(&S.p_full[w], 128);
+      tc::mbar_init(&S.o_full[w], 1);
+      tc::mbar_init(&S.tm_free[w], 128);
+    }
     tc::mbar_init_fence();
     S.abort = 0;
+    S.dep_bh = -1;
+    S.dep_r = -1;
   }
-  if (warp == 0) {
-    tc::tmem_alloc(&S.tmem_base, 256);
+  if (warp == 9) {
+    tc::tmem_alloc(&S.tmem_base, 512);
     tc::tmem_relinquish();
   }
-  // structural zeros of P: key block 0 for rows 64..127, block 2 for rows 0..63
-  for (int e = tid; e < 64 * 8 * 2; e += blockDim.x) {
-    const int half = e / 512, row = (e % 512) / 8 + (half ? 0 : 64), ch = e % 8;
-    uint8_t* blk = pbuf + (half ? 2 : 0) * 16384;
-    *reinterpret_cast<uint4*>(blk + tc::sw128_offset(row, ch)) = make_uint4(0, 0, 0, 0);
-  }
-  tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -194,154 +236,202 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    int s = 0;
-    uint32_t empty_phase = 0;  // bit s: parity to wait for on empty[s]
     long long item = -1;
     int r = 0, bh = 0, t = 0, t_end = 0;
-    for (;;) {
-      int done = 0;
+    int done_marks = 0;
+    for (uint32_t n = 0;; ++n) {
+      const int s = n % kAtSlots;
+      bool done = false;
       if (t >= t_end) {  // next item
         long long tk = 0;
         if (lane == 0) tk = (long long)atomicAdd(ticket_ctr, 1u);
         tk = __shfl_sync(0xffffffffu, tk, 0);
         if (tk >= a.n_items) {
-          done = 1;
+          done = true;
         } else {
           item = tk;
           at_decode(a, item, r, bh, t);
           t_end = min(t + a.tpi, a.n_tiles);
         }
       }
-      // wait until the consumers released this slot (first pass: free)
       const bool ok = __all_sync(0xffffffffu,
-                                 tc::mbar_wait(&S.empty[s], ((empty_phase >> s) & 1u) ^ 1u));
-      empty_phase ^= 1u << s;
-      if (!ok || *(volatile int*)&S.abort) {
-        if (lane == 0) { record_status(tc::kErrTimeout); S.abort = 1; }
-        // still release the consumers waiting on this slot
+                                 at_wait(&S.empty[s], ((n / kAtSlots) & 1u) ^ 1u, &S.abort));
+      if (!ok) break;
+      if (done) {
+        // one end marker for each warpgroup (and the issuing warp sees the first)
         if (lane == 0) S.info[s].done = 1;
-        tc::mbar_arrive(&S.full[s]);
+        tc::fence_async_smem();
         cp_async_arrive_noinc(&S.full[s]);
-        break;
+        tc::mbar_arrive(&S.full[s]);
+        if (++done_marks == 2) break;
+        t = t_end;  // stay done
+        continue;
       }
       AtInfo inf;
-      inf.done = done;
-      if (!done) {
-        const int k0 = 2 * t;
-        inf.r = r; inf.bh = bh; inf.t = t;
-        inf.first = (t == (int)((item % a.ipr) * a.tpi)) ? 1 : 0;
-        inf.last = (t + 1 == t_end) ? 1 : 0;
-        inf.nq = (k0 + 1 < a.n_chunks) ? 2 : 1;
-        inf.has_prev = a.n_chunks > 1 ? 1 : 0;
-        const size_t rowbase = ((size_t)r * a.BH + bh) * a.L;
-        const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
-        // window slot u in [0,192): chunk u/64 of (prev, k0, k0+1)
-        uint32_t pos[6];
-        bool present[6];
+      const int k0 = 2 * t;
+      inf.done = 0;
+      inf.r = r;
+      inf.bh = bh;
+      inf.t = t;
+      inf.first = (t == (int)((item % a.ipr) * a.tpi)) ? 1 : 0;
+      inf.last = (t + 1 == t_end) ? 1 : 0;
+      inf.nq = (k0 + 1 < a.n_chunks) ? 2 : 1;
+      inf.has_prev = a.n_chunks > 1 ? 1 : 0;
+      const size_t rowbase = ((size_t)r * a.BH + bh) * a.L;
+      const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
+      uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
+      const __nv_bfloat16* Qbh = a.Q + (size_t)bh * a.L * 64;
+      const __nv_bfloat16* Vbh = a.V + (size_t)bh * a.L * 64;
+      const float* rnbh = a.rn + (size_t)bh * a.L;
+      uint32_t pos[6];
 #pragma unroll
-        for (int e = 0; e < 6; ++e) {
-          const int u = lane + 32 * e;
-          const int cw = u >> 6;
-          const int ch = cw == 0 ? prev : k0 + cw - 1;
-          present[e] = (cw == 0) ? (inf.has_prev != 0) : (ch < a.n_chunks);
-          uint32_t p = 0;
-          if (present[e]) {
-            p = (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)];
-            if (p >= (uint32_t)a.L) { record_status(kErrBadKeys); p = 0; }
-          }
-          pos[e] = p;
+      for (int e = 0; e < 6; ++e) {  // window slot u = lane + 32e: chunk u/64 of (prev, k0, k0+1)
+        const int u = lane + 32 * e;
+        const int cw = u >> 6;
+        const int ch = cw == 0 ? prev : k0 + cw - 1;
+        const bool present = (cw == 0) ? (inf.has_prev != 0) : (ch < a.n_chunks);
+        uint32_t p = kAtNoKey;
+        if (present) {
+          p = (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)];
+          if (p >= (uint32_t)a.L) { record_status(kErrBadKeys); p = 0; }
         }
-        uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
-        const __nv_bfloat16* Qbh = a.Q + (size_t)bh * a.L * 64;
-        const __nv_bfloat16* Vbh = a.V + (size_t)bh * a.L * 64;
-#pragma unroll
-        for (int e = 0; e < 6; ++e) {
-          const int u = lane + 32 * e;
-          const int cw = u >> 6, row = u & 63;
-          S.pos[s][u] = pos[e];
-          S.key[s][u] = present[e] ? a.keys[rowbase + pos[e]] : kAtNoKey;
-          uint8_t* qd = slot + cw * kAtChunkBytes;
-          uint8_t* vd = slot + (3 + cw) * kAtChunkBytes;
-          if (present[e]) {
-            const __nv_bfloat16* qs = Qbh + (size_t)pos[e] * 64;
-            const __nv_bfloat16* vs = Vbh + (size_t)pos[e] * 64;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              tc::cp_async16(tc::smem_u32(qd + tc::sw128_offset(row, c)), qs + c * 8);
-              tc::cp_async16(tc::smem_u32(vd + tc::sw128_offset(row, c)), vs + c * 8);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              *reinterpret_cast<uint4*>(qd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4*>(vd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
-            }
-          }
-        }
-        if (lane == 0) S.info[s] = inf;
-        ++t;
-      } else if (lane == 0) {
-        S.info[s].done = 1;
+        pos[e] = p;
       }
+#pragma unroll
+      for (int e = 0; e < 6; ++e) {
+        const int u = lane + 32 * e;
+        const int cw = u >> 6, row = u & 63;
+        uint8_t* qd = slot + cw * kAtChunkBytes;
+        uint8_t* vd = slot + (3 + cw) * kAtChunkBytes;
+        if (pos[e] != kAtNoKey) {
+          S.pos[s][u] = pos[e];
+          cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + pos[e]);
+          cp_async4(tc::smem_u32(&S.rn[s][u]), rnbh + pos[e]);
+          const __nv_bfloat16* qs = Qbh + (size_t)pos[e] * 64;
+          const __nv_bfloat16* vs = Vbh + (size_t)pos[e] * 64;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            tc::cp_async16(tc::smem_u32(qd + tc::sw128_offset(row, c)), qs + c * 8);
+            tc::cp_async16(tc::smem_u32(vd + tc::sw128_offset(row, c)), vs + c * 8);
+          }
+        } else {
+          S.pos[s][u] = 0;
+          S.key[s][u] = kAtNoKey;
+          S.rn[s][u] = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            *reinterpret_cast<uint4*>(qd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      if (lane == 0) S.info[s] = inf;
+      ++t;
       tc::fence_async_smem();
       cp_async_arrive_noinc(&S.full[s]);
       tc::mbar_arrive(&S.full[s]);
-      s = (s + 1 == kAtSlots) ? 0 : s + 1;
-      if (done) break;
     }
-  } else {
-    // ------------------------------------------------------------ compute
-    const int wg = tid >> 7;      // which half of the row's window
-    const int m = tid & 127;      // query row = TMEM lane
-    const int qc = m >> 6;        // query chunk within the tile
-    const int kc = qc + wg;       // window chunk this thread scores
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t idesc_s = tc::idesc_bf16(128, 64, 0, 0);
-    const uint32_t idesc_o = tc::idesc_bf16(128, 64, 0, 1);
-    int s = 0;
-    uint32_t full_phase = 0;
-    uint32_t tile_n = 0;
-    for (;;) {
-      bool ok = tc::mbar_wait(&S.full[s], (full_phase >> s) & 1u);
-      full_phase ^= 1u << s;
-      if (consumers_or(!ok)) {
-        if (tid == 0) { record_status(tc::kErrTimeout); S.abort = 1; }
-        break;
-      }
-      const AtInfo inf = S.info[s];
-      if (consumers_or(inf.done || *(volatile int*)&S.abort)) break;
-      uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
-
-      // online mode: rounds of a head run in order
-      if (a.online && inf.first && inf.r > 0) {
-        bool waited = true;
-        if (tid == 0) {
-          const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
-          const long long t0 = clock64();
-          while (ld_acquire(c) < (unsigned)a.ipr) {
-            if (clock64() - t0 > tc::kSpinCycles) { waited = false; break; }
+  } else if (warp == 9) {
+    // ------------------------------------------------------ tensor-core issue
+    if (lane == 0) {
+      const uint32_t idesc_s = tc::idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc_o = tc::idesc_bf16(128, 64, 0, 1);
+      uint32_t n_s = 0, n_p = 0;  // next S to issue, next P.V to issue
+      bool s_done = false;
+      long long idle_since = clock64();
+      for (;;) {
+        bool progress = false;
+        if (!s_done && n_s <= n_p + 1) {
+          const int s = n_s % kAtSlots, w = n_s & 1;
+          if (tc::mbar_probe(&S.full[s], (n_s / kAtSlots) & 1u)) {
+            if (S.info[s].done) {
+              s_done = true;
+            } else if (tc::mbar_probe(&S.tm_free[w], ((n_s >> 1) & 1u) ^ 1u)) {
+              tc::fence_after_sync();
+              tc::fence_async_smem();  // cp.async rows of this slot -> tensor-core reads
+              uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
+              const uint32_t qa = tc::smem_u32(slot + kAtChunkBytes);  // chunks k0, k0+1
+              const uint32_t d = tmem + w * 256;
+#pragma unroll
+              for (int c = 0; c < 3; ++c) {
+                const uint32_t kb = tc::smem_u32(slot + c * kAtChunkBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  tc::mma_bf16(d + c * 64, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                               tc::sdesc_sw128(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+              }
+              tc::mma_commit(&S.s_full[w]);
+              ++n_s;
+              progress = true;
+            }
           }
         }
-        if (consumers_or(!waited)) {
-          if (tid == 0) { record_status(tc::kErrTimeout); S.abort = 1; }
-          break;
+        if (n_p < n_s) {
+          const int s = n_p % kAtSlots, w = n_p & 1;
+          if (tc::mbar_probe(&S.p_full[w], (n_p >> 1) & 1u)) {
+            tc::fence_after_sync();
+            uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
+            const uint32_t pa = tmem + w * 256;  // P over S: key block c at columns 32c
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+              const uint32_t vb = tc::smem_u32(slot + (3 + c) * kAtChunkBytes);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16_ts(tmem + w * 256 + 192, pa + c * 32 + kk * 8,
+                                tc::sdesc_sw128(vb + kk * 2048, 8192, 1024), idesc_o,
+                                (c | kk) != 0);
+            }
+            tc::mma_commit(&S.o_full[w]);
+            ++n_p;
+            progress = true;
+          }
+        }
+        if (s_done && n_p == n_s) break;
+        if (progress) {
+          idle_since = clock64();
+        } else {
+          if (*(volatile int*)&S.abort) break;
+          if (clock64() - idle_since > tc::kSpinCycles) {
+            record_status(tc::kErrTimeout);
+            *(volatile int*)&S.abort = 1;
+            break;
+          }
         }
       }
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------- softmax and epilogue
+    const int w = warp >> 2;            // warpgroup
+    const int m = tid & 127;            // query row = TMEM lane
+    const int qc = m >> 6;              // query chunk within the tile
+    const uint32_t region = tmem + (uint32_t)w * 256 + ((uint32_t)((warp & 3) * 32) << 16);
+    for (uint32_t j = 0;; ++j) {
+      const uint32_t n = (uint32_t)w + 2 * j;
+      const int s = n % kAtSlots;
+      const bool okf = at_wait(&S.full[s], (n / kAtSlots) & 1u, &S.abort);
+      const AtInfo inf = S.info[s];
+      if (wg_or(w, !okf || inf.done)) break;
 
-      // S = Q . K^T (three window chunks)
-      if (tid == 0) {
-        tc::fence_after_sync();
-        tc::fence_async_smem();  // cp.async rows of this slot -> tensor-core reads
-        const uint32_t qa = tc::smem_u32(slot + kAtChunkBytes);  // chunks k0, k0+1
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          const uint32_t kb = tc::smem_u32(slot + c * kAtChunkBytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + c * 64, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                         tc::sdesc_sw128(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+      if (a.online && inf.r > 0) {  // rounds of a head run in order
+        // every tile of round r-1 of this head must be folded in; the last
+        // (head, round) seen complete is cached so later tiles skip the load
+        bool waited = true;
+        if (m == 0 && !(S.dep_bh == inf.bh && S.dep_r == inf.r)) {
+          const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
+          const long long t0 = clock64();
+          while (ld_acquire(c) < (unsigned)a.n_tiles) {
+            if (*(volatile int*)&S.abort) { waited = false; break; }
+            if (clock64() - t0 > tc::kSpinCycles) {
+              record_status(tc::kErrTimeout);
+              *(volatile int*)&S.abort = 1;
+              waited = false;
+              break;
+            }
+          }
+          if (waited) { S.dep_bh = inf.bh; S.dep_r = inf.r; }
         }
-        tc::mma_commit(&S.bar_s);
+        if (wg_or(w, !waited)) break;
       }
 
       const bool valid = qc < inf.nq;
@@ -349,184 +439,173 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const uint32_t ki = S.key[s][64 + m];
       const size_t tok = (size_t)inf.bh * a.L + my_pos;
 
-      // online mode: fetch this row's running state early (L2, not L1)
-      float acc[32];
-      float2 ml = make_float2(0.f, 0.f);
-      if (a.online && inf.r > 0 && valid) {
-        const float4* src = reinterpret_cast<const float4*>(a.acc_o + tok * 64 + wg * 32);
+      // scores of this row's two window chunks (qc, qc + 1), 32 columns at a
+      // time.  Reference for the exponentials: the bound |q_i|/sqrt(d) on any
+      // score (keys are unit vectors) instead of the row maximum, so one pass
+      // suffices; a warp with a row whose bound exceeds kRefLimit (where
+      // exp(score - bound) could underflow) takes the exact two-pass route.
+      const bool oks = at_wait(&S.s_full[w], j & 1u, &S.abort);
+      if (wg_or(w, !oks)) break;
+      tc::fence_after_sync();
+      const uint32_t lo = ki - ki % (uint32_t)a.L;
+      const uint32_t span = a.causal ? (ki - lo) : (uint32_t)a.L;
+      const float rn_i = S.rn[s][64 + m];  // 1/(|q_i| sqrt d) in log2 units
+      const float bound = rn_i > 0.f ? 1.f / (64.f * rn_i * (1.f / kLog2e)) : 0.f;
+      const bool exact = __any_sync(0xffffffffu, bound > kRefLimit);
+      float ref2 = bound * kLog2e;  // reference in log2 units
+      // masked scores of 32 columns (log2 units), -inf where masked
+      auto masked = [&](int c, float* v) {
+        const int kc = qc + (c >> 1);
+        const bool active = valid && (kc != 0 || inf.has_prev);
+        const uint32_t* kw = &S.key[s][kc * 64 + 32 * (c & 1)];
+        const float* rw = &S.rn[s][kc * 64 + 32 * (c & 1)];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int jj = 0; jj < 32; jj += 4) {
+          const uint4 k4 = *reinterpret_cast<const uint4*>(kw + jj);
+          const float4 r4 = *reinterpret_cast<const float4*>(rw + jj);
+          const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
+          const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            bool in = active && (kj[x] - lo) < span;
+            if (!a.causal) in = in && kj[x] != ki;
+            v[jj + x] = in ? v[jj + x] * rj[x] : -INFINITY;
+          }
+        }
+      };
+      if (exact) {  // pass 1: masked scores back into S, exact row maximum
+        float mx2 = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tc::tmem_ld32(region + qc * 64 + 32 * c, v);
+          tc::tmem_ld_wait();
+          masked(c, v);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) mx2 = fmaxf(mx2, v[x]);
+          tc::tmem_st32(region + qc * 64 + 32 * c, reinterpret_cast<const uint32_t*>(v));
+        }
+        tc::tmem_st_wait();
+        ref2 = mx2 == -INFINITY ? 0.f : mx2;
+      }
+      float lsum = 0.f;
+      // P (bf16, two per column) over S: key block b at columns [32b, 32b+32);
+      // all of S is read before the first P column is written (32-column
+      // steps of S at qc*64 + 32c stay ahead of P at 32*qc + 16c).
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tc::tmem_ld32(region + qc * 64 + 32 * c, v);
+        tc::tmem_ld_wait();
+        if (!exact) masked(c, v);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float p0 = ex2(v[2 * x] - ref2);
+          const float p1 = ex2(v[2 * x + 1] - ref2);
+          lsum += p0 + p1;
+          pk[16 * (c & 1) + x] = pack_bf16(p0, p1);
+        }
+        if (c & 1) tc::tmem_st32(region + (qc + (c >> 1)) * 32, pk);
+      }
+#pragma unroll
+      for (int x = 0; x < 32; ++x) pk[x] = 0u;
+      tc::tmem_st32(region + (qc == 0 ? 2 : 0) * 32, pk);  // the block outside the window
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&S.p_full[w]);
+      const bool lone = !(lsum > 0.f);  // nothing but itself in this round
+      const float mx = ref2 * (1.f / kLog2e);
+
+      // running state of this row (online, rounds after the first)
+      float acc[64];
+      float2 ml = make_float2(0.f, 0.f);
+      const bool fold = a.online && inf.r > 0 && valid;
+      if (fold) {
+        const float4* src = reinterpret_cast<const float4*>(a.acc_o + tok * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
           const float4 f = __ldcg(src + q);
           acc[4 * q] = f.x; acc[4 * q + 1] = f.y; acc[4 * q + 2] = f.z; acc[4 * q + 3] = f.w;
         }
         ml = __ldcg(a.acc_ml + tok);
       }
 
-      // key scale 1 / (|q_j| sqrt(d)) of the 192 window rows
-      if (tid < 192) {
-        const uint8_t* qrow = slot + (tid >> 6) * kAtChunkBytes;
-        const int row = tid & 63;
-        float ssq = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(qrow + tc::sw128_offset(row, c));
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const float2 f = __bfloat1622float2(h[x]);
-            ssq = fmaf(f.x, f.x, ssq);
-            ssq = fmaf(f.y, f.y, ssq);
-          }
-        }
-        S.rn[tid] = ssq > 0.f ? rsqrtf(ssq) * 0.125f : 0.f;
-      }
-      consumers_sync();
-
-      bool okw = tc::mbar_wait(&S.bar_s, tile_n & 1u);
-      if (consumers_or(!okw)) {
-        if (tid == 0) { record_status(tc::kErrTimeout); S.abort = 1; }
-        break;
-      }
+      const bool oko = at_wait(&S.o_full[w], j & 1u, &S.abort);
+      if (wg_or(w, !oko)) break;
       tc::fence_after_sync();
 
-      // masked, scaled scores of this thread's 64 window columns
-      float sv[64];
-      tc::tmem_ld32(lane_addr + kc * 64, sv);
-      tc::tmem_ld32(lane_addr + kc * 64 + 32, sv + 32);
-      tc::tmem_ld_wait();
-      const bool active = valid && (kc != 0 || inf.has_prev);
-      const uint32_t lo = ki - ki % (uint32_t)a.L;
-      const uint32_t span = a.causal ? (ki - lo) : (uint32_t)a.L;
-      const uint32_t* kw = &S.key[s][kc * 64];
-      const float* rw = &S.rn[kc * 64];
-      float mloc = -INFINITY;
+      // this round's (max, sum); a row with nothing but itself takes its value
+      const float m_r = lone ? kSelfScore : mx;
+      const float l_r = lone ? 1.f : lsum;
+      float M = m_r, Lsum = l_r, ea = 0.f, eb = 1.f;
+      if (fold) {
+        M = fmaxf(ml.x, m_r);
+        ea = __expf(ml.x - M);
+        eb = __expf(m_r - M);
+        Lsum = ml.y * ea + l_r * eb;
+      }
+      const bool last_round = inf.r + 1 == a.R;
+      const float scale = !a.online ? 1.f / l_r : (last_round ? eb / Lsum : eb);
+      const float scale_acc = last_round ? ea / Lsum : ea;
+      // O in two 32-column halves (keeps the register footprint small)
 #pragma unroll
-      for (int j = 0; j < 64; j += 4) {
-        const uint4 k4 = *reinterpret_cast<const uint4*>(kw + j);
-        const float4 r4 = *reinterpret_cast<const float4*>(rw + j);
-        const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
-        const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          bool in = active && (kj[x] - lo) < span;
-          if (!a.causal) in = in && kj[x] != ki;
-          const float v = in ? sv[j + x] * rj[x] : -INFINITY;
-          sv[j + x] = v;
-          mloc = fmaxf(mloc, v);
+      for (int hh = 0; hh < 2; ++hh) {
+        float o[32];
+        tc::tmem_ld32(region + 192 + 32 * hh, o);
+        tc::tmem_ld_wait();
+        if (hh == 1) {  // this warpgroup's half of tensor memory is free again
+          tc::fence_before_sync();
+          tc::mbar_arrive(&S.tm_free[w]);
         }
-      }
-      S.red_max[wg][m] = mloc;
-      consumers_sync();
-      const float mrow = fmaxf(S.red_max[0][m], S.red_max[1][m]);
-      const bool lone = mrow == -INFINITY;  // nothing but itself in this round
-      const float mb = lone ? 0.f : mrow * kLog2e;
-      float lsum = 0.f;
-      uint8_t* pblk = pbuf + kc * 16384;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float p0 = ex2(fmaf(sv[8 * c + 2 * x], kLog2e, -mb));
-          const float p1 = ex2(fmaf(sv[8 * c + 2 * x + 1], kLog2e, -mb));
-          lsum += p0 + p1;
-          const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-          w[x] = *reinterpret_cast<const uint32_t*>(&b);
-        }
-        *reinterpret_cast<uint4*>(pblk + tc::sw128_offset(m, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      S.red_sum[wg][m] = lsum;
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      consumers_sync();
-      const float lrow = S.red_sum[0][m] + S.red_sum[1][m];
-
-      // O = P . V (192 keys)
-      if (tid == 0) {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          const uint32_t pa = tc::smem_u32(pbuf + c * 16384);
-          const uint32_t vb = tc::smem_u32(slot + (3 + c) * kAtChunkBytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + 192, tc::sdesc_sw128(pa + kk * 32, 16, 1024),
-                         tc::sdesc_sw128(vb + kk * 2048, 8192, 1024), idesc_o,
-                         (c | kk) != 0);
-        }
-        tc::mma_commit(&S.bar_o);
-      }
-      okw = tc::mbar_wait(&S.bar_o, tile_n & 1u);
-      if (consumers_or(!okw)) {
-        if (tid == 0) { record_status(tc::kErrTimeout); S.abort = 1; }
-        break;
-      }
-      tc::fence_after_sync();
-      float o[32];
-      tc::tmem_ld32(lane_addr + 192 + wg * 32, o);
-      tc::tmem_ld_wait();
-
-      if (valid) {
-        // this round: max m_r, sum l_r, unnormalised output o (or the lone case)
-        float m_r = mrow, l_r = lrow;
+        if (!valid) continue;
         if (lone) {
-          m_r = kSelfScore;
-          l_r = 1.f;
-          const __nv_bfloat16* vs = a.V + tok * 64 + wg * 32;
+          const __nv_bfloat16* vs = a.V + tok * 64 + 32 * hh;
 #pragma unroll
           for (int q = 0; q < 4; ++q) load8(vs + 8 * q, o + 8 * q);
         }
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          o[x] *= scale;
+          if (fold) o[x] = fmaf(acc[32 * hh + x], scale_acc, o[x]);
+        }
         if (!a.online) {
-          const size_t pr = (size_t)inf.r * n_tok + tok;
-          const float inv = 1.f / l_r;
-          float* dst = a.o_part + pr * 64 + wg * 32;
+          float4* dst = reinterpret_cast<float4*>(a.o_part + ((size_t)inf.r * n_tok + tok) * 64 + 32 * hh);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(dst + 4 * q) =
-                make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
-          if (wg == 0) a.lse_r[pr] = lone ? kSelfScore : m_r + logf(l_r);
+            dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        } else if (!last_round) {
+          float4* dst = reinterpret_cast<float4*>(a.acc_o + tok * 64 + 32 * hh);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            __stcg(dst + q, make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
         } else {
-          float M = m_r, Lsum = l_r;
-          if (inf.r > 0) {  // fold into the running state
-            M = fmaxf(ml.x, m_r);
-            const float ea = __expf(ml.x - M), eb = __expf(m_r - M);
-            Lsum = ml.y * ea + l_r * eb;
+          __nv_bfloat16* dst = a.O + tok * 64 + 32 * hh;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = fmaf(acc[x], ea, o[x] * eb);
-          }
-          if (inf.r + 1 < a.R) {
-            float4* dst = reinterpret_cast<float4*>(a.acc_o + tok * 64 + wg * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              __stcg(dst + q, make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
-            if (wg == 0) __stcg(a.acc_ml + tok, make_float2(M, Lsum));
-          } else {
-            const float inv = 1.f / Lsum;
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] *= inv;
-            __nv_bfloat16* dst = a.O + tok * 64 + wg * 32;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) store8(dst + 8 * q, o + 8 * q);
-            if (wg == 0 && a.lse) a.lse[tok] = M + logf(Lsum);
-          }
+          for (int q = 0; q < 4; ++q) store8(dst + 8 * q, o + 8 * q);
         }
       }
-      tc::fence_before_sync();
-      consumers_sync();
-      if (tid == 0) {
-        tc::mbar_arrive(&S.empty[s]);
-        if (a.online && inf.last) {
+      if (valid) {
+        if (!a.online)
+          a.lse_r[(size_t)inf.r * n_tok + tok] = lone ? kSelfScore : m_r + logf(l_r);
+        else if (!last_round)
+          __stcg(a.acc_ml + tok, make_float2(M, Lsum));
+        else if (a.lse)
+          a.lse[tok] = M + logf(Lsum);
+      }
+      tc::mbar_arrive(&S.empty[s]);
+      if (a.online && inf.r + 1 < a.R) {  // publish this tile of round r
+        if (wg_or(w, false)) break;       // all of its stores are issued
+        if (m == 0) {
           __threadfence();
           atomicAdd(a.counters + (size_t)inf.bh * a.R + inf.r, 1u);
         }
       }
-      s = (s + 1 == kAtSlots) ? 0 : s + 1;
-      ++tile_n;
     }
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+  if (warp == 9) tc::tmem_dealloc(tmem, 512);
 }
 
 }  // namespace lsh

@@ -85,11 +85,13 @@ size_t counters_bytes(const Dims& D) {
 // caller supplies.
 size_t attend_fwd_ws_bytes(const Dims& D, bool has_o_part, bool has_lse_r, bool has_O) {
   if (attend_tc_supported(D)) {
+    // counters, per-token key scale, then the running state or the partials
+    const size_t base = counters_bytes(D) + align_up(D.n_tok * sizeof(float));
     if (has_O && !has_o_part && !has_lse_r)  // online combine: running state per token
-      return counters_bytes(D) + align_up(D.n_tok * kHeadDim * sizeof(float)) +
+      return base + align_up(D.n_tok * kHeadDim * sizeof(float)) +
              align_up(D.n_tok * sizeof(float2));
     const size_t all = (size_t)D.R * D.n_tok;  // every round's partials
-    return counters_bytes(D) + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
+    return base + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
            (has_lse_r ? 0 : align_up(all * sizeof(float)));
   }
   if (!has_O) return 0;
@@ -233,6 +235,9 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   char* w = static_cast<char*>(ws);
   a.counters = reinterpret_cast<unsigned*>(w);
   w += counters_bytes(D);
+  float* rn = reinterpret_cast<float*>(w);
+  a.rn = rn;
+  w += align_up(D.n_tok * sizeof(float));
   a.acc_o = nullptr;
   a.acc_ml = nullptr;
   a.O = static_cast<__nv_bfloat16*>(O);
@@ -252,6 +257,8 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
     if (!a.lse_r) a.lse_r = reinterpret_cast<float*>(w);
   }
   if (cudaMemsetAsync(a.counters, 0, counters_bytes(D), st) != cudaSuccess) return LSH_ERR_CUDA;
+  lsh::key_scale_kernel<<<(unsigned)((D.n_tok + 255) / 256), 256, 0, st>>>(a.Q, D.n_tok, rn);
+  if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
   const size_t smem = lsh::attend_tc_smem_bytes();
   lsh_status s0 = allow_smem(lsh::attend_tc_kernel, smem);
   if (s0 != LSH_OK) return s0;

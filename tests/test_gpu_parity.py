@@ -271,3 +271,12 @@ def test_tensor_core_hash_exact_ties_take_lowest_index():
     # p_3 == -p_2: z_3 ties z_{half+2} and z_2 ties z_{half+3}; the lower index wins
     assert not np.isin(b, [half + 2, half + 3]).any()
     assert np.isin(b, [0, half, 2, 3]).any()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_large_norm_queries_take_the_exact_softmax(oracle, causal):
+    """Queries scaled by 100 (score bound |q|/sqrt(d) ~ 100): the tensor-core
+    softmax leaves the bound-referenced fast path for the exact two-pass one."""
+    inp = W.make_random(1, 2, 320, 64, 16, 2, torch.bfloat16, seed=77)
+    inp["Q"] = (inp["Q"].float() * 100).to(torch.bfloat16)
+    check_all(oracle, inp, 16, 64, causal)
