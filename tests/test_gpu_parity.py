@@ -94,10 +94,13 @@ def check_all(oracle, inp, nb, chunk, causal, heads=None):
     np.testing.assert_allclose(_np(g["lse_r"])[:, sl[0], sl[1]], lse_r, rtol=1e-6, atol=tol)
     np.testing.assert_allclose(_np(g["O"])[sl], O, rtol=0, atol=tol)
     np.testing.assert_allclose(_np(g["lse"])[sl], lse, rtol=1e-6, atol=tol)
-    # standalone combine of the GPU partials equals the fused epilogue
+    # standalone combine of the GPU partials equals the fused / online combine
+    # up to one output ulp (two fp32 summation orders can round to adjacent
+    # bf16 values: 2^-7 relative)
     Oc, lsec = L.lsh_combine(g["o_part"], g["lse_r"], g["Q"].dtype)
     torch.cuda.synchronize()
-    np.testing.assert_allclose(_np(Oc), _np(g["O"]), rtol=0, atol=tol / 4)
+    ulp = 2.0 ** -7 if g["Q"].dtype == torch.bfloat16 else 2.0 ** -20
+    np.testing.assert_allclose(_np(Oc), _np(g["O"]), rtol=ulp, atol=tol / 4)
     np.testing.assert_allclose(_np(lsec), _np(g["lse"]), rtol=1e-6, atol=1e-5)
     return g
 
