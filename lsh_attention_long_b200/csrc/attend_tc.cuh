@@ -59,10 +59,15 @@
 
 namespace lsh {
 
-constexpr int kAtSlots = 4;
+constexpr int kAtSlots = 3;
 constexpr int kAtThreads = 320;
 constexpr int kAtChunkBytes = 64 * 128;          // 64 rows of 128 B
 constexpr int kAtSlotBytes = 6 * kAtChunkBytes;  // q then v of 3 chunks
+// Per warpgroup, the running state of its tile's 128 rows (online mode),
+// staged by cp.async while the softmax runs: 64 fp32 per row (16-byte pieces
+// swizzled by row) and the (max, sum) pair padded to 16 bytes.
+constexpr int kAtAccBytes = 2 * 128 * 256;
+constexpr int kAtMlBytes = 2 * 128 * 16;
 constexpr uint32_t kAtNoKey = 0xffffffffu;       // never inside a bucket range
 constexpr float kLog2e = 1.4426950408889634f;
 // Largest score bound |q_i|/sqrt(d) used directly as the softmax reference:
@@ -94,7 +99,7 @@ struct AttnTcArgs {
   float* o_part;     // partial mode
   float* lse_r;
   float* acc_o;      // online mode: [n_tok][64] unnormalised output
-  float2* acc_ml;    // online mode: [n_tok] (running max, running sum)
+  float4* acc_ml;    // online mode: [n_tok] (running max, running sum, -, -)
   __nv_bfloat16* O;  // online mode, last round
   float* lse;
   unsigned* counters;  // [BH][R] tiles done; then one ticket counter
@@ -113,7 +118,7 @@ struct AtSmem {
 };
 
 __host__ __device__ inline size_t attend_tc_smem_bytes() {
-  return 1024 + (size_t)kAtSlots * kAtSlotBytes + sizeof(AtSmem);
+  return 1024 + (size_t)kAtSlots * kAtSlotBytes + kAtAccBytes + kAtMlBytes + sizeof(AtSmem);
 }
 
 // Named barrier (id 1 + w) over the 128 threads of warpgroup w; OR of pred.
@@ -204,7 +209,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* slots = sm;
-  AtSmem& S = *reinterpret_cast<AtSmem*>(sm + kAtSlots * kAtSlotBytes);
+  uint8_t* acc_s = sm + kAtSlots * kAtSlotBytes;
+  float4* ml_s = reinterpret_cast<float4*>(acc_s + kAtAccBytes);
+  AtSmem& S = *reinterpret_cast<AtSmem*>(acc_s + kAtAccBytes + kAtMlBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -236,79 +243,100 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    long long item = -1;
-    int r = 0, bh = 0, t = 0, t_end = 0;
+    // The next tile's ticket and perm entries are fetched one tile ahead so
+    // their latency overlaps the current tile's gathers.
+    struct Pt {
+      long long item;
+      int r, bh, t, t_end, done;
+    };
+    auto fetch_item = [&](Pt& p) {
+      long long tk = 0;
+      if (lane == 0) tk = (long long)atomicAdd(ticket_ctr, 1u);
+      tk = __shfl_sync(0xffffffffu, tk, 0);
+      if (tk >= a.n_items) {
+        p.done = 1;
+        return;
+      }
+      p.item = tk;
+      at_decode(a, tk, p.r, p.bh, p.t);
+      p.t_end = min(p.t + a.tpi, a.n_tiles);
+      p.done = 0;
+    };
+    // window slot u = lane + 32e: chunk u/64 of (prev, k0, k0+1); kAtNoKey if absent
+    auto load_pos = [&](const Pt& p, uint32_t* pos) {
+      const size_t rowbase = ((size_t)p.r * a.BH + p.bh) * a.L;
+      const int k0 = 2 * p.t;
+      const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
+#pragma unroll
+      for (int e = 0; e < 6; ++e) {
+        const int u = lane + 32 * e;
+        const int cw = u >> 6;
+        const int ch = cw == 0 ? prev : k0 + cw - 1;
+        const bool present = (cw == 0) ? (a.n_chunks > 1) : (ch < a.n_chunks);
+        pos[e] = present ? (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)] : kAtNoKey;
+      }
+    };
+    Pt nxt;
+    nxt.item = 0; nxt.r = 0; nxt.bh = 0; nxt.t = 0; nxt.t_end = 0; nxt.done = 0;
+    fetch_item(nxt);
+    uint32_t pos_n[6];
+    if (!nxt.done) load_pos(nxt, pos_n);
     int done_marks = 0;
     for (uint32_t n = 0;; ++n) {
       const int s = n % kAtSlots;
-      bool done = false;
-      if (t >= t_end) {  // next item
-        long long tk = 0;
-        if (lane == 0) tk = (long long)atomicAdd(ticket_ctr, 1u);
-        tk = __shfl_sync(0xffffffffu, tk, 0);
-        if (tk >= a.n_items) {
-          done = true;
-        } else {
-          item = tk;
-          at_decode(a, item, r, bh, t);
-          t_end = min(t + a.tpi, a.n_tiles);
-        }
+      const Pt cur = nxt;
+      uint32_t pos[6];
+#pragma unroll
+      for (int e = 0; e < 6; ++e) pos[e] = pos_n[e];
+      if (!cur.done) {
+        nxt.t = cur.t + 1;
+        if (nxt.t >= nxt.t_end) fetch_item(nxt);
+        if (!nxt.done) load_pos(nxt, pos_n);
       }
       const bool ok = __all_sync(0xffffffffu,
                                  at_wait(&S.empty[s], ((n / kAtSlots) & 1u) ^ 1u, &S.abort));
       if (!ok) break;
-      if (done) {
-        // one end marker for each warpgroup (and the issuing warp sees the first)
+      if (cur.done) {
+        // one end marker for each warpgroup (the issuing warp sees the first)
         if (lane == 0) S.info[s].done = 1;
         tc::fence_async_smem();
         cp_async_arrive_noinc(&S.full[s]);
         tc::mbar_arrive(&S.full[s]);
         if (++done_marks == 2) break;
-        t = t_end;  // stay done
         continue;
       }
       AtInfo inf;
-      const int k0 = 2 * t;
+      const int k0 = 2 * cur.t;
       inf.done = 0;
-      inf.r = r;
-      inf.bh = bh;
-      inf.t = t;
-      inf.first = (t == (int)((item % a.ipr) * a.tpi)) ? 1 : 0;
-      inf.last = (t + 1 == t_end) ? 1 : 0;
+      inf.r = cur.r;
+      inf.bh = cur.bh;
+      inf.t = cur.t;
+      inf.first = (cur.t == (int)((cur.item % a.ipr) * a.tpi)) ? 1 : 0;
+      inf.last = (cur.t + 1 == cur.t_end) ? 1 : 0;
       inf.nq = (k0 + 1 < a.n_chunks) ? 2 : 1;
       inf.has_prev = a.n_chunks > 1 ? 1 : 0;
-      const size_t rowbase = ((size_t)r * a.BH + bh) * a.L;
-      const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
+      const size_t rowbase = ((size_t)cur.r * a.BH + cur.bh) * a.L;
       uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
-      const __nv_bfloat16* Qbh = a.Q + (size_t)bh * a.L * 64;
-      const __nv_bfloat16* Vbh = a.V + (size_t)bh * a.L * 64;
-      const float* rnbh = a.rn + (size_t)bh * a.L;
-      uint32_t pos[6];
-#pragma unroll
-      for (int e = 0; e < 6; ++e) {  // window slot u = lane + 32e: chunk u/64 of (prev, k0, k0+1)
-        const int u = lane + 32 * e;
-        const int cw = u >> 6;
-        const int ch = cw == 0 ? prev : k0 + cw - 1;
-        const bool present = (cw == 0) ? (inf.has_prev != 0) : (ch < a.n_chunks);
-        uint32_t p = kAtNoKey;
-        if (present) {
-          p = (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)];
-          if (p >= (uint32_t)a.L) { record_status(kErrBadKeys); p = 0; }
-        }
-        pos[e] = p;
-      }
+      const __nv_bfloat16* Qbh = a.Q + (size_t)cur.bh * a.L * 64;
+      const __nv_bfloat16* Vbh = a.V + (size_t)cur.bh * a.L * 64;
+      const float* rnbh = a.rn + (size_t)cur.bh * a.L;
 #pragma unroll
       for (int e = 0; e < 6; ++e) {
         const int u = lane + 32 * e;
         const int cw = u >> 6, row = u & 63;
         uint8_t* qd = slot + cw * kAtChunkBytes;
         uint8_t* vd = slot + (3 + cw) * kAtChunkBytes;
-        if (pos[e] != kAtNoKey) {
-          S.pos[s][u] = pos[e];
-          cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + pos[e]);
-          cp_async4(tc::smem_u32(&S.rn[s][u]), rnbh + pos[e]);
-          const __nv_bfloat16* qs = Qbh + (size_t)pos[e] * 64;
-          const __nv_bfloat16* vs = Vbh + (size_t)pos[e] * 64;
+        uint32_t p = pos[e];
+        if (p != kAtNoKey && p >= (uint32_t)a.L) {  // not a permutation of the row
+          record_status(kErrBadKeys);
+          p = 0;
+        }
+        if (p != kAtNoKey) {
+          S.pos[s][u] = p;
+          cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + p);
+          cp_async4(tc::smem_u32(&S.rn[s][u]), rnbh + p);
+          const __nv_bfloat16* qs = Qbh + (size_t)p * 64;
+          const __nv_bfloat16* vs = Vbh + (size_t)p * 64;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             tc::cp_async16(tc::smem_u32(qd + tc::sw128_offset(row, c)), qs + c * 8);
@@ -326,7 +354,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         }
       }
       if (lane == 0) S.info[s] = inf;
-      ++t;
       tc::fence_async_smem();
       cp_async_arrive_noinc(&S.full[s]);
       tc::mbar_arrive(&S.full[s]);
@@ -390,6 +417,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         if (progress) {
           idle_since = clock64();
         } else {
+          __nanosleep(32);  // leave issue slots to the softmax warps on this SMSP
           if (*(volatile int*)&S.abort) break;
           if (clock64() - idle_since > tc::kSpinCycles) {
             record_status(tc::kErrTimeout);
@@ -439,7 +467,20 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const uint32_t ki = S.key[s][64 + m];
       const size_t tok = (size_t)inf.bh * a.L + my_pos;
 
-      // scores of this row's two window chunks (qc, qc + 1), 32 columns at a
+      // running state of this row (online, rounds after the first): staged
+      // into shared memory by cp.async while the softmax runs
+      const bool fold = a.online && inf.r > 0 && valid;
+      uint8_t* my_acc = acc_s + (size_t)(w * 128 + m) * 256;
+      if (fold) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.acc_o + tok * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          tc::cp_async16(tc::smem_u32(my_acc + ((q ^ (m & 15)) << 4)), src + 16 * q);
+        tc::cp_async16(tc::smem_u32(&ml_s[w * 128 + m]), a.acc_ml + tok);
+      }
+      tc::cp_async_commit();
+
+      // scores of this row's two window chunks (qc, qc + 1), 64 columns at a
       // time.  Reference for the exponentials: the bound |q_i|/sqrt(d) on any
       // score (keys are unit vectors) instead of the row maximum, so one pass
       // suffices; a warp with a row whose bound exceeds kRefLimit (where
@@ -449,18 +490,19 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       tc::fence_after_sync();
       const uint32_t lo = ki - ki % (uint32_t)a.L;
       const uint32_t span = a.causal ? (ki - lo) : (uint32_t)a.L;
-      const float rn_i = S.rn[s][64 + m];  // 1/(|q_i| sqrt d) in log2 units
+      const float rn_i = S.rn[s][64 + m];  // log2(e)/(|q_i| sqrt d)
       const float bound = rn_i > 0.f ? 1.f / (64.f * rn_i * (1.f / kLog2e)) : 0.f;
       const bool exact = __any_sync(0xffffffffu, bound > kRefLimit);
       float ref2 = bound * kLog2e;  // reference in log2 units
-      // masked scores of 32 columns (log2 units), -inf where masked
-      auto masked = [&](int c, float* v) {
-        const int kc = qc + (c >> 1);
+      // masked scores (log2 units, -inf where masked) of the 64 columns of
+      // window chunk kc = qc + pp
+      auto masked = [&](int pp, float* v) {
+        const int kc = qc + pp;
         const bool active = valid && (kc != 0 || inf.has_prev);
-        const uint32_t* kw = &S.key[s][kc * 64 + 32 * (c & 1)];
-        const float* rw = &S.rn[s][kc * 64 + 32 * (c & 1)];
+        const uint32_t* kw = &S.key[s][kc * 64];
+        const float* rw = &S.rn[s][kc * 64];
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 4) {
+        for (int jj = 0; jj < 64; jj += 4) {
           const uint4 k4 = *reinterpret_cast<const uint4*>(kw + jj);
           const float4 r4 = *reinterpret_cast<const float4*>(rw + jj);
           const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
@@ -476,64 +518,59 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       if (exact) {  // pass 1: masked scores back into S, exact row maximum
         float mx2 = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tc::tmem_ld32(region + qc * 64 + 32 * c, v);
+        for (int pp = 0; pp < 2; ++pp) {
+          float v[64];
+          tc::tmem_ld32(region + qc * 64 + 64 * pp, v);
+          tc::tmem_ld32(region + qc * 64 + 64 * pp + 32, v + 32);
           tc::tmem_ld_wait();
-          masked(c, v);
+          masked(pp, v);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) mx2 = fmaxf(mx2, v[x]);
-          tc::tmem_st32(region + qc * 64 + 32 * c, reinterpret_cast<const uint32_t*>(v));
+          for (int x = 0; x < 64; ++x) mx2 = fmaxf(mx2, v[x]);
+          tc::tmem_st32(region + qc * 64 + 64 * pp, reinterpret_cast<const uint32_t*>(v));
+          tc::tmem_st32(region + qc * 64 + 64 * pp + 32, reinterpret_cast<const uint32_t*>(v + 32));
         }
         tc::tmem_st_wait();
         ref2 = mx2 == -INFINITY ? 0.f : mx2;
       }
       float lsum = 0.f;
-      // P (bf16, two per column) over S: key block b at columns [32b, 32b+32);
-      // all of S is read before the first P column is written (32-column
-      // steps of S at qc*64 + 32c stay ahead of P at 32*qc + 16c).
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tc::tmem_ld32(region + qc * 64 + 32 * c, v);
+      // P (bf16, two per column) over S: key block b at columns [32b, 32b+32).
+      // Window chunk qc + pp (S columns qc*64 + 64pp) becomes P block qc + pp
+      // (columns 32(qc + pp)); each step reads its S columns before writing,
+      // and never writes columns a later step still reads.
+#pragma unroll 1
+      for (int pp = 0; pp < 2; ++pp) {
+        float v[64];
+        tc::tmem_ld32(region + qc * 64 + 64 * pp, v);
+        tc::tmem_ld32(region + qc * 64 + 64 * pp + 32, v + 32);
         tc::tmem_ld_wait();
-        if (!exact) masked(c, v);
+        if (!exact) masked(pp, v);
+        uint32_t pk[32];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
+        for (int x = 0; x < 32; ++x) {
           const float p0 = ex2(v[2 * x] - ref2);
           const float p1 = ex2(v[2 * x + 1] - ref2);
           lsum += p0 + p1;
-          pk[16 * (c & 1) + x] = pack_bf16(p0, p1);
+          pk[x] = pack_bf16(p0, p1);
         }
-        if (c & 1) tc::tmem_st32(region + (qc + (c >> 1)) * 32, pk);
+        tc::tmem_st32(region + (qc + pp) * 32, pk);
       }
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int x = 0; x < 32; ++x) pk[x] = 0u;
-      tc::tmem_st32(region + (qc == 0 ? 2 : 0) * 32, pk);  // the block outside the window
+        for (int x = 0; x < 32; ++x) pk[x] = 0u;
+        tc::tmem_st32(region + (qc == 0 ? 2 : 0) * 32, pk);  // the block outside the window
+      }
       tc::tmem_st_wait();
       tc::fence_before_sync();
       tc::mbar_arrive(&S.p_full[w]);
       const bool lone = !(lsum > 0.f);  // nothing but itself in this round
       const float mx = ref2 * (1.f / kLog2e);
 
-      // running state of this row (online, rounds after the first)
-      float acc[64];
-      float2 ml = make_float2(0.f, 0.f);
-      const bool fold = a.online && inf.r > 0 && valid;
-      if (fold) {
-        const float4* src = reinterpret_cast<const float4*>(a.acc_o + tok * 64);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float4 f = __ldcg(src + q);
-          acc[4 * q] = f.x; acc[4 * q + 1] = f.y; acc[4 * q + 2] = f.z; acc[4 * q + 3] = f.w;
-        }
-        ml = __ldcg(a.acc_ml + tok);
-      }
-
       const bool oko = at_wait(&S.o_full[w], j & 1u, &S.abort);
       if (wg_or(w, !oko)) break;
       tc::fence_after_sync();
+      tc::cp_async_wait<0>();  // this thread's staged running state has landed
+      const float4 ml = fold ? ml_s[w * 128 + m] : make_float4(0.f, 0.f, 0.f, 0.f);
 
       // this round's (max, sum); a row with nothing but itself takes its value
       const float m_r = lone ? kSelfScore : mx;
@@ -565,9 +602,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
           for (int q = 0; q < 4; ++q) load8(vs + 8 * q, o + 8 * q);
         }
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          o[x] *= scale;
-          if (fold) o[x] = fmaf(acc[32 * hh + x], scale_acc, o[x]);
+        for (int x = 0; x < 32; ++x) o[x] *= scale;
+        if (fold) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 f = *reinterpret_cast<const float4*>(my_acc + (((8 * hh + q) ^ (m & 15)) << 4));
+            o[4 * q] = fmaf(f.x, scale_acc, o[4 * q]);
+            o[4 * q + 1] = fmaf(f.y, scale_acc, o[4 * q + 1]);
+            o[4 * q + 2] = fmaf(f.z, scale_acc, o[4 * q + 2]);
+            o[4 * q + 3] = fmaf(f.w, scale_acc, o[4 * q + 3]);
+          }
         }
         if (!a.online) {
           float4* dst = reinterpret_cast<float4*>(a.o_part + ((size_t)inf.r * n_tok + tok) * 64 + 32 * hh);
@@ -589,7 +633,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         if (!a.online)
           a.lse_r[(size_t)inf.r * n_tok + tok] = lone ? kSelfScore : m_r + logf(l_r);
         else if (!last_round)
-          __stcg(a.acc_ml + tok, make_float2(M, Lsum));
+          __stcg(a.acc_ml + tok, make_float4(M, Lsum, 0.f, 0.f));
         else if (a.lse)
           a.lse[tok] = M + logf(Lsum);
       }

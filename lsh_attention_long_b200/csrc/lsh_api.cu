@@ -89,7 +89,7 @@ size_t attend_fwd_ws_bytes(const Dims& D, bool has_o_part, bool has_lse_r, bool 
     const size_t base = counters_bytes(D) + align_up(D.n_tok * sizeof(float));
     if (has_O && !has_o_part && !has_lse_r)  // online combine: running state per token
       return base + align_up(D.n_tok * kHeadDim * sizeof(float)) +
-             align_up(D.n_tok * sizeof(float2));
+             align_up(D.n_tok * sizeof(float4));
     const size_t all = (size_t)D.R * D.n_tok;  // every round's partials
     return base + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
            (has_lse_r ? 0 : align_up(all * sizeof(float)));
@@ -247,7 +247,7 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   if (online) {
     a.acc_o = reinterpret_cast<float*>(w);
     w += align_up(D.n_tok * kHeadDim * sizeof(float));
-    a.acc_ml = reinterpret_cast<float2*>(w);
+    a.acc_ml = reinterpret_cast<float4*>(w);
   } else {
     const size_t all = (size_t)D.R * D.n_tok;
     if (!a.o_part) {
