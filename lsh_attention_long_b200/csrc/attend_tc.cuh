@@ -320,12 +320,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const __nv_bfloat16* Qbh = a.Q + (size_t)cur.bh * a.L * 64;
       const __nv_bfloat16* Vbh = a.V + (size_t)cur.bh * a.L * 64;
       const float* rnbh = a.rn + (size_t)cur.bh * a.L;
+      // slot metadata, lane-per-row: position, packed key, key scale
 #pragma unroll
       for (int e = 0; e < 6; ++e) {
         const int u = lane + 32 * e;
-        const int cw = u >> 6, row = u & 63;
-        uint8_t* qd = slot + cw * kAtChunkBytes;
-        uint8_t* vd = slot + (3 + cw) * kAtChunkBytes;
         uint32_t p = pos[e];
         if (p != kAtNoKey && p >= (uint32_t)a.L) {  // not a permutation of the row
           record_status(kErrBadKeys);
@@ -335,24 +333,34 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
           S.pos[s][u] = p;
           cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + p);
           cp_async4(tc::smem_u32(&S.rn[s][u]), rnbh + p);
-          const __nv_bfloat16* qs = Qbh + (size_t)p * 64;
-          const __nv_bfloat16* vs = Vbh + (size_t)p * 64;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            tc::cp_async16(tc::smem_u32(qd + tc::sw128_offset(row, c)), qs + c * 8);
-            tc::cp_async16(tc::smem_u32(vd + tc::sw128_offset(row, c)), vs + c * 8);
-          }
         } else {
-          S.pos[s][u] = 0;
+          S.pos[s][u] = kAtNoKey;
           S.key[s][u] = kAtNoKey;
           S.rn[s][u] = 0.f;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(qd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(vd + tc::sw128_offset(row, c)) = make_uint4(0, 0, 0, 0);
-          }
         }
       }
+      __syncwarp();
+      // q and v rows, eight lanes per 128-byte row (coalesced per row): four
+      // rows per warp instruction instead of 32 scattered 16-byte pieces
+#pragma unroll 4
+      for (int i = 0; i < 48; ++i) {
+        const int u = 4 * i + (lane >> 3), c = lane & 7;
+        const int cw = u >> 6, row = u & 63;
+        uint8_t* qd = slot + cw * kAtChunkBytes + tc::sw128_offset(row, c);
+        uint8_t* vd = slot + (3 + cw) * kAtChunkBytes + tc::sw128_offset(row, c);
+        const uint32_t p = S.pos[s][u];
+        if (p != kAtNoKey) {
+          tc::cp_async16(tc::smem_u32(qd), Qbh + (size_t)p * 64 + c * 8);
+          tc::cp_async16(tc::smem_u32(vd), Vbh + (size_t)p * 64 + c * 8);
+        } else {
+          *reinterpret_cast<uint4*>(qd) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < 6; ++e)  // absent rows read as position 0 downstream
+        if (S.pos[s][lane + 32 * e] == kAtNoKey) S.pos[s][lane + 32 * e] = 0;
       if (lane == 0) S.info[s] = inf;
       tc::fence_async_smem();
       cp_async_arrive_noinc(&S.full[s]);
@@ -433,7 +441,21 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
     const int w = warp >> 2;            // warpgroup
     const int m = tid & 127;            // query row = TMEM lane
     const int qc = m >> 6;              // query chunk within the tile
-    const uint32_t region = tmem + (uint32_t)w * 256 + ((uint32_t)((warp & 3) * 32) << 16);
+    const int wrow0 = (warp & 3) * 32;  // first row of this warp
+    const uint32_t region = tmem + (uint32_t)w * 256 + ((uint32_t)wrow0 << 16);
+    uint8_t* wg_acc = acc_s + (size_t)w * 128 * 256;  // this warpgroup's staging rows
+    // online mode: this warpgroup's last tile whose completion is not yet
+    // counted; it is published (fence + counter) once its stores are old,
+    // before a dependency wait, and at exit -- a fence right after the
+    // stores would stall the warpgroup for their whole latency
+    int pend_bh = -1, pend_r = 0;
+    auto publish = [&]() {
+      if (pend_bh >= 0 && m == 0) {
+        __threadfence();
+        atomicAdd(a.counters + (size_t)pend_bh * a.R + pend_r, 1u);
+      }
+      pend_bh = -1;
+    };
     for (uint32_t j = 0;; ++j) {
       const uint32_t n = (uint32_t)w + 2 * j;
       const int s = n % kAtSlots;
@@ -445,37 +467,42 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         // every tile of round r-1 of this head must be folded in; the last
         // (head, round) seen complete is cached so later tiles skip the load
         bool waited = true;
-        if (m == 0 && !(S.dep_bh == inf.bh && S.dep_r == inf.r)) {
-          const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
-          const long long t0 = clock64();
-          while (ld_acquire(c) < (unsigned)a.n_tiles) {
-            if (*(volatile int*)&S.abort) { waited = false; break; }
-            if (clock64() - t0 > tc::kSpinCycles) {
-              record_status(tc::kErrTimeout);
-              *(volatile int*)&S.abort = 1;
-              waited = false;
-              break;
+        if (!(S.dep_bh == inf.bh && S.dep_r == inf.r)) {
+          publish();  // never wait while holding an unpublished tile
+          if (m == 0) {
+            const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
+            const long long t0 = clock64();
+            while (ld_acquire(c) < (unsigned)a.n_tiles) {
+              if (*(volatile int*)&S.abort) { waited = false; break; }
+              if (clock64() - t0 > tc::kSpinCycles) {
+                record_status(tc::kErrTimeout);
+                *(volatile int*)&S.abort = 1;
+                waited = false;
+                break;
+              }
             }
+            if (waited) { S.dep_bh = inf.bh; S.dep_r = inf.r; }
           }
-          if (waited) { S.dep_bh = inf.bh; S.dep_r = inf.r; }
         }
         if (wg_or(w, !waited)) break;
       }
 
       const bool valid = qc < inf.nq;
-      const uint32_t my_pos = S.pos[s][64 + m];
       const uint32_t ki = S.key[s][64 + m];
-      const size_t tok = (size_t)inf.bh * a.L + my_pos;
+      const size_t tok = (size_t)inf.bh * a.L + S.pos[s][64 + m];
+      const size_t bhL = (size_t)inf.bh * a.L;
+      const bool fold = a.online && inf.r > 0 && valid;  // uniform per warp
 
-      // running state of this row (online, rounds after the first): staged
-      // into shared memory by cp.async while the softmax runs
-      const bool fold = a.online && inf.r > 0 && valid;
-      uint8_t* my_acc = acc_s + (size_t)(w * 128 + m) * 256;
+      // running state of this warp's 32 rows: staged by cp.async while the
+      // softmax runs, sixteen lanes per 256-byte row
       if (fold) {
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.acc_o + tok * 64);
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          tc::cp_async16(tc::smem_u32(my_acc + ((q ^ (m & 15)) << 4)), src + 16 * q);
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
+          const size_t t2 = bhL + S.pos[s][64 + rr];
+          tc::cp_async16(tc::smem_u32(wg_acc + (size_t)rr * 256 + ((q ^ (rr & 15)) << 4)),
+                         a.acc_o + t2 * 64 + 4 * q);
+        }
         tc::cp_async16(tc::smem_u32(&ml_s[w * 128 + m]), a.acc_ml + tok);
       }
       tc::cp_async_commit();
@@ -532,7 +559,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         tc::tmem_st_wait();
         ref2 = mx2 == -INFINITY ? 0.f : mx2;
       }
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
       // P (bf16, two per column) over S: key block b at columns [32b, 32b+32).
       // Window chunk qc + pp (S columns qc*64 + 64pp) becomes P block qc + pp
       // (columns 32(qc + pp)); each step reads its S columns before writing,
@@ -549,7 +576,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         for (int x = 0; x < 32; ++x) {
           const float p0 = ex2(v[2 * x] - ref2);
           const float p1 = ex2(v[2 * x + 1] - ref2);
-          lsum += p0 + p1;
+          ls[x & 3] += p0 + p1;
           pk[x] = pack_bf16(p0, p1);
         }
         tc::tmem_st32(region + (qc + pp) * 32, pk);
@@ -563,13 +590,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       tc::tmem_st_wait();
       tc::fence_before_sync();
       tc::mbar_arrive(&S.p_full[w]);
+      const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       const bool lone = !(lsum > 0.f);  // nothing but itself in this round
       const float mx = ref2 * (1.f / kLog2e);
 
       const bool oko = at_wait(&S.o_full[w], j & 1u, &S.abort);
       if (wg_or(w, !oko)) break;
       tc::fence_after_sync();
-      tc::cp_async_wait<0>();  // this thread's staged running state has landed
+      publish();               // the previous tile's stores are long issued
+      tc::cp_async_wait<0>();  // this lane's staged pieces have landed
+      __syncwarp();            // ... and the other lanes' (rows are shared)
       const float4 ml = fold ? ml_s[w * 128 + m] : make_float4(0.f, 0.f, 0.f, 0.f);
 
       // this round's (max, sum); a row with nothing but itself takes its value
@@ -583,9 +613,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         Lsum = ml.y * ea + l_r * eb;
       }
       const bool last_round = inf.r + 1 == a.R;
+      const bool out_bf16 = a.online && last_round;
       const float scale = !a.online ? 1.f / l_r : (last_round ? eb / Lsum : eb);
       const float scale_acc = last_round ? ea / Lsum : ea;
-      // O in two 32-column halves (keeps the register footprint small)
+      uint8_t* my_row = wg_acc + (size_t)m * 256;
+      // O in two 32-column halves; the result goes back into this row's
+      // staging space (fp32, or bf16 for the final output)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float o[32];
@@ -603,30 +636,32 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         }
 #pragma unroll
         for (int x = 0; x < 32; ++x) o[x] *= scale;
-        if (fold) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 f = *reinterpret_cast<const float4*>(my_acc + (((8 * hh + q) ^ (m & 15)) << 4));
+        for (int q = 0; q < 8; ++q) {
+          uint8_t* piece = my_row + (((8 * hh + q) ^ (m & 15)) << 4);
+          if (fold) {
+            const float4 f = *reinterpret_cast<const float4*>(piece);
             o[4 * q] = fmaf(f.x, scale_acc, o[4 * q]);
             o[4 * q + 1] = fmaf(f.y, scale_acc, o[4 * q + 1]);
             o[4 * q + 2] = fmaf(f.z, scale_acc, o[4 * q + 2]);
             o[4 * q + 3] = fmaf(f.w, scale_acc, o[4 * q + 3]);
           }
+          if (!out_bf16)
+            *reinterpret_cast<float4*>(piece) =
+                make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         }
-        if (!a.online) {
-          float4* dst = reinterpret_cast<float4*>(a.o_part + ((size_t)inf.r * n_tok + tok) * 64 + 32 * hh);
+        if (out_bf16) {  // 64 B of bf16 per half: pieces 4hh .. 4hh+3 of a 128-B row
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        } else if (!last_round) {
-          float4* dst = reinterpret_cast<float4*>(a.acc_o + tok * 64 + 32 * hh);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            __stcg(dst + q, make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
-        } else {
-          __nv_bfloat16* dst = a.O + tok * 64 + 32 * hh;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) store8(dst + 8 * q, o + 8 * q);
+          for (int q = 0; q < 4; ++q) {
+            uint4 b;
+            b.x = pack_bf16(o[8 * q], o[8 * q + 1]);
+            b.y = pack_bf16(o[8 * q + 2], o[8 * q + 3]);
+            b.z = pack_bf16(o[8 * q + 4], o[8 * q + 5]);
+            b.w = pack_bf16(o[8 * q + 6], o[8 * q + 7]);
+            // bf16 rows live in the second half of the staging row, so the
+            // fp32 pieces the other half still reads are not overwritten
+            *reinterpret_cast<uint4*>(my_row + 128 + (((4 * hh + q) ^ (m & 7)) << 4)) = b;
+          }
         }
       }
       if (valid) {
@@ -637,15 +672,42 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         else if (a.lse)
           a.lse[tok] = M + logf(Lsum);
       }
-      tc::mbar_arrive(&S.empty[s]);
-      if (a.online && inf.r + 1 < a.R) {  // publish this tile of round r
-        if (wg_or(w, false)) break;       // all of its stores are issued
-        if (m == 0) {
-          __threadfence();
-          atomicAdd(a.counters + (size_t)inf.bh * a.R + inf.r, 1u);
+      __syncwarp();
+      // the warp's 32 result rows to their original positions, coalesced
+      // per row: fp32 rows by sixteen lanes (256 B), bf16 rows by eight (128 B)
+      if (valid) {
+        if (!out_bf16) {
+          float* base = !a.online ? a.o_part + (size_t)inf.r * n_tok * 64 : a.acc_o;
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
+            const size_t t2 = bhL + S.pos[s][64 + rr];
+            const float4 f =
+                *reinterpret_cast<const float4*>(wg_acc + (size_t)rr * 256 + ((q ^ (rr & 15)) << 4));
+            if (!a.online) *reinterpret_cast<float4*>(base + t2 * 64 + 4 * q) = f;
+            else __stcg(reinterpret_cast<float4*>(base + t2 * 64 + 4 * q), f);
+          }
+        } else {
+#pragma unroll 4
+          for (int i = 0; i < 8; ++i) {
+            const int rr = wrow0 + 4 * i + (lane >> 3), q = lane & 7;
+            const size_t t2 = bhL + S.pos[s][64 + rr];
+            const uint4 b = *reinterpret_cast<const uint4*>(wg_acc + (size_t)rr * 256 + 128 +
+                                                            ((q ^ (rr & 7)) << 4));
+            *reinterpret_cast<uint4*>(a.O + t2 * 64 + 8 * q) = b;
+          }
         }
       }
+      tc::mbar_arrive(&S.empty[s]);
+      if (a.online && !last_round) {
+        pend_bh = inf.bh;
+        pend_r = inf.r;
+      }
     }
+    // stores of the last tile: every thread's are ordered before thread 0's
+    // fence by this barrier
+    wg_or(w, false);
+    publish();
   }
   tc::fence_before_sync();
   __syncthreads();
