@@ -658,9 +658,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             b.y = pack_bf16(o[8 * q + 2], o[8 * q + 3]);
             b.z = pack_bf16(o[8 * q + 4], o[8 * q + 5]);
             b.w = pack_bf16(o[8 * q + 6], o[8 * q + 7]);
-            // bf16 rows live in the second half of the staging row, so the
-            // fp32 pieces the other half still reads are not overwritten
-            *reinterpret_cast<uint4*>(my_row + 128 + (((4 * hh + q) ^ (m & 7)) << 4)) = b;
+            // bf16 piece 4hh+q takes the place of fp32 piece 4hh+q, which
+            // the first half (hh = 0) has already read; the pieces the
+            // second half still reads (8..15) are not touched
+            *reinterpret_cast<uint4*>(my_row + (((4 * hh + q) ^ (m & 15)) << 4)) = b;
           }
         }
       }
@@ -692,8 +693,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
           for (int i = 0; i < 8; ++i) {
             const int rr = wrow0 + 4 * i + (lane >> 3), q = lane & 7;
             const size_t t2 = bhL + S.pos[s][64 + rr];
-            const uint4 b = *reinterpret_cast<const uint4*>(wg_acc + (size_t)rr * 256 + 128 +
-                                                            ((q ^ (rr & 7)) << 4));
+            const uint4 b = *reinterpret_cast<const uint4*>(wg_acc + (size_t)rr * 256 +
+                                                            ((q ^ (rr & 15)) << 4));
             *reinterpret_cast<uint4*>(a.O + t2 * 64 + 8 * q) = b;
           }
         }
