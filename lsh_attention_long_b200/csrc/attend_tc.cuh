@@ -27,7 +27,7 @@
 // own entry enters only when a row has no other key in its round's window:
 // then the round's output is its own value and lse = -1e5.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3, 4-7  two softmax/epilogue warpgroups; warpgroup w takes the
 //                   CTA's tiles w, w+2, w+4, ... so one warpgroup's softmax
 //                   overlaps the other's MMAs and epilogue.  Each owns half of
@@ -39,6 +39,8 @@
 //   warp 9          tensor-core issue: one thread polls the barriers and
 //                   issues S for tile n+1 as soon as its data and TMEM half
 //                   are free, and P.V for tile n as soon as P is written.
+//   warp 10         publisher (online mode): fences and counts finished
+//                   tiles so the compute warps never wait on store latency.
 //
 // Two output modes:
 //   partial  every round's normalised o_r (fp32) and lse_r go to o_part /
@@ -60,7 +62,8 @@
 namespace lsh {
 
 constexpr int kAtSlots = 3;
-constexpr int kAtThreads = 320;
+constexpr int kAtThreads = 352;
+constexpr int kAtPubRing = 16;
 constexpr int kAtChunkBytes = 64 * 128;          // 64 rows of 128 B
 constexpr int kAtSlotBytes = 6 * kAtChunkBytes;  // q then v of 3 chunks
 // Per warpgroup, the running state of its tile's 128 rows (online mode),
@@ -112,6 +115,13 @@ struct AtSmem {
   AtInfo info[kAtSlots];
   uint64_t full[kAtSlots], empty[kAtSlots];
   uint64_t s_full[2], p_full[2], o_full[2], tm_free[2];
+  uint32_t perm_stage[kAtSlots][192];  // perm entries of the tile two ahead
+  // completion ring (online mode): compute warpgroups post finished tiles,
+  // the publisher warp makes them visible and counts them
+  int pub_bh[kAtPubRing], pub_r[kAtPubRing];
+  unsigned pub_seq[kAtPubRing];
+  unsigned pub_head;  // tiles published so far
+  unsigned n_total;   // tiles this CTA will process (set when known)
   uint32_t tmem_base;
   int abort;
   int dep_bh, dep_r;  // last (head, round) whose previous round was seen complete
@@ -150,6 +160,14 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+__device__ __forceinline__ unsigned ld_acquire_cta(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(tc::smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(unsigned* p, unsigned v) {
+  asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(tc::smem_u32(p)), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -229,6 +247,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
     S.abort = 0;
     S.dep_bh = -1;
     S.dep_r = -1;
+    S.pub_head = 0;
+    S.n_total = 0xffffffffu;
+    for (int i = 0; i < kAtPubRing; ++i) S.pub_seq[i] = 0;
   }
   if (warp == 9) {
     tc::tmem_alloc(&S.tmem_base, 512);
@@ -243,16 +264,18 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    // The next tile's ticket and perm entries are fetched one tile ahead so
-    // their latency overlaps the current tile's gathers.
+    // The perm entries of tile n+2 are staged (cp.async) while tile n is
+    // gathered, and the ticket of the next item is fetched one item ahead,
+    // so neither latency sits on the gather path.
     struct Pt {
       long long item;
       int r, bh, t, t_end, done;
     };
-    auto fetch_item = [&](Pt& p) {
-      long long tk = 0;
-      if (lane == 0) tk = (long long)atomicAdd(ticket_ctr, 1u);
-      tk = __shfl_sync(0xffffffffu, tk, 0);
+    long long tk_pending = 0;  // lane 0: the ticket reserved for the next item
+    if (lane == 0) tk_pending = (long long)atomicAdd(ticket_ctr, 1u);
+    auto next_item = [&](Pt& p) {
+      const long long tk = __shfl_sync(0xffffffffu, tk_pending, 0);
+      if (lane == 0 && tk < a.n_items) tk_pending = (long long)atomicAdd(ticket_ctr, 1u);
       if (tk >= a.n_items) {
         p.done = 1;
         return;
@@ -262,49 +285,65 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       p.t_end = min(p.t + a.tpi, a.n_tiles);
       p.done = 0;
     };
-    // window slot u = lane + 32e: chunk u/64 of (prev, k0, k0+1); kAtNoKey if absent
-    auto load_pos = [&](const Pt& p, uint32_t* pos) {
-      const size_t rowbase = ((size_t)p.r * a.BH + p.bh) * a.L;
-      const int k0 = 2 * p.t;
-      const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
-#pragma unroll
-      for (int e = 0; e < 6; ++e) {
-        const int u = lane + 32 * e;
-        const int cw = u >> 6;
-        const int ch = cw == 0 ? prev : k0 + cw - 1;
-        const bool present = (cw == 0) ? (a.n_chunks > 1) : (ch < a.n_chunks);
-        pos[e] = present ? (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)] : kAtNoKey;
+    auto advance = [&](const Pt& p) {
+      Pt q = p;
+      if (!p.done) {
+        q.t = p.t + 1;
+        if (q.t >= q.t_end) next_item(q);
       }
+      return q;
     };
-    Pt nxt;
-    nxt.item = 0; nxt.r = 0; nxt.bh = 0; nxt.t = 0; nxt.t_end = 0; nxt.done = 0;
-    fetch_item(nxt);
-    uint32_t pos_n[6];
-    if (!nxt.done) load_pos(nxt, pos_n);
+    // window slot u: chunk u/64 of (prev, k0, k0+1); absent chunks read kAtNoKey
+    auto stage_perm = [&](const Pt& p, int st) {
+      if (!p.done) {
+        const size_t rowbase = ((size_t)p.r * a.BH + p.bh) * a.L;
+        const int k0 = 2 * p.t;
+        const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
+        for (int piece = lane; piece < 48; piece += 32) {  // 16-byte pieces
+          const int cw = piece >> 4;
+          const int ch = cw == 0 ? prev : k0 + cw - 1;
+          const bool present = (cw == 0) ? (a.n_chunks > 1) : (ch < a.n_chunks);
+          uint32_t* dst = &S.perm_stage[st][cw * 64 + (piece & 15) * 4];
+          if (present)
+            tc::cp_async16(tc::smem_u32(dst), a.perm + rowbase + (size_t)ch * 64 + (piece & 15) * 4);
+          else
+            *reinterpret_cast<uint4*>(dst) = make_uint4(kAtNoKey, kAtNoKey, kAtNoKey, kAtNoKey);
+        }
+      }
+      tc::cp_async_commit();
+    };
+    Pt q0;
+    q0.item = 0; q0.r = 0; q0.bh = 0; q0.t = 0; q0.t_end = 0; q0.done = 0;
+    next_item(q0);
+    Pt q1 = advance(q0);
+    stage_perm(q0, 0);
+    stage_perm(q1, 1);
     int done_marks = 0;
     for (uint32_t n = 0;; ++n) {
       const int s = n % kAtSlots;
-      const Pt cur = nxt;
-      uint32_t pos[6];
-#pragma unroll
-      for (int e = 0; e < 6; ++e) pos[e] = pos_n[e];
-      if (!cur.done) {
-        nxt.t = cur.t + 1;
-        if (nxt.t >= nxt.t_end) fetch_item(nxt);
-        if (!nxt.done) load_pos(nxt, pos_n);
-      }
+      const Pt cur = q0;
+      if (n == 0) tc::cp_async_wait<1>(); else tc::cp_async_wait<2>();  // perm of tile n
+      __syncwarp();
       const bool ok = __all_sync(0xffffffffu,
                                  at_wait(&S.empty[s], ((n / kAtSlots) & 1u) ^ 1u, &S.abort));
       if (!ok) break;
       if (cur.done) {
         // one end marker for each warpgroup (the issuing warp sees the first)
-        if (lane == 0) S.info[s].done = 1;
+        if (lane == 0) {
+          S.info[s].done = 1;
+          if (done_marks == 0) st_release_cta(&S.n_total, n);
+        }
         tc::fence_async_smem();
         cp_async_arrive_noinc(&S.full[s]);
         tc::mbar_arrive(&S.full[s]);
+        tc::cp_async_commit();  // keep two groups per iteration
+        tc::cp_async_commit();
         if (++done_marks == 2) break;
         continue;
       }
+      uint32_t pos[6];
+#pragma unroll
+      for (int e = 0; e < 6; ++e) pos[e] = S.perm_stage[n % kAtSlots][lane + 32 * e];
       AtInfo inf;
       const int k0 = 2 * cur.t;
       inf.done = 0;
@@ -362,9 +401,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       for (int e = 0; e < 6; ++e)  // absent rows read as position 0 downstream
         if (S.pos[s][lane + 32 * e] == kAtNoKey) S.pos[s][lane + 32 * e] = 0;
       if (lane == 0) S.info[s] = inf;
+      tc::cp_async_commit();  // this tile's gathers
       tc::fence_async_smem();
       cp_async_arrive_noinc(&S.full[s]);
       tc::mbar_arrive(&S.full[s]);
+      // two tiles ahead: its ticket (if it starts an item) and perm entries
+      q0 = q1;
+      q1 = advance(q1);
+      stage_perm(q1, (n + 2) % kAtSlots);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------ tensor-core issue
@@ -436,6 +480,39 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       }
     }
     __syncwarp();
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ publisher
+    // Online mode: makes each finished tile's stores visible device-wide and
+    // counts it for its (head, round).  One fence covers every tile posted
+    // since the last one, so fence latency never reaches the compute warps.
+    if (a.online && lane == 0) {
+      unsigned head = 0;
+      long long idle_since = clock64();
+      for (;;) {
+        unsigned tail = head;
+        while (ld_acquire_cta(&S.pub_seq[tail % kAtPubRing]) == tail + 1) ++tail;
+        if (tail > head) {
+          __threadfence();
+          for (unsigned t = head; t < tail; ++t) {
+            const int bh = S.pub_bh[t % kAtPubRing];
+            if (bh >= 0) atomicAdd(a.counters + (size_t)bh * a.R + S.pub_r[t % kAtPubRing], 1u);
+          }
+          head = tail;
+          st_release_cta(&S.pub_head, head);
+          idle_since = clock64();
+          continue;
+        }
+        if (head == ld_acquire_cta(&S.n_total)) break;  // every tile of this CTA published
+        if (*(volatile int*)&S.abort) break;
+        if (clock64() - idle_since > tc::kSpinCycles) {
+          record_status(tc::kErrTimeout);
+          *(volatile int*)&S.abort = 1;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __syncwarp();
   } else {
     // --------------------------------------------- softmax and epilogue
     const int w = warp >> 2;            // warpgroup
@@ -444,18 +521,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
     const int wrow0 = (warp & 3) * 32;  // first row of this warp
     const uint32_t region = tmem + (uint32_t)w * 256 + ((uint32_t)wrow0 << 16);
     uint8_t* wg_acc = acc_s + (size_t)w * 128 * 256;  // this warpgroup's staging rows
-    // online mode: this warpgroup's last tile whose completion is not yet
-    // counted; it is published (fence + counter) once its stores are old,
-    // before a dependency wait, and at exit -- a fence right after the
-    // stores would stall the warpgroup for their whole latency
-    int pend_bh = -1, pend_r = 0;
-    auto publish = [&]() {
-      if (pend_bh >= 0 && m == 0) {
-        __threadfence();
-        atomicAdd(a.counters + (size_t)pend_bh * a.R + pend_r, 1u);
-      }
-      pend_bh = -1;
-    };
     for (uint32_t j = 0;; ++j) {
       const uint32_t n = (uint32_t)w + 2 * j;
       const int s = n % kAtSlots;
@@ -468,7 +533,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         // (head, round) seen complete is cached so later tiles skip the load
         bool waited = true;
         if (!(S.dep_bh == inf.bh && S.dep_r == inf.r)) {
-          publish();  // never wait while holding an unpublished tile
           if (m == 0) {
             const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
             const long long t0 = clock64();
@@ -597,7 +661,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const bool oko = at_wait(&S.o_full[w], j & 1u, &S.abort);
       if (wg_or(w, !oko)) break;
       tc::fence_after_sync();
-      publish();               // the previous tile's stores are long issued
       tc::cp_async_wait<0>();  // this lane's staged pieces have landed
       __syncwarp();            // ... and the other lanes' (rows are shared)
       const float4 ml = fold ? ml_s[w * 128 + m] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -700,15 +763,27 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         }
       }
       tc::mbar_arrive(&S.empty[s]);
-      if (a.online && !last_round) {
-        pend_bh = inf.bh;
-        pend_r = inf.r;
+      if (a.online) {
+        // hand the finished tile to the publisher: every thread's stores are
+        // ordered before the release below by this barrier
+        if (wg_or(w, false)) break;
+        if (m == 0) {
+          const int k = n % kAtPubRing;
+          bool room = true;
+          const long long t0 = clock64();
+          while (ld_acquire_cta(&S.pub_head) + kAtPubRing <= n) {  // ring full (never in practice)
+            if (*(volatile int*)&S.abort || clock64() - t0 > tc::kSpinCycles) { room = false; break; }
+          }
+          if (!room) {
+            record_status(tc::kErrTimeout);
+            *(volatile int*)&S.abort = 1;
+          }
+          S.pub_bh[k] = last_round ? -1 : (int)inf.bh;  // the last round has no waiter
+          S.pub_r[k] = inf.r;
+          st_release_cta(&S.pub_seq[k], n + 1);
+        }
       }
     }
-    // stores of the last tile: every thread's are ordered before thread 0's
-    // fence by this barrier
-    wg_or(w, false);
-    publish();
   }
   tc::fence_before_sync();
   __syncthreads();
