@@ -205,6 +205,49 @@ __device__ __forceinline__ void at_decode(const AttnTcArgs& a, long long ticket,
   t0 = (rem % a.ipr) * a.tpi;
 }
 
+// Masked, scaled scores (log2 units; -inf where masked) of 32 window
+// columns whose packed keys and key scales are kw[0..31], rw[0..31].
+__device__ __forceinline__ void mask32(float* v, const uint32_t* kw, const float* rw,
+                                       uint32_t lo, uint32_t span, uint32_t ki, bool active,
+                                       bool causal) {
+#pragma unroll
+  for (int jj = 0; jj < 32; jj += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(kw + jj);
+    const float4 r4 = *reinterpret_cast<const float4*>(rw + jj);
+    const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
+    const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      bool in = active && (kj[x] - lo) < span;
+      if (!causal) in = in && kj[x] != ki;
+      v[jj + x] = in ? v[jj + x] * rj[x] : -INFINITY;
+    }
+  }
+}
+
+// Exact route for rows with a large score bound: writes the masked scores
+// back over S and returns the row maximum (log2 units; 0 if all masked).
+// Out of line: rarely taken, kept out of the hot loop's instruction cache.
+__device__ __noinline__ float exact_row_max(uint32_t region, int qc, const uint32_t* key_s,
+                                            const float* rn_s, uint32_t lo, uint32_t span,
+                                            uint32_t ki, bool valid, bool has_prev, bool causal) {
+  float mx2 = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    const int kc = qc + (c >> 1);
+    float v[32];
+    tc::tmem_ld32(region + qc * 64 + 32 * c, v);
+    tc::tmem_ld_wait();
+    mask32(v, key_s + kc * 64 + 32 * (c & 1), rn_s + kc * 64 + 32 * (c & 1), lo, span, ki,
+           valid && (kc != 0 || has_prev), causal);
+#pragma unroll
+    for (int x = 0; x < 32; ++x) mx2 = fmaxf(mx2, v[x]);
+    tc::tmem_st32(region + qc * 64 + 32 * c, reinterpret_cast<const uint32_t*>(v));
+  }
+  tc::tmem_st_wait();
+  return mx2 == -INFINITY ? 0.f : mx2;
+}
+
 // log2(e) / (|q| sqrt(d)) per token (0 for a zero row): the key
 // normalisation and score scale, in the log2 units the softmax uses.
 __global__ void key_scale_kernel(const __nv_bfloat16* __restrict__ Q, size_t n_tok,
@@ -381,7 +424,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       __syncwarp();
       // q and v rows, eight lanes per 128-byte row (coalesced per row): four
       // rows per warp instruction instead of 32 scattered 16-byte pieces
-#pragma unroll 4
+#pragma unroll 2
       for (int i = 0; i < 48; ++i) {
         const int u = 4 * i + (lane >> 3), c = lane & 7;
         const int cw = u >> 6, row = u & 63;
@@ -560,7 +603,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       // running state of this warp's 32 rows: staged by cp.async while the
       // softmax runs, sixteen lanes per 256-byte row
       if (fold) {
-#pragma unroll 4
+#pragma unroll 2
         for (int i = 0; i < 16; ++i) {
           const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
           const size_t t2 = bhL + S.pos[s][64 + rr];
@@ -585,65 +628,32 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const float bound = rn_i > 0.f ? 1.f / (64.f * rn_i * (1.f / kLog2e)) : 0.f;
       const bool exact = __any_sync(0xffffffffu, bound > kRefLimit);
       float ref2 = bound * kLog2e;  // reference in log2 units
-      // masked scores (log2 units, -inf where masked) of the 64 columns of
-      // window chunk kc = qc + pp
-      auto masked = [&](int pp, float* v) {
-        const int kc = qc + pp;
-        const bool active = valid && (kc != 0 || inf.has_prev);
-        const uint32_t* kw = &S.key[s][kc * 64];
-        const float* rw = &S.rn[s][kc * 64];
-#pragma unroll
-        for (int jj = 0; jj < 64; jj += 4) {
-          const uint4 k4 = *reinterpret_cast<const uint4*>(kw + jj);
-          const float4 r4 = *reinterpret_cast<const float4*>(rw + jj);
-          const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
-          const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            bool in = active && (kj[x] - lo) < span;
-            if (!a.causal) in = in && kj[x] != ki;
-            v[jj + x] = in ? v[jj + x] * rj[x] : -INFINITY;
-          }
-        }
-      };
-      if (exact) {  // pass 1: masked scores back into S, exact row maximum
-        float mx2 = -INFINITY;
-#pragma unroll 1
-        for (int pp = 0; pp < 2; ++pp) {
-          float v[64];
-          tc::tmem_ld32(region + qc * 64 + 64 * pp, v);
-          tc::tmem_ld32(region + qc * 64 + 64 * pp + 32, v + 32);
-          tc::tmem_ld_wait();
-          masked(pp, v);
-#pragma unroll
-          for (int x = 0; x < 64; ++x) mx2 = fmaxf(mx2, v[x]);
-          tc::tmem_st32(region + qc * 64 + 64 * pp, reinterpret_cast<const uint32_t*>(v));
-          tc::tmem_st32(region + qc * 64 + 64 * pp + 32, reinterpret_cast<const uint32_t*>(v + 32));
-        }
-        tc::tmem_st_wait();
-        ref2 = mx2 == -INFINITY ? 0.f : mx2;
-      }
+      if (exact)  // pass 1: masked scores back into S, exact row maximum
+        ref2 = exact_row_max(region, qc, S.key[s], S.rn[s], lo, span, ki, valid, inf.has_prev,
+                             a.causal != 0);
       float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
       // P (bf16, two per column) over S: key block b at columns [32b, 32b+32).
-      // Window chunk qc + pp (S columns qc*64 + 64pp) becomes P block qc + pp
-      // (columns 32(qc + pp)); each step reads its S columns before writing,
-      // and never writes columns a later step still reads.
+      // Step c reads S columns qc*64 + 32c .. +32 (window chunk qc + c/2) and
+      // writes P columns 32(qc + c/2) + 16(c&1) .. +16; every write lands on
+      // columns already read and never on ones a later step reads.
 #pragma unroll 1
-      for (int pp = 0; pp < 2; ++pp) {
-        float v[64];
-        tc::tmem_ld32(region + qc * 64 + 64 * pp, v);
-        tc::tmem_ld32(region + qc * 64 + 64 * pp + 32, v + 32);
+      for (int c = 0; c < 4; ++c) {
+        const int kc = qc + (c >> 1);
+        float v[32];
+        tc::tmem_ld32(region + qc * 64 + 32 * c, v);
         tc::tmem_ld_wait();
-        if (!exact) masked(pp, v);
-        uint32_t pk[32];
+        if (!exact)
+          mask32(v, &S.key[s][kc * 64 + 32 * (c & 1)], &S.rn[s][kc * 64 + 32 * (c & 1)], lo,
+                 span, ki, valid && (kc != 0 || inf.has_prev), a.causal != 0);
+        uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
+        for (int x = 0; x < 16; ++x) {
           const float p0 = ex2(v[2 * x] - ref2);
           const float p1 = ex2(v[2 * x + 1] - ref2);
           ls[x & 3] += p0 + p1;
           pk[x] = pack_bf16(p0, p1);
         }
-        tc::tmem_st32(region + (qc + pp) * 32, pk);
+        tc::tmem_st16(region + kc * 32 + 16 * (c & 1), pk);
       }
       {
         uint32_t pk[32];
@@ -682,7 +692,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       uint8_t* my_row = wg_acc + (size_t)m * 256;
       // O in two 32-column halves; the result goes back into this row's
       // staging space (fp32, or bf16 for the final output)
-#pragma unroll
+#pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         float o[32];
         tc::tmem_ld32(region + 192 + 32 * hh, o);
@@ -742,7 +752,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       if (valid) {
         if (!out_bf16) {
           float* base = !a.online ? a.o_part + (size_t)inf.r * n_tok * 64 : a.acc_o;
-#pragma unroll 4
+#pragma unroll 2
           for (int i = 0; i < 16; ++i) {
             const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
             const size_t t2 = bhL + S.pos[s][64 + rr];
@@ -752,7 +762,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             else __stcg(reinterpret_cast<float4*>(base + t2 * 64 + 4 * q), f);
           }
         } else {
-#pragma unroll 4
+#pragma unroll 2
           for (int i = 0; i < 8; ++i) {
             const int rr = wrow0 + 4 * i + (lane >> 3), q = lane & 7;
             const size_t t2 = bhL + S.pos[s][64 + rr];

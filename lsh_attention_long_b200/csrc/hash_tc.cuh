@@ -8,8 +8,9 @@
 // The projection is a GEMM: P[tokens, R*nb/2] = Q[tokens, 64] x [R_0 | R_1 | ..].
 // bf16 x bf16 products are exact in fp32, so only the fp32 accumulation order
 // differs from an exact computation.  tcgen05.mma (M = 128 tokens, N <= 256
-// rotation columns, K = 64) accumulates into tensor memory; the epilogue reads
-// each token's row (one TMEM lane per thread) and keeps the signed argmax.
+// rotation columns, K = 64) accumulates into tensor memory; two epilogue
+// warpgroups read each token's row (one TMEM lane per thread, each warpgroup
+// one 128-column half of the N-tile) and keep the signed argmax.
 //
 // Signed argmax, exactly as defined: the maximum of [p ; -p] is max_j |p_j|;
 // among the entries reaching it the lowest index of the concatenation wins,
@@ -31,6 +32,7 @@
 namespace lsh {
 
 constexpr int kHashTcRotBytes = 128 * 1024;
+constexpr int kHashTcThreads = 256;  // two epilogue warpgroups
 
 struct HashTcArgs {
   const __nv_bfloat16* Q;
@@ -43,9 +45,10 @@ struct HashTcArgs {
 
 __host__ __device__ inline size_t hash_tc_smem_bytes(int rounds_per_group, int half) {
   // alignment slack, rotation columns, two Q tiles, one 128-byte slot per
-  // thread; at least 120 KB so that one CTA (holding all 512 TMEM columns)
-  // runs per SM
-  const size_t need = 1024 + (size_t)rounds_per_group * half * 128 + 2 * 16384 + 128 * 128;
+  // thread, the cross-warpgroup hand-off; at least 120 KB so that one CTA
+  // (holding all 512 TMEM columns) runs per SM
+  const size_t need = 1024 + (size_t)rounds_per_group * half * 128 + 2 * 16384 +
+                      kHashTcThreads * 128 + 128 * 8;
   return need > 120 * 1024 ? need : 120 * 1024;
 }
 
@@ -122,7 +125,7 @@ __device__ __forceinline__ void hash_segment(uint32_t ta, int len, int jbase, in
 }
 
 template <int CW>
-__global__ void __launch_bounds__(128, 1) hash_tc_kernel(HashTcArgs a) {
+__global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[2];
   __shared__ uint32_t tmem_base_s;
@@ -140,6 +143,12 @@ __global__ void __launch_bounds__(128, 1) hash_tc_kernel(HashTcArgs a) {
   uint8_t* q_s = sm + (size_t)a.rounds_per_group * a.half * 128;
   uint8_t* slot = q_s + 2 * 16384 + threadIdx.x * 128;
   const int sw = threadIdx.x & 7;
+  // warpgroup wg reads columns [128 wg, 128 wg + 128) of each N-tile for the
+  // token in TMEM lane `row`; for rounds wider than 128 columns the two
+  // halves meet here at the round's end
+  float* comb_best = reinterpret_cast<float*>(q_s + 2 * 16384 + kHashTcThreads * 128);
+  int* comb_bkt = reinterpret_cast<int*>(comb_best + 128);
+  const int wg = threadIdx.x >> 7, row = threadIdx.x & 127;
 
   if (warp == 0) {
     tc::tmem_alloc(&tmem_base_s, 512);
@@ -191,12 +200,12 @@ __global__ void __launch_bounds__(128, 1) hash_tc_kernel(HashTcArgs a) {
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base_s;
-  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 
   float rbest = -1.f;
   int rbkt = 0;
   const int n_jobs = n_items * T;
-  const int seg_len = min(a.half, 256);
+  const int seg_len = min(a.half, 128);
   for (int n = 0; n <= n_jobs; ++n) {
     if (n < n_jobs) {
       const int k = n / T, t = n % T;
@@ -227,19 +236,41 @@ __global__ void __launch_bounds__(128, 1) hash_tc_kernel(HashTcArgs a) {
       const int k = m / T, t = m % T;
       const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[m & 1], (m >> 1) & 1));
       tc::fence_after_sync();
+      const int tok = (c + k * a.ctas_per_group) * 128 + row;
+      const int nt = min(256, cols - t * 256);
       if (ok) {
-        const int tok = (c + k * a.ctas_per_group) * 128 + tid;
-        const int nt = min(256, cols - t * 256);
-        for (int s0 = 0; s0 < nt; s0 += seg_len) {
+        for (int s0 = wg * 128; s0 < min(nt, wg * 128 + 128); s0 += seg_len) {
           const int gcol = t * 256 + s0;
           const int rl = gcol / a.half, jbase = gcol % a.half;
-          if (jbase == 0) { rbest = -1.f; rbkt = 0; }
+          // a round starts: at its first column, or (rounds wider than 128
+          // columns) at this warpgroup's first columns of the round's first tile
+          if (jbase == 0 || (s0 == wg * 128 && (t * 256) % a.half == 0)) {
+            rbest = -1.f;
+            rbkt = 0;
+          }
           float sb;
           int sk;
           hash_segment<CW>(lane_base + (m & 1) * 256 + s0, seg_len, jbase, a.half, slot, sw, sb,
                            sk);
           if (sb > rbest || (sb == rbest && sk < rbkt)) { rbest = sb; rbkt = sk; }
-          if (jbase + seg_len == a.half && tok < a.n_tok) {
+          if (a.half <= 128 && jbase + seg_len == a.half && tok < a.n_tok) {
+            const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
+            a.keys[o] = (uint32_t)rbkt * (uint32_t)a.L + (uint32_t)(tok % a.L);
+            if (a.buckets) a.buckets[o] = rbkt;
+          }
+        }
+      }
+      // rounds wider than 128 columns: the second warpgroup's half joins the
+      // first's at the N-tile holding the round's last column
+      if (a.half > 128 && ((t + 1) * 256) % a.half == 0) {
+        if (wg == 1) { comb_best[row] = rbest; comb_bkt[row] = rbkt; }
+        __syncthreads();
+        if (wg == 0 && ok) {
+          const float ob = comb_best[row];
+          const int okk = comb_bkt[row];
+          if (ob > rbest || (ob == rbest && okk < rbkt)) { rbest = ob; rbkt = okk; }
+          const int rl = (t * 256) / a.half;
+          if (tok < a.n_tok) {
             const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
             a.keys[o] = (uint32_t)rbkt * (uint32_t)a.L + (uint32_t)(tok % a.L);
             if (a.buckets) a.buckets[o] = rbkt;

@@ -164,11 +164,11 @@ lsh_status hash_tc_launch(const Dims& D, const void* Q, const void* rot, uint32_
   if (a.half >= 32) {
     lsh_status s0 = allow_smem(lsh::hash_tc_kernel<32>, smem);
     if (s0 != LSH_OK) return s0;
-    lsh::hash_tc_kernel<32><<<grid, 128, smem, st>>>(a);
+    lsh::hash_tc_kernel<32><<<grid, lsh::kHashTcThreads, smem, st>>>(a);
   } else {
     lsh_status s0 = allow_smem(lsh::hash_tc_kernel<16>, smem);
     if (s0 != LSH_OK) return s0;
-    lsh::hash_tc_kernel<16><<<grid, 128, smem, st>>>(a);
+    lsh::hash_tc_kernel<16><<<grid, lsh::kHashTcThreads, smem, st>>>(a);
   }
   return last_launch();
 }
