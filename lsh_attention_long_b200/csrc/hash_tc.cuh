@@ -8,9 +8,9 @@
 // The projection is a GEMM: P[tokens, R*nb/2] = Q[tokens, 64] x [R_0 | R_1 | ..].
 // bf16 x bf16 products are exact in fp32, so only the fp32 accumulation order
 // differs from an exact computation.  tcgen05.mma (M = 128 tokens, N <= 256
-// rotation columns, K = 64) accumulates into tensor memory; four epilogue
+// rotation columns, K = 64) accumulates into tensor memory; two epilogue
 // warpgroups read each token's row (one TMEM lane per thread, each warpgroup
-// one 64-column quarter of the N-tile) and keep the signed argmax.
+// one 128-column half of the N-tile) and keep the signed argmax.
 //
 // Signed argmax, exactly as defined: the maximum of [p ; -p] is max_j |p_j|;
 // among the entries reaching it the lowest index of the concatenation wins,
@@ -32,7 +32,7 @@
 namespace lsh {
 
 constexpr int kHashTcRotBytes = 128 * 1024;
-constexpr int kHashTcThreads = 512;  // four epilogue warpgroups
+constexpr int kHashTcThreads = 256;  // two epilogue warpgroups
 
 struct HashTcArgs {
   const __nv_bfloat16* Q;
@@ -48,15 +48,14 @@ __host__ __device__ inline size_t hash_tc_smem_bytes(int rounds_per_group, int h
   // thread, the cross-warpgroup hand-off; at least 120 KB so that one CTA
   // (holding all 512 TMEM columns) runs per SM
   const size_t need = 1024 + (size_t)rounds_per_group * half * 128 + 2 * 16384 +
-                      kHashTcThreads * 128;
+                      kHashTcThreads * 128 + 128 * 8;
   return need > 120 * 1024 ? need : 120 * 1024;
 }
 
 // Exact (max |p|, bucket) over `len` columns starting at TMEM address `ta`
 // whose first column is column `jbase` of its round.
 //
-// Pass A: per CW columns (all of the segment loaded under one wait), max |p|
-// (one FMNMX per value); a chunk that raises
+// Pass A: per CW columns, max |p| (one FMNMX per value); a chunk that raises
 // the running maximum is copied to this thread's 128-byte slot in shared
 // memory (16-byte pieces, swizzled by thread).  Pass B: the slot holds the
 // chunk of the maximum; an exact scan there gives the lowest bucket
@@ -66,34 +65,23 @@ template <int CW>
 __device__ __forceinline__ void hash_segment(uint32_t ta, int len, int jbase, int half,
                                              uint8_t* slot, int sw, float& best_out,
                                              int& bkt_out) {
-  // pass A: the segment's columns (at most 64) land with one wait
-  float va[64];
-  const int nch = len / CW;
-#pragma unroll
-  for (int c = 0; c < 64 / CW; ++c)
-    if (c < nch) {
-      if (CW == 32) tc::tmem_ld32(ta + c * CW, va + c * CW); else tc::tmem_ld16(ta + c * CW, va + c * CW);
-    }
-  tc::tmem_ld_wait();
+  float v[CW];
   float best = -1.f;
   int bc = -1;
   bool tie = false;
+  for (int cc = 0; cc < len; cc += CW) {
+    if (CW == 32) tc::tmem_ld32(ta + cc, v); else tc::tmem_ld16(ta + cc, v);
+    tc::tmem_ld_wait();
+    float m0 = fabsf(v[0]), m1 = fabsf(v[1]);
 #pragma unroll
-  for (int c = 0; c < 64 / CW; ++c) {
-    if (c >= nch) break;
-    const float* v = va + c * CW;
-    float m0 = fabsf(v[0]), m1 = fabsf(v[1]), m2 = fabsf(v[2]), m3 = fabsf(v[3]);
-#pragma unroll
-    for (int j = 4; j < CW; j += 4) {
+    for (int j = 2; j < CW; j += 2) {
       m0 = fmaxf(m0, fabsf(v[j]));
       m1 = fmaxf(m1, fabsf(v[j + 1]));
-      m2 = fmaxf(m2, fabsf(v[j + 2]));
-      m3 = fmaxf(m3, fabsf(v[j + 3]));
     }
-    const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    const float m = fmaxf(m0, m1);
     if (m > best) {
       best = m;
-      bc = c * CW;
+      bc = cc;
       tie = false;
 #pragma unroll
       for (int q = 0; q < CW / 4; ++q)
@@ -103,7 +91,6 @@ __device__ __forceinline__ void hash_segment(uint32_t ta, int len, int jbase, in
       tie = true;
     }
   }
-  float v[CW];
   int bkt = jbase;
   if (__any_sync(0xffffffffu, tie)) {
     // exact scan of every chunk for the lanes with a tie (warp-uniform loads)
@@ -156,13 +143,12 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
   uint8_t* q_s = sm + (size_t)a.rounds_per_group * a.half * 128;
   uint8_t* slot = q_s + 2 * 16384 + threadIdx.x * 128;
   const int sw = threadIdx.x & 7;
-  // warpgroup wg reads columns [64 wg, 64 wg + 64) of each N-tile for the
-  // token in TMEM lane `row`; for rounds wider than 64 columns the
-  // warpgroups' partial results meet at the round's end in the first 4 KB of
-  // the slot area (free then: every segment of the tile is done)
-  float* comb_best = reinterpret_cast<float*>(q_s + 2 * 16384);
-  int* comb_bkt = reinterpret_cast<int*>(comb_best + 4 * 128);
-  const int wg = threadIdx.x >> 7, row = threadIdx.x & 127;  // 4 warpgroups
+  // warpgroup wg reads columns [128 wg, 128 wg + 128) of each N-tile for the
+  // token in TMEM lane `row`; for rounds wider than 128 columns the two
+  // halves meet here at the round's end
+  float* comb_best = reinterpret_cast<float*>(q_s + 2 * 16384 + kHashTcThreads * 128);
+  int* comb_bkt = reinterpret_cast<int*>(comb_best + 128);
+  const int wg = threadIdx.x >> 7, row = threadIdx.x & 127;
 
   if (warp == 0) {
     tc::tmem_alloc(&tmem_base_s, 512);
@@ -219,7 +205,7 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
   float rbest = -1.f;
   int rbkt = 0;
   const int n_jobs = n_items * T;
-  const int seg_len = min(a.half, 64);
+  const int seg_len = min(a.half, 128);
   for (int n = 0; n <= n_jobs; ++n) {
     if (n < n_jobs) {
       const int k = n / T, t = n % T;
@@ -253,12 +239,12 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
       const int tok = (c + k * a.ctas_per_group) * 128 + row;
       const int nt = min(256, cols - t * 256);
       if (ok) {
-        for (int s0 = wg * 64; s0 < min(nt, wg * 64 + 64); s0 += seg_len) {
+        for (int s0 = wg * 128; s0 < min(nt, wg * 128 + 128); s0 += seg_len) {
           const int gcol = t * 256 + s0;
           const int rl = gcol / a.half, jbase = gcol % a.half;
-          // a round starts: at its first column, or (rounds wider than 64
+          // a round starts: at its first column, or (rounds wider than 128
           // columns) at this warpgroup's first columns of the round's first tile
-          if (jbase == 0 || (s0 == wg * 64 && (t * 256) % a.half == 0)) {
+          if (jbase == 0 || (s0 == wg * 128 && (t * 256) % a.half == 0)) {
             rbest = -1.f;
             rbkt = 0;
           }
@@ -267,35 +253,27 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
           hash_segment<CW>(lane_base + (m & 1) * 256 + s0, seg_len, jbase, a.half, slot, sw, sb,
                            sk);
           if (sb > rbest || (sb == rbest && sk < rbkt)) { rbest = sb; rbkt = sk; }
-          if (a.half <= 64 && jbase + seg_len == a.half && tok < a.n_tok) {
+          if (a.half <= 128 && jbase + seg_len == a.half && tok < a.n_tok) {
             const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
             a.keys[o] = (uint32_t)rbkt * (uint32_t)a.L + (uint32_t)(tok % a.L);
             if (a.buckets) a.buckets[o] = rbkt;
           }
         }
       }
-      // rounds wider than 64 columns: the warpgroups covering a round join at
-      // the N-tile holding its last column (half = 128: pairs of warpgroups;
-      // wider: all four, across the round's tiles)
-      if (a.half > 64 && ((t + 1) * 256) % a.half == 0) {
-        __syncthreads();  // every thread is past its segments: the slots are free
-        comb_best[wg * 128 + row] = rbest;
-        comb_bkt[wg * 128 + row] = rbkt;
+      // rounds wider than 128 columns: the second warpgroup's half joins the
+      // first's at the N-tile holding the round's last column
+      if (a.half > 128 && ((t + 1) * 256) % a.half == 0) {
+        if (wg == 1) { comb_best[row] = rbest; comb_bkt[row] = rbkt; }
         __syncthreads();
-        const int per = a.half >= 256 ? 4 : 2;  // warpgroups per round in this tile
-        if (wg % per == 0 && ok && t * 256 + wg * 64 < cols) {  // the round exists
-          float b = comb_best[wg * 128 + row];
-          int k2 = comb_bkt[wg * 128 + row];
-          for (int o2 = 1; o2 < per; ++o2) {
-            const float ob = comb_best[(wg + o2) * 128 + row];
-            const int okk = comb_bkt[(wg + o2) * 128 + row];
-            if (ob > b || (ob == b && okk < k2)) { b = ob; k2 = okk; }
-          }
-          const int rl = (t * 256 + wg * 64) / a.half;
+        if (wg == 0 && ok) {
+          const float ob = comb_best[row];
+          const int okk = comb_bkt[row];
+          if (ob > rbest || (ob == rbest && okk < rbkt)) { rbest = ob; rbkt = okk; }
+          const int rl = (t * 256) / a.half;
           if (tok < a.n_tok) {
             const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
-            a.keys[o] = (uint32_t)k2 * (uint32_t)a.L + (uint32_t)(tok % a.L);
-            if (a.buckets) a.buckets[o] = k2;
+            a.keys[o] = (uint32_t)rbkt * (uint32_t)a.L + (uint32_t)(tok % a.L);
+            if (a.buckets) a.buckets[o] = rbkt;
           }
         }
       }
