@@ -84,6 +84,7 @@ struct AtInfo {
   int done;
   int nq;           // query chunks present: 1 or 2
   int has_prev;     // window has a previous chunk (the row has > 1 chunk)
+  int seq;          // tile sequence number the slot holds
 };
 
 struct AttnTcArgs {
@@ -374,6 +375,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         // one end marker for each warpgroup (the issuing warp sees the first)
         if (lane == 0) {
           S.info[s].done = 1;
+          S.info[s].seq = (int)n;
           if (done_marks == 0) st_release_cta(&S.n_total, n);
         }
         tc::fence_async_smem();
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       AtInfo inf;
       const int k0 = 2 * cur.t;
       inf.done = 0;
+      inf.seq = (int)n;
       inf.r = cur.r;
       inf.bh = cur.bh;
       inf.t = cur.t;
@@ -567,7 +570,20 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
     for (uint32_t j = 0;; ++j) {
       const uint32_t n = (uint32_t)w + 2 * j;
       const int s = n % kAtSlots;
-      const bool okf = at_wait(&S.full[s], (n / kAtSlots) & 1u, &S.abort);
+      // slot s last held tile n - 3, the other warpgroup's: a parity wait
+      // can pass on that older phase, so the slot's sequence number decides
+      bool okf;
+      const long long t_full = clock64();
+      for (;;) {
+        okf = at_wait(&S.full[s], (n / kAtSlots) & 1u, &S.abort);
+        if (!okf || *(volatile int*)&S.info[s].seq == (int)n) break;
+        if (clock64() - t_full > tc::kSpinCycles) {
+          record_status(tc::kErrTimeout);
+          *(volatile int*)&S.abort = 1;
+          okf = false;
+          break;
+        }
+      }
       const AtInfo inf = S.info[s];
       if (wg_or(w, !okf || inf.done)) break;
 
