@@ -8,17 +8,18 @@
 // The projection is a GEMM: P[tokens, R*nb/2] = Q[tokens, 64] x [R_0 | R_1 | ..].
 // bf16 x bf16 products are exact in fp32, so only the fp32 accumulation order
 // differs from an exact computation.  tcgen05.mma (M = 128 tokens, N <= 256
-// rotation columns, K = 64) accumulates into tensor memory; two epilogue
-// warpgroups read each token's row (one TMEM lane per thread, each warpgroup
-// one 128-column half of the N-tile) and keep the signed argmax.
+// rotation columns, K = 64) accumulates into tensor memory; epilogue
+// warpgroups read each token's row (one TMEM lane per thread) and keep the
+// signed argmax.
 //
 // Signed argmax, exactly as defined: the maximum of [p ; -p] is max_j |p_j|;
 // among the entries reaching it the lowest index of the concatenation wins,
 // i.e. the smallest "bucket candidate" b_j = j (p_j >= 0) or j + nb/2
-// (p_j < 0).  Pass A takes max |p| per 32 columns with one FMNMX per value
-// and parks the chunk holding the running maximum in shared memory; pass B
-// scans that chunk for the index.  Exactly tied chunk maxima take a slow path
-// that scans every candidate.
+// (p_j < 0).  Each token's row is reduced in chunks of 32 columns: a tree of
+// 3-input maxima gives the chunk's max |p|; the first chunk to reach the
+// round's running maximum is parked in shared memory, and once per round an
+// exact scan of the parked chunk gives the index.  A later chunk whose maximum
+// ties the running one exactly is scanned on the spot.
 //
 // Work split: CTAs are grouped by rounds; a group keeps its rounds' rotation
 // columns resident in shared memory (transposed to K-major, 128B-swizzled,
@@ -57,92 +58,90 @@ __host__ __device__ inline size_t hash_tc_smem_bytes(int rounds_per_group, int h
   return need > 120 * 1024 ? need : 120 * 1024;
 }
 
-// Exact (max |p|, bucket) over `len` columns starting at TMEM address `ta`
-// whose first column is column `jbase` of its round.
-//
-// Pass A: per CW columns (the segment's columns loaded under one wait), max
-// |p| (one FMNMX per value); a chunk that raises
-// the running maximum is copied to this thread's 128-byte slot in shared
-// memory (16-byte pieces, swizzled by thread).  Pass B: the slot holds the
-// chunk of the maximum; an exact scan there gives the lowest bucket
-// candidate.  Chunks whose maxima tie exactly send the warp through a slow
-// exact scan of every chunk.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max over N values as a tree of 3-input maxima (short dependency chains)
+template <int N>
+__device__ __forceinline__ float max_tree(const float* x) {
+  if constexpr (N == 1) {
+    return x[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(x[0], x[1]);
+  } else {
+    constexpr int M = (N + 2) / 3;
+    float y[M];
+#pragma unroll
+    for (int i = 0; i < N / 3; ++i) y[i] = max3f(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+    if constexpr (N % 3 == 1) y[M - 1] = x[N - 1];
+    if constexpr (N % 3 == 2) y[M - 1] = fmaxf(x[N - 2], x[N - 1]);
+    return max_tree<M>(y);
+  }
+}
+
+// Running signed argmax of one token over one round, fed CW columns at a
+// time.  `slot` (this thread's 128 bytes of shared memory, 16-byte pieces
+// swizzled by `sw`) keeps the first chunk that reached the running maximum
+// `best` and `bc` its first column; chunks arriving later whose maximum equals
+// `best` exactly are resolved on the spot into `tie_cand`.
+struct ArgmaxState {
+  float best;
+  int bc;
+  int tie_cand;
+  __device__ __forceinline__ void reset() {
+    best = -1.f;
+    bc = 0;
+    tie_cand = 0x7fffffff;
+  }
+};
+
+// lowest bucket candidate (column j -> j for p_j >= 0, j + nb/2 for p_j < 0)
+// among the CW values of a chunk whose |p| equals m
 template <int CW>
-__device__ __forceinline__ void hash_segment(uint32_t ta, int len, int jbase, int half,
-                                             uint8_t* slot, int sw, float& best_out,
-                                             int& bkt_out) {
-  // pass A: batches of kHashBatch columns, each loaded under one wait
-  float best = -1.f;
-  int bc = -1;
-  bool tie = false;
-  for (int b0 = 0; b0 < len; b0 += kHashBatch) {
-    float va[kHashBatch];
-    const int nch = min(len - b0, kHashBatch) / CW;
+__device__ __forceinline__ int chunk_candidate(const float* v, float m, int base, int half) {
+  int jp = 0x7fffffff, jn = 0x7fffffff;
 #pragma unroll
-    for (int ch = 0; ch < kHashBatch / CW; ++ch)
-      if (ch < nch) {
-        if (CW == 32) tc::tmem_ld32(ta + b0 + ch * CW, va + ch * CW);
-        else tc::tmem_ld16(ta + b0 + ch * CW, va + ch * CW);
-      }
-    tc::tmem_ld_wait();
-#pragma unroll
-    for (int ch = 0; ch < kHashBatch / CW; ++ch) {
-      if (ch >= nch) break;
-      const float* v = va + ch * CW;
-      float m0 = fabsf(v[0]), m1 = fabsf(v[1]), m2 = fabsf(v[2]), m3 = fabsf(v[3]);
-#pragma unroll
-      for (int j = 4; j < CW; j += 4) {
-        m0 = fmaxf(m0, fabsf(v[j]));
-        m1 = fmaxf(m1, fabsf(v[j + 1]));
-        m2 = fmaxf(m2, fabsf(v[j + 2]));
-        m3 = fmaxf(m3, fabsf(v[j + 3]));
-      }
-      const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-      if (m > best) {
-        best = m;
-        bc = b0 + ch * CW;
-        tie = false;
-#pragma unroll
-        for (int q = 0; q < CW / 4; ++q)
-          *reinterpret_cast<float4*>(slot + ((q ^ sw) << 4)) =
-              make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else if (m == best) {
-        tie = true;
-      }
-    }
+  for (int j = CW - 1; j >= 0; --j) {
+    if (v[j] == m) jp = j;
+    if (v[j] == -m) jn = j;
   }
+  return jp != 0x7fffffff ? base + jp : (jn != 0x7fffffff ? base + jn + half : 0x7fffffff);
+}
+
+template <int CW>
+__device__ __forceinline__ void argmax_update(ArgmaxState& st, const float* v, int base, int half,
+                                              uint8_t* slot, int sw) {
+  float a[CW];
+#pragma unroll
+  for (int j = 0; j < CW; ++j) a[j] = fabsf(v[j]);
+  const float m = max_tree<CW>(a);
+  if (m > st.best) {
+    st.best = m;
+    st.bc = base;
+    st.tie_cand = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < CW / 4; ++q)
+      *reinterpret_cast<float4*>(slot + ((q ^ sw) << 4)) =
+          make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else if (m == st.best) {  // exact tie with an earlier chunk: rare
+    st.tie_cand = min(st.tie_cand, chunk_candidate<CW>(v, m, base, half));
+  }
+}
+
+// bucket of the round: the parked chunk's lowest candidate, or a later tied one
+template <int CW>
+__device__ __forceinline__ int argmax_finish(const ArgmaxState& st, int half, const uint8_t* slot,
+                                             int sw) {
   float v[CW];
-  int bkt = jbase;
-  if (__any_sync(0xffffffffu, tie)) {
-    // exact scan of every chunk for the lanes with a tie (warp-uniform loads)
-    int b_all = 0x7fffffff;
-    for (int cc = 0; cc < len; cc += CW) {
-      if (CW == 32) tc::tmem_ld32(ta + cc, v); else tc::tmem_ld16(ta + cc, v);
-      tc::tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int b = jbase + cc + j + (v[j] < 0.f ? half : 0);
-        if (fabsf(v[j]) == best && b < b_all) b_all = b;
-      }
-    }
-    if (tie) bkt = b_all;
+  for (int q = 0; q < CW / 4; ++q) {
+    const float4 f = *reinterpret_cast<const float4*>(slot + ((q ^ sw) << 4));
+    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
   }
-  if (!tie && bc >= 0) {
-#pragma unroll
-    for (int q = 0; q < CW / 4; ++q) {
-      const float4 f = *reinterpret_cast<const float4*>(slot + ((q ^ sw) << 4));
-      v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-    }
-    int b_min = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < CW; ++j) {
-      const int b = j + (v[j] < 0.f ? half : 0);
-      if (fabsf(v[j]) == best && b < b_min) b_min = b;
-    }
-    bkt = jbase + bc + b_min;  // b_min already carries + nb/2 for a negative maximum
-  }
-  best_out = best;
-  bkt_out = bkt;
+  return min(chunk_candidate<CW>(v, st.best, st.bc, half), st.tie_cand);
 }
 
 // Bounded mbarrier wait that also gives up once the CTA has aborted.
@@ -282,9 +281,11 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
     uint8_t* slot = q_s + 2 * 16384 + tid * 128;
     const int sw = tid & 7;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int seg_len = min(a.half, 128);
-    float rbest = -1.f;
-    int rbkt = 0;
+    const int bw = min(a.half, kHashBatch);  // columns per TMEM load batch; divides a round
+    const int bw_shift = __ffs(bw) - 1, half_shift = __ffs(a.half) - 1;  // powers of two
+    const int nch = bw / CW;
+    ArgmaxState st;
+    st.reset();
     uint32_t seen = 0;  // bit b: parity of this warpgroup's next job in buffer b
     for (int n = 0; n < n_jobs; ++n) {
       if (job_wg(n) != wgi) continue;
@@ -294,20 +295,40 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
       seen ^= 1u << b;
       tc::fence_after_sync();
       const int tok = (c + k * a.ctas_per_group) * 128 + row;
+      const uint32_t pos = (uint32_t)(tok % a.L);
       const int nt = min(256, cols - t * 256);
-      for (int s0 = 0; s0 < nt; s0 += seg_len) {
-        const int gcol = t * 256 + s0;
-        const int rl = gcol / a.half, jbase = gcol % a.half;
-        if (jbase == 0) { rbest = -1.f; rbkt = 0; }
-        float sb;
-        int sk;
-        hash_segment<CW>(lane_base + b * 256 + s0, seg_len, jbase, a.half, slot, sw, sb, sk);
-        if (sb > rbest || (sb == rbest && sk < rbkt)) { rbest = sb; rbkt = sk; }
-        if (jbase + seg_len == a.half && tok < a.n_tok) {
-          const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
-          a.keys[o] = (uint32_t)rbkt * (uint32_t)a.L + (uint32_t)(tok % a.L);
-          if (a.buckets) a.buckets[o] = rbkt;
+      const int nbat = nt >> bw_shift;
+      const uint32_t ta = lane_base + b * 256;
+      auto load = [&](float* va, int i) {
+#pragma unroll
+        for (int ch = 0; ch < kHashBatch / CW; ++ch)
+          if (ch < nch) {
+            if (CW == 32) tc::tmem_ld32(ta + (i << bw_shift) + ch * CW, va + ch * CW);
+            else tc::tmem_ld16(ta + (i << bw_shift) + ch * CW, va + ch * CW);
+          }
+      };
+      auto process = [&](float* va, int i) {
+        const int gcol = t * 256 + (i << bw_shift);
+        const int rl = gcol >> half_shift, jb = gcol & (a.half - 1);
+#pragma unroll
+        for (int ch = 0; ch < kHashBatch / CW; ++ch)
+          if (ch < nch) argmax_update<CW>(st, va + ch * CW, jb + ch * CW, a.half, slot, sw);
+        if (jb + bw == a.half) {  // the round is complete
+          const int bkt = argmax_finish<CW>(st, a.half, slot, sw);
+          st.reset();
+          if (tok < a.n_tok) {
+            const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
+            a.keys[o] = (uint32_t)bkt * (uint32_t)a.L + pos;
+            if (a.buckets) a.buckets[o] = bkt;
+          }
         }
+      };
+      for (int i = 0; i < nbat; ++i) {
+        float va[kHashBatch];
+        load(va, i);
+        tc::tmem_ld_wait();
+        tc::tmem_pin<kHashBatch>(va);
+        process(va, i);
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&buf_empty[b]);

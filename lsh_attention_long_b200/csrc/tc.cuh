@@ -121,6 +121,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// After tmem_ld_wait(): ties N registers written by earlier tcgen05.ld to the
+// wait, so that no use of them can be scheduled ahead of it.
+template <int N>
+__device__ __forceinline__ void tmem_pin(float* v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
 // 32 consecutive fp32 columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
