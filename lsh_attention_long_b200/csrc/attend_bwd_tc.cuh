@@ -1,0 +1,442 @@
+// Backward of chunked shared-QK LSH attention on the 5th-generation tensor
+// cores (bf16 inputs, d = 64, chunk = 64).  Buckets and permutations are
+// constants of the backward pass.
+//
+// "Reformer explainer" (akshathtiwari.co.in/blog/reformer), chunked attention
+// over sorted buckets and the union of hash rounds: every round's window
+// entries taken together form one softmax per query over all rounds, so with
+// the combined logsumexp lse_i of the forward pass and G_i = dO_i . O_i,
+// entry (i, j) of any round has
+//   P = exp(s_ij - lse_i),  dS = P (dO_i . v_j - G_i),
+//   dv_j += P dO_i,  dq_i += dS khat_j / sqrt(d),  dkhat_j += dS q_i / sqrt(d),
+// where khat_j = q_j / |q_j| (the shared-QK keys).  Masked entries (another
+// bucket, a later position, the token itself) have no dS; a token alone in
+// every round gives its own value the weight 1/R in each round.
+//
+// Tile = two consecutive chunks of one (round, head) row: 128 query rows,
+// window of three chunks (k-1, k, k+1) = 192 keys, as in the forward kernel.
+// Per tile (TMEM columns in brackets):
+//   S   = Q[128 x 64] . Qw[192 x 64]^T          [0, 192)      tcgen05.mma
+//   dP  = dO[128 x 64] . Vw[192 x 64]^T         [192, 384)    tcgen05.mma
+//   P, dS per entry on the CUDA cores (one TMEM lane = one query row); P^T
+//   and dS^T go to shared memory as MN-major operands, dS scaled by the key
+//   normalisation goes back to TMEM columns [0, 96) (bf16 pairs);
+//   dQ  = dS' [128 x 192] . Qw [192 x 64]       [384, 448)    A from TMEM
+//   dV1 = P^T[w0,w1 ; q0] . dO[q0]              [448, 512)
+//   dV2 = P^T[w1,w2 ; q1] . dO[q1]              [192, 256)
+//   dK1 = dS^T[w0,w1 ; q0] . Q[q0]              [256, 320)
+//   dK2 = dS^T[w1,w2 ; q1] . Q[q1]              [320, 384)
+// Query chunk q0 sees window chunks w0, w1 and q1 sees w1, w2, so the two
+// key-side products cover every entry with M = 128 and no padding.  The
+// accumulators are added into fp32 gradient buffers (vector reductions);
+// they sum over tiles and rounds.  dQ = dq + (dkhat - khat (khat . dkhat))/|q|
+// is formed afterwards per token.
+//
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  two compute warpgroups; warpgroup g takes window chunk
+//                   qc + g of each query row (64 columns) and 32 of the 64
+//                   columns of every accumulator in the drain.
+//   warp 8          producer: gathers the tile's window (q, v rows, packed
+//                   keys, key scales) and its queries' dO rows, lse and G into
+//                   one of two shared-memory slots.
+//   warp 9          one thread issues the MMAs.
+#pragma once
+
+#include "attend_tc.cuh"
+
+namespace lsh {
+
+constexpr int kBwThreads = 320;
+constexpr int kBwSlots = 2;
+constexpr int kBwChunkBytes = 64 * 128;                 // 64 rows of 128 B
+constexpr int kBwSlotBytes = 8 * kBwChunkBytes;         // q x3, v x3, dO x2
+constexpr int kBwOpBytes = 2 * 2 * kBwChunkBytes;       // one MN-major operand pair
+constexpr uint32_t kBwColS = 0, kBwColDP = 192, kBwColDQ = 384, kBwColDV1 = 448,
+                   kBwColDV2 = 192, kBwColDK1 = 256, kBwColDK2 = 320;
+
+struct BwInfo {
+  int r, bh, nq, has_prev, done;
+};
+
+struct BwSmem {
+  uint32_t pos[kBwSlots][192];
+  uint32_t key[kBwSlots][192];
+  float rn[kBwSlots][192];
+  float lse[kBwSlots][128];
+  float G[kBwSlots][128];
+  BwInfo info[kBwSlots];
+  uint64_t full[kBwSlots], empty[kBwSlots];
+  uint64_t s_full, p_full, o_full, tm_free;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct AttnBwdTcArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* V;
+  const __nv_bfloat16* dO;
+  const uint32_t* keys;
+  const int32_t* perm;
+  const float* rn;   // [n_tok] log2(e) / (|q| sqrt(d)), 0 for a zero row
+  const float* lse;  // [n_tok] combined logsumexp of the forward pass
+  const float* G;    // [n_tok] dO . O
+  int L, R, BH, n_chunks, causal;
+  int n_tiles;       // tiles per (round, head) row
+  long long total_tiles;
+  float inv_rounds;
+  float* dq_acc;     // [n_tok][64] fp32, zeroed
+  float* dk_acc;
+  float* dv_acc;
+};
+
+__host__ __device__ inline size_t attend_bwd_tc_smem_bytes() {
+  return 1024 + (size_t)kBwSlots * kBwSlotBytes + 2 * (size_t)kBwOpBytes + sizeof(BwSmem);
+}
+
+// OR of pred over the 256 compute threads (named barrier 1).
+__device__ __forceinline__ bool bw_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// 32 accumulator columns of this lane into row `dst` (fp32, 16-byte aligned)
+__device__ __forceinline__ void drain32(uint32_t taddr, float* dst, bool live) {
+  float v[32];
+  tc::tmem_ld32(taddr, v);
+  tc::tmem_ld_wait();
+  tc::tmem_pin<32>(v);
+  if (live) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) red_add_v4(dst + 4 * q, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* slots = sm;
+  uint8_t* opP = sm + kBwSlots * kBwSlotBytes;  // P^T: [query chunk][window atom][64 rows]
+  uint8_t* opD = opP + kBwOpBytes;              // dS^T / sqrt(d), same layout
+  BwSmem& S = *reinterpret_cast<BwSmem*>(opD + kBwOpBytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < kBwSlots; ++s) {
+      tc::mbar_init(&S.full[s], 32);    // producer lanes
+      tc::mbar_init(&S.empty[s], 256);  // compute threads
+    }
+    tc::mbar_init(&S.s_full, 1);
+    tc::mbar_init(&S.p_full, 256);
+    tc::mbar_init(&S.o_full, 1);
+    tc::mbar_init(&S.tm_free, 256);
+    tc::mbar_init_fence();
+    S.abort = 0;
+  }
+  if (warp == 9) {
+    tc::tmem_alloc(&S.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    for (uint32_t n = 0;; ++n) {
+      const int s = n % kBwSlots;
+      const long long tile = (long long)blockIdx.x + (long long)n * gridDim.x;
+      if (!__all_sync(0xffffffffu, at_wait(&S.empty[s], ((n / kBwSlots) & 1u) ^ 1u, &S.abort)))
+        break;
+      if (tile >= a.total_tiles) {
+        if (lane == 0) S.info[s].done = 1;
+        tc::mbar_arrive(&S.full[s]);
+        break;
+      }
+      const int per_round = a.BH * a.n_tiles;
+      const int r = (int)(tile / per_round);
+      const int rem = (int)(tile - (long long)r * per_round);
+      const int bh = rem / a.n_tiles, t = rem % a.n_tiles;
+      const int k0 = 2 * t;
+      const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
+      const int has_prev = a.n_chunks > 1 ? 1 : 0;
+      const int nq = (k0 + 1 < a.n_chunks) ? 2 : 1;
+      const size_t rowbase = ((size_t)r * a.BH + bh) * a.L;
+      const size_t bhL = (size_t)bh * a.L;
+      uint8_t* slot = slots + (size_t)s * kBwSlotBytes;
+      // window slot u: chunk u/64 of (prev, k0, k0+1); absent chunks read kAtNoKey
+#pragma unroll
+      for (int e = 0; e < 6; ++e) {
+        const int u = lane + 32 * e, cw = u >> 6;
+        const int ch = cw == 0 ? prev : k0 + cw - 1;
+        const bool present = cw == 0 ? has_prev != 0 : (cw == 1 || nq == 2);
+        uint32_t p = present ? (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)] : kAtNoKey;
+        if (p != kAtNoKey && p >= (uint32_t)a.L) {  // not a permutation of the row
+          record_status(kErrBadKeys);
+          p = 0;
+        }
+        S.pos[s][u] = p;
+        if (p != kAtNoKey) {
+          cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + p);
+          cp_async4(tc::smem_u32(&S.rn[s][u]), a.rn + bhL + p);
+          if (u >= 64) {
+            cp_async4(tc::smem_u32(&S.lse[s][u - 64]), a.lse + bhL + p);
+            cp_async4(tc::smem_u32(&S.G[s][u - 64]), a.G + bhL + p);
+          }
+        } else {
+          S.key[s][u] = kAtNoKey;
+          S.rn[s][u] = 0.f;
+          if (u >= 64) {
+            S.lse[s][u - 64] = 0.f;
+            S.G[s][u - 64] = 0.f;
+          }
+        }
+      }
+      __syncwarp();
+      // q and v rows of the window, dO rows of the queries: eight lanes per
+      // 128-byte row, four rows per warp instruction
+      const __nv_bfloat16* Qbh = a.Q + bhL * 64;
+      const __nv_bfloat16* Vbh = a.V + bhL * 64;
+      const __nv_bfloat16* dObh = a.dO + bhL * 64;
+#pragma unroll 2
+      for (int i = 0; i < 48; ++i) {
+        const int u = 4 * i + (lane >> 3), c = lane & 7;
+        const uint32_t p = S.pos[s][u];
+        uint8_t* qd = slot + tc::sw128_offset(u, c);
+        uint8_t* vd = slot + 3 * kBwChunkBytes + tc::sw128_offset(u, c);
+        uint8_t* dd = slot + 6 * kBwChunkBytes + tc::sw128_offset(u - 64, c);
+        if (p != kAtNoKey) {
+          tc::cp_async16(tc::smem_u32(qd), Qbh + (size_t)p * 64 + c * 8);
+          tc::cp_async16(tc::smem_u32(vd), Vbh + (size_t)p * 64 + c * 8);
+          if (u >= 64) tc::cp_async16(tc::smem_u32(dd), dObh + (size_t)p * 64 + c * 8);
+        } else {
+          *reinterpret_cast<uint4*>(qd) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
+          if (u >= 64) *reinterpret_cast<uint4*>(dd) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (lane == 0) {
+        BwInfo inf;
+        inf.r = r;
+        inf.bh = bh;
+        inf.nq = nq;
+        inf.has_prev = has_prev;
+        inf.done = 0;
+        S.info[s] = inf;
+      }
+      // the rows land, become visible to the tensor cores' (async proxy)
+      // reads, then the slot is published
+      tc::cp_async_commit();
+      tc::cp_async_wait<0>();
+      tc::fence_async_smem();
+      __syncwarp();
+      tc::mbar_arrive(&S.full[s]);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_bf16(128, 192, 0, 0);
+      const uint32_t id_q = tc::idesc_bf16(128, 64, 0, 1);
+      const uint32_t id_k = tc::idesc_bf16(128, 64, 1, 1);
+      for (uint32_t n = 0;; ++n) {
+        const int s = n % kBwSlots;
+        if (!at_wait(&S.full[s], (n / kBwSlots) & 1u, &S.abort)) break;
+        if (S.info[s].done) break;
+        const int nq = S.info[s].nq;
+        if (!at_wait(&S.tm_free, (n & 1u) ^ 1u, &S.abort)) break;
+        tc::fence_after_sync();
+        const uint32_t sq = tc::smem_u32(slots + (size_t)s * kBwSlotBytes);
+        const uint32_t sv = sq + 3 * kBwChunkBytes, sdo = sq + 6 * kBwChunkBytes;
+        // S = Q(window rows 64..191) . Qw^T,  dP = dO . Vw^T  (K-major, K = 64)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(tmem + kBwColS, tc::sdesc_sw128(sq + kBwChunkBytes + kk * 32, 16, 1024),
+                       tc::sdesc_sw128(sq + kk * 32, 16, 1024), id_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(tmem + kBwColDP, tc::sdesc_sw128(sdo + kk * 32, 16, 1024),
+                       tc::sdesc_sw128(sv + kk * 32, 16, 1024), id_s, kk > 0);
+        tc::mma_commit(&S.s_full);
+        if (!at_wait(&S.p_full, n & 1u, &S.abort)) break;
+        tc::fence_after_sync();
+        // dQ = dS' (TMEM, 192 keys = 96 columns) . Qw (MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 12; ++kk)
+          tc::mma_bf16_ts(tmem + kBwColDQ, tmem + kBwColS + kk * 8,
+                          tc::sdesc_sw128(sq + (kk >> 2) * kBwChunkBytes + (kk & 3) * 2048, 8192, 1024),
+                          id_q, kk > 0);
+        // key side: A = P^T / dS^T of one query chunk (two 64-key atoms,
+        // MN-major), B = that chunk's dO / q rows (MN-major), K = 64 queries
+        const uint32_t p0 = tc::smem_u32(opP), d0 = tc::smem_u32(opD);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          tc::mma_bf16(tmem + kBwColDV1, tc::sdesc_sw128(p0 + kk * 2048, kBwChunkBytes, 1024),
+                       tc::sdesc_sw128(sdo + kk * 2048, 8192, 1024), id_k, kk > 0);
+          tc::mma_bf16(tmem + kBwColDK1, tc::sdesc_sw128(d0 + kk * 2048, kBwChunkBytes, 1024),
+                       tc::sdesc_sw128(sq + kBwChunkBytes + kk * 2048, 8192, 1024), id_k, kk > 0);
+        }
+        if (nq == 2) {
+          const uint32_t p1 = p0 + 2 * kBwChunkBytes, d1 = d0 + 2 * kBwChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            tc::mma_bf16(tmem + kBwColDV2, tc::sdesc_sw128(p1 + kk * 2048, kBwChunkBytes, 1024),
+                         tc::sdesc_sw128(sdo + kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
+                         kk > 0);
+            tc::mma_bf16(tmem + kBwColDK2, tc::sdesc_sw128(d1 + kk * 2048, kBwChunkBytes, 1024),
+                         tc::sdesc_sw128(sq + 2 * kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
+                         kk > 0);
+          }
+        }
+        tc::mma_commit(&S.o_full);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ compute warpgroups
+    const int g = warp >> 2;            // window chunk qc + g of each row
+    const int m = tid & 127;            // query row = TMEM lane
+    const int qc = m >> 6, qi = m & 63;  // query chunk, row within it
+    const int wc = qc + g;              // this thread's window chunk
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t region = tmem + lane_off;
+    for (uint32_t n = 0;; ++n) {
+      const int s = n % kBwSlots;
+      const bool okf = at_wait(&S.full[s], (n / kBwSlots) & 1u, &S.abort);
+      const BwInfo inf = S.info[s];
+      if (bw_or(!okf || inf.done)) break;
+      const bool valid = qc < inf.nq;
+      const bool active = valid && (wc != 0 || inf.has_prev);
+      const uint32_t ki = S.key[s][64 + m];
+      const uint32_t lo = ki - ki % (uint32_t)a.L;
+      const uint32_t span = a.causal ? (ki - lo) : (uint32_t)a.L;
+      const float lse_i = S.lse[s][m];
+      const float lse2 = lse_i * kLog2e;
+      const float G_i = S.G[s][m];
+      const bool lone = valid && lse_i < kSelfScore + kLoneMargin;
+      const bool oks = at_wait(&S.s_full, n & 1u, &S.abort);
+      if (bw_or(!oks)) break;
+      tc::fence_after_sync();
+
+      uint32_t dsq[32];  // dS scaled by the key normalisation, bf16 pairs
+      // P^T / dS^T operand row: query chunk qc, atom g (window chunk wc), K-row qi
+      uint8_t* prow = opP + qc * 2 * kBwChunkBytes + g * kBwChunkBytes;
+      uint8_t* drow = opD + qc * 2 * kBwChunkBytes + g * kBwChunkBytes;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        const int u0 = 64 * wc + 16 * blk;  // first window column of the block
+        float sv[16], dp[16];
+        tc::tmem_ld16(region + kBwColS + u0, sv);
+        tc::tmem_ld16(region + kBwColDP + u0, dp);
+        tc::tmem_ld_wait();
+        tc::tmem_pin<16>(sv);
+        tc::tmem_pin<16>(dp);
+        uint32_t pp[8], pd[8];
+#pragma unroll
+        for (int jj = 0; jj < 16; jj += 4) {
+          const uint4 k4 = *reinterpret_cast<const uint4*>(&S.key[s][u0 + jj]);
+          const float4 r4 = *reinterpret_cast<const float4*>(&S.rn[s][u0 + jj]);
+          const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
+          const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+          float pv[4], dv[4], qv[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            bool in = active && (kj[x] - lo) < span;
+            if (!a.causal) in = in && kj[x] != ki;
+            const float p = in ? ex2(sv[jj + x] * rj[x] - lse2) : 0.f;
+            const float ds = p * (dp[jj + x] - G_i);
+            pv[x] = p;
+            dv[x] = ds * 0.125f;                    // dkhat side: dS / sqrt(d)
+            qv[x] = ds * (rj[x] * (1.f / kLog2e));  // dq side: dS / (|q_j| sqrt(d))
+          }
+          if (lone) {  // only its own entry, with weight 1/R and no dS
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              pv[x] = (u0 + jj + x == 64 + m) ? a.inv_rounds : 0.f;
+              dv[x] = 0.f;
+              qv[x] = 0.f;
+            }
+          }
+          pp[jj / 2] = pack_bf16(pv[0], pv[1]);
+          pp[jj / 2 + 1] = pack_bf16(pv[2], pv[3]);
+          pd[jj / 2] = pack_bf16(dv[0], dv[1]);
+          pd[jj / 2 + 1] = pack_bf16(dv[2], dv[3]);
+          dsq[8 * blk + jj / 2] = pack_bf16(qv[0], qv[1]);
+          dsq[8 * blk + jj / 2 + 1] = pack_bf16(qv[2], qv[3]);
+        }
+        // 16-byte pieces 2blk, 2blk+1 of the 128-byte operand row
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t off = tc::sw128_offset(qi, 2 * blk + q);
+          *reinterpret_cast<uint4*>(prow + off) =
+              make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+          *reinterpret_cast<uint4*>(drow + off) =
+              make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+        }
+      }
+      // every lane's S and dP are read (both warpgroups): dS' may now go
+      // over S, with zeros for the window chunk outside this row's window
+      bw_or(false);
+      tc::tmem_st32(region + kBwColS + 32 * wc, dsq);
+      if (g != qc) {
+        uint32_t z[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) z[x] = 0u;
+        tc::tmem_st32(region + kBwColS + (qc == 0 ? 64 : 0), z);
+      }
+      tc::tmem_st_wait();
+      tc::fence_async_smem();  // P^T, dS^T rows -> tensor-core reads
+      tc::fence_before_sync();
+      tc::mbar_arrive(&S.p_full);
+
+      const bool oko = at_wait(&S.o_full, n & 1u, &S.abort);
+      if (bw_or(!oko)) break;
+      tc::fence_after_sync();
+      // drain: this warpgroup's 32 of the 64 columns of each accumulator
+      const uint32_t c0 = 32 * g;
+      const size_t bhL = (size_t)inf.bh * a.L;
+      {
+        const uint32_t p = S.pos[s][64 + m];
+        drain32(region + kBwColDQ + c0, a.dq_acc + (bhL + p) * 64 + c0, valid);
+      }
+      {
+        const uint32_t p = S.pos[s][m];  // keys [w0 ; w1]
+        const bool live = p != kAtNoKey;
+        const size_t t = (bhL + (live ? p : 0)) * 64 + c0;
+        drain32(region + kBwColDV1 + c0, a.dv_acc + t, live);
+        drain32(region + kBwColDK1 + c0, a.dk_acc + t, live);
+      }
+      if (inf.nq == 2) {
+        const uint32_t p = S.pos[s][64 + m];  // keys [w1 ; w2]
+        const size_t t = (bhL + p) * 64 + c0;
+        drain32(region + kBwColDV2 + c0, a.dv_acc + t, true);
+        drain32(region + kBwColDK2 + c0, a.dk_acc + t, true);
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&S.tm_free);
+      tc::mbar_arrive(&S.empty[s]);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace lsh

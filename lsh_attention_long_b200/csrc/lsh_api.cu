@@ -8,6 +8,7 @@
 
 #include <mutex>
 
+#include "attend_bwd_tc.cuh"
 #include "attend_simt.cuh"
 #include "attend_tc.cuh"
 #include "common.cuh"
@@ -109,8 +110,9 @@ size_t fwd_ws_bytes(const Dims& D) {
   return m;
 }
 
+// G = dO . O and the key scales per token, then the dq, dkhat, dv accumulators
 size_t bwd_ws_bytes(const Dims& D) {
-  return align_up(D.n_tok * sizeof(float)) + 3 * align_up(D.n_tok * kHeadDim * sizeof(float));
+  return 2 * align_up(D.n_tok * sizeof(float)) + 3 * align_up(D.n_tok * kHeadDim * sizeof(float));
 }
 
 lsh::AttnDims attn_dims(const Dims& D) {
@@ -333,9 +335,11 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   if (!ws || ws_bytes < bwd_ws_bytes(D)) return LSH_ERR_WORKSPACE;
   const lsh::AttnDims a = attn_dims(D);
   char* w = static_cast<char*>(ws);
-  float* G = reinterpret_cast<float*>(w);
+  const size_t tok_bytes = align_up(D.n_tok * sizeof(float));
   const size_t acc_bytes = align_up(D.n_tok * kHeadDim * sizeof(float));
-  float* dq = reinterpret_cast<float*>(w + align_up(D.n_tok * sizeof(float)));
+  float* G = reinterpret_cast<float*>(w);
+  float* rn = reinterpret_cast<float*>(w + tok_bytes);
+  float* dq = reinterpret_cast<float*>(w + 2 * tok_bytes);
   float* dk = reinterpret_cast<float*>(reinterpret_cast<char*>(dq) + acc_bytes);
   float* dv = reinterpret_cast<float*>(reinterpret_cast<char*>(dk) + acc_bytes);
   if (cudaMemsetAsync(dq, 0, 3 * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
@@ -344,13 +348,45 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   lsh::bwd_dot_kernel<T><<<tb, 256, 0, st>>>(static_cast<const T*>(O), static_cast<const T*>(dO),
                                              D.n_tok, G);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  const size_t smem = lsh::simt_bwd_smem_bytes(a.chunk, a.W);
-  lsh_status s0 = allow_smem(lsh::attend_bwd_simt_kernel<T>, smem);
-  if (s0 != LSH_OK) return s0;
-  const dim3 grid((unsigned)a.n_chunks, (unsigned)(D.R * a.BH));
-  lsh::attend_bwd_simt_kernel<T><<<grid, 256, smem, st>>>(
-      q, static_cast<const T*>(V), static_cast<const T*>(dO), keys, perm, lse, G, a,
-      1.f / (float)D.R, dq, dk, dv);
+  if (attend_tc_supported(D)) {
+    lsh::key_scale_kernel<<<tb, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(Q), D.n_tok,
+                                              rn);
+    if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+    lsh::AttnBwdTcArgs b;
+    b.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+    b.V = static_cast<const __nv_bfloat16*>(V);
+    b.dO = static_cast<const __nv_bfloat16*>(dO);
+    b.keys = keys;
+    b.perm = perm;
+    b.rn = rn;
+    b.lse = lse;
+    b.G = G;
+    b.L = D.L;
+    b.R = D.R;
+    b.BH = D.B * D.H;
+    b.n_chunks = D.L / D.c;
+    b.causal = D.causal;
+    b.n_tiles = (b.n_chunks + 1) / 2;
+    b.total_tiles = (long long)D.R * b.BH * b.n_tiles;
+    b.inv_rounds = 1.f / (float)D.R;
+    b.dq_acc = dq;
+    b.dk_acc = dk;
+    b.dv_acc = dv;
+    const size_t smem = lsh::attend_bwd_tc_smem_bytes();
+    lsh_status s0 = allow_smem(lsh::attend_bwd_tc_kernel, smem);
+    if (s0 != LSH_OK) return s0;
+    const long long sms = num_sms();
+    const unsigned grid = (unsigned)(b.total_tiles < sms ? b.total_tiles : sms);
+    lsh::attend_bwd_tc_kernel<<<grid, lsh::kBwThreads, smem, st>>>(b);
+  } else {
+    const size_t smem = lsh::simt_bwd_smem_bytes(a.chunk, a.W);
+    lsh_status s0 = allow_smem(lsh::attend_bwd_simt_kernel<T>, smem);
+    if (s0 != LSH_OK) return s0;
+    const dim3 grid((unsigned)a.n_chunks, (unsigned)(D.R * a.BH));
+    lsh::attend_bwd_simt_kernel<T><<<grid, 256, smem, st>>>(
+        q, static_cast<const T*>(V), static_cast<const T*>(dO), keys, perm, lse, G, a,
+        1.f / (float)D.R, dq, dk, dv);
+  }
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
   lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok, static_cast<T*>(dQ),
                                                   static_cast<T*>(dV));

@@ -196,6 +196,8 @@ BWD_CASES = [
     (1, 1, 256, 1, 2, 64, True),
     (1, 1, 256, 1024, 2, 64, False),
     (1, 2, 64, 4, 1, 4, True),
+    (2, 2, 1024, 64, 3, 64, False),   # sixteen chunks, several tiles per row
+    (1, 2, 1088, 32, 2, 64, True),    # seventeen chunks: last tile has one query chunk
 ]
 
 
