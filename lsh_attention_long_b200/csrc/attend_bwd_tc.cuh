@@ -9,33 +9,41 @@
 // entry (i, j) of any round has
 //   P = exp(s_ij - lse_i),  dS = P (dO_i . v_j - G_i),
 //   dv_j += P dO_i,  dq_i += dS khat_j / sqrt(d),  dkhat_j += dS q_i / sqrt(d),
-// where khat_j = q_j / |q_j| (the shared-QK keys).  Masked entries (another
+// where khat_j = q_j / |q_j| (the shared-QK keys) and dQ = dq + (dkhat -
+// khat (khat . dkhat)) / |q| per token.  Masked entries (another
 // bucket, a later position, the token itself) have no dS; a token alone in
 // every round gives its own value the weight 1/R in each round.
 //
-// Tile = two consecutive chunks of one (round, head) row: 128 query rows,
-// window of three chunks (k-1, k, k+1) = 192 keys, as in the forward kernel.
-// Per tile (TMEM columns in brackets):
-//   S   = Q[128 x 64] . Qw[192 x 64]^T          [0, 192)      tcgen05.mma
-//   dP  = dO[128 x 64] . Vw[192 x 64]^T         [192, 384)    tcgen05.mma
+// Tile = two consecutive chunks k0, k0+1 of one (round, head) row: 128 query
+// rows against a window of three chunks, 192 keys, as in the forward kernel.
+// The window chunks are held in the order [w0, w2, w1] = [k0-1, k0+1, k0]
+// (window column c, chunk c/64); the queries are columns 64..191, so TMEM
+// lane m holds query column 64 + m: chunk k0+1 (q1) for m < 64, k0 (q0) for
+// m >= 64.  Per tile (TMEM columns in brackets):
+//   S   = Q[cols 64..191] . Q[cols 0..191]^T    [0, 192)      tcgen05.mma
+//   dP  = dO[128 x 64] . V[cols 0..191]^T       [192, 384)    tcgen05.mma
 //   P, dS per entry on the CUDA cores (one TMEM lane = one query row); P^T
 //   and dS^T go to shared memory as MN-major operands, dS scaled by the key
-//   normalisation goes back to TMEM columns [0, 96) (bf16 pairs);
-//   dQ  = dS' [128 x 192] . Qw [192 x 64]       [384, 448)    A from TMEM
-//   dV1 = P^T[w0,w1 ; q0] . dO[q0]              [448, 512)
-//   dV2 = P^T[w1,w2 ; q1] . dO[q1]              [192, 256)
-//   dK1 = dS^T[w0,w1 ; q0] . Q[q0]              [256, 320)
-//   dK2 = dS^T[w1,w2 ; q1] . Q[q1]              [320, 384)
-// Query chunk q0 sees window chunks w0, w1 and q1 sees w1, w2, so the two
-// key-side products cover every entry with M = 128 and no padding.  The
-// accumulators are added into fp32 gradient buffers (vector reductions);
-// they sum over tiles and rounds.  dQ = dq + (dkhat - khat (khat . dkhat))/|q|
-// is formed afterwards per token.
+//   normalisation goes to TMEM columns [416, 512) (bf16 pairs);
+//   dQ  = dS' [128 x 192] . Q[cols 0..191]      [0, 64)       A from TMEM
+//   dV1 = P^T[w0 ; w1 | q0] . dO[q0]            [64, 128)
+//   dK1 = dS^T[w0 ; w1 | q0] . Q[q0]            [128, 192)
+//   dV2 = P^T[w2 ; w1 | q1] . dO[q1]            [192, 256)
+//   dK2 = dS^T[w2 ; w1 | q1] . Q[q1]            [256, 320)
+// q0 sees w0, w1 and q1 sees w1, w2.  With this order every accumulator row
+// of a token sits on one TMEM lane: lanes 64..127 hold w1 in dQ, dV1, dK1,
+// dV2 and dK2, lanes 0..63 hold w2 in dQ, dV2, dK2 and w0 in dV1, dK1.  So
+// the drain merges per lane, projects the key gradient onto the query
+// (dq += (dkhat - khat (khat . dkhat)) / |q|, linear, so it can be applied
+// per contribution) and adds two rows per token and tile (dq, dv) into the
+// fp32 gradient buffers with vector reductions; they sum over tiles and
+// rounds.
 //
 // Warp roles (320 threads):
-//   warps 0-3, 4-7  two compute warpgroups; warpgroup g takes window chunk
-//                   qc + g of each query row (64 columns) and 32 of the 64
-//                   columns of every accumulator in the drain.
+//   warps 0-3, 4-7  two compute warpgroups; warpgroup 1 takes the w1 columns
+//                   of every query row, warpgroup 0 the row's other window
+//                   chunk (w0 for q0, w2 for q1); in the drain warpgroup 0
+//                   forms the dq rows and warpgroup 1 the dv rows.
 //   warp 8          producer: gathers the tile's window (q, v rows, packed
 //                   keys, key scales) and its queries' dO rows, lse and G into
 //                   one of two shared-memory slots.
@@ -51,8 +59,12 @@ constexpr int kBwSlots = 2;
 constexpr int kBwChunkBytes = 64 * 128;                 // 64 rows of 128 B
 constexpr int kBwSlotBytes = 8 * kBwChunkBytes;         // q x3, v x3, dO x2
 constexpr int kBwOpBytes = 2 * 2 * kBwChunkBytes;       // one MN-major operand pair
-constexpr uint32_t kBwColS = 0, kBwColDP = 192, kBwColDQ = 384, kBwColDV1 = 448,
-                   kBwColDV2 = 192, kBwColDK1 = 256, kBwColDK2 = 320;
+// TMEM columns: S and dP during the softmax, dS' (bf16 pairs, A of the dQ
+// product) in columns no softmax read touches, the five accumulators over S
+// and dP once both are consumed.
+constexpr uint32_t kBwColS = 0, kBwColDP = 192, kBwColDS = 416;
+constexpr uint32_t kBwColDQ = 0, kBwColDV1 = 64, kBwColDK1 = 128, kBwColDV2 = 192,
+                   kBwColDK2 = 256;
 
 struct BwInfo {
   int r, bh, nq, has_prev, done;
@@ -84,8 +96,7 @@ struct AttnBwdTcArgs {
   int n_tiles;       // tiles per (round, head) row
   long long total_tiles;
   float inv_rounds;
-  float* dq_acc;     // [n_tok][64] fp32, zeroed
-  float* dk_acc;
+  float* dq_acc;     // [n_tok][64] fp32, zeroed: dq with the dkhat projection added
   float* dv_acc;
 };
 
@@ -113,15 +124,86 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                : "memory");
 }
 
-// 32 accumulator columns of this lane into row `dst` (fp32, 16-byte aligned)
-__device__ __forceinline__ void drain32(uint32_t taddr, float* dst, bool live) {
-  float v[32];
-  tc::tmem_ld32(taddr, v);
-  tc::tmem_ld_wait();
-  tc::tmem_pin<32>(v);
-  if (live) {
+// dq row of one token from its accumulator rows on this lane:
+//   dQ (query side, if has_q) + P(dK1 (if k1) + dK2 (if k2)),
+//   P(x) = (x - khat (khat . x)) / |q| with khat = q / |q|,
+// q = the token's bf16 row in shared memory (128B-swizzled), inv = 1/|q|.
+// Sixteen columns at a time: two passes (the projection needs khat . x).
+// Every accumulator is loaded and the absent ones are selected away (a
+// conditional tcgen05.ld costs registers).
+__device__ __forceinline__ void drain_dq(uint32_t region, bool has_q, bool k1, bool k2,
+                                         const uint8_t* qrow, uint32_t qr, float inv, float* dst) {
+  float dot = 0.f;  // q . (dK1 + dK2)
+#pragma unroll 1
+  for (int h = 0; h < 4; ++h) {
+    float x[16], y[16];
+    tc::tmem_ld16(region + kBwColDK1 + 16 * h, x);
+    tc::tmem_ld16(region + kBwColDK2 + 16 * h, y);
+    tc::tmem_ld_wait();
+    tc::tmem_pin<16>(x);
+    tc::tmem_pin<16>(y);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) red_add_v4(dst + 4 * q, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    for (int q = 0; q < 2; ++q) {
+      const uint4 w = *reinterpret_cast<const uint4*>(qrow + tc::sw128_offset(qr, 2 * h + q));
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+        const int j = 8 * q + 2 * e;
+        const float a0 = (k1 ? x[j] : 0.f) + (k2 ? y[j] : 0.f);
+        const float a1 = (k1 ? x[j + 1] : 0.f) + (k2 ? y[j + 1] : 0.f);
+        dot = fmaf(f.x, a0, fmaf(f.y, a1, dot));
+      }
+    }
+  }
+  const float c = dot * inv * inv;  // khat (khat . x) = q (q . x) / |q|^2
+#pragma unroll 1
+  for (int h = 0; h < 4; ++h) {
+    float x[16], y[16], z[16];
+    tc::tmem_ld16(region + kBwColDK1 + 16 * h, x);
+    tc::tmem_ld16(region + kBwColDK2 + 16 * h, y);
+    tc::tmem_ld16(region + kBwColDQ + 16 * h, z);
+    tc::tmem_ld_wait();
+    tc::tmem_pin<16>(x);
+    tc::tmem_pin<16>(y);
+    tc::tmem_pin<16>(z);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 w = *reinterpret_cast<const uint4*>(qrow + tc::sw128_offset(qr, 2 * h + q));
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+        const int j = 8 * q + 2 * e;
+        const float a0 = (k1 ? x[j] : 0.f) + (k2 ? y[j] : 0.f);
+        const float a1 = (k1 ? x[j + 1] : 0.f) + (k2 ? y[j + 1] : 0.f);
+        o[2 * e] = (has_q ? z[j] : 0.f) + (a0 - f.x * c) * inv;
+        o[2 * e + 1] = (has_q ? z[j + 1] : 0.f) + (a1 - f.y * c) * inv;
+      }
+      red_add_v4(dst + 16 * h + 8 * q, o[0], o[1], o[2], o[3]);
+      red_add_v4(dst + 16 * h + 8 * q + 4, o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// dv row of one token: dV1 (if v1) + dV2 (if v2) on this lane
+__device__ __forceinline__ void drain_dv(uint32_t region, bool v1, bool v2, float* dst) {
+#pragma unroll 1
+  for (int h = 0; h < 4; ++h) {
+    float x[16], y[16];
+    tc::tmem_ld16(region + kBwColDV1 + 16 * h, x);
+    tc::tmem_ld16(region + kBwColDV2 + 16 * h, y);
+    tc::tmem_ld_wait();
+    tc::tmem_pin<16>(x);
+    tc::tmem_pin<16>(y);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = (v1 ? x[4 * q + e] : 0.f) + (v2 ? y[4 * q + e] : 0.f);
+      red_add_v4(dst + 16 * h + 4 * q, o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -168,10 +250,12 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
         tc::mbar_arrive(&S.full[s]);
         break;
       }
-      const int per_round = a.BH * a.n_tiles;
-      const int r = (int)(tile / per_round);
-      const int rem = (int)(tile - (long long)r * per_round);
-      const int bh = rem / a.n_tiles, t = rem % a.n_tiles;
+      // head-major order: the rounds of a head follow one another, so the
+      // head's gradient rows stay in L2 while its rounds add into them
+      const int per_head = a.R * a.n_tiles;
+      const int bh = (int)(tile / per_head);
+      const int rem = (int)(tile - (long long)bh * per_head);
+      const int r = rem / a.n_tiles, t = rem % a.n_tiles;
       const int k0 = 2 * t;
       const int prev = (k0 == 0) ? a.n_chunks - 1 : k0 - 1;
       const int has_prev = a.n_chunks > 1 ? 1 : 0;
@@ -179,13 +263,19 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       const size_t rowbase = ((size_t)r * a.BH + bh) * a.L;
       const size_t bhL = (size_t)bh * a.L;
       uint8_t* slot = slots + (size_t)s * kBwSlotBytes;
-      // window slot u: chunk u/64 of (prev, k0, k0+1); absent chunks read kAtNoKey
+      // window column u: chunk u/64 of (prev, k0+1, k0); absent chunks read kAtNoKey
+      uint32_t pe[6];  // all six loads in flight together
 #pragma unroll
       for (int e = 0; e < 6; ++e) {
         const int u = lane + 32 * e, cw = u >> 6;
-        const int ch = cw == 0 ? prev : k0 + cw - 1;
-        const bool present = cw == 0 ? has_prev != 0 : (cw == 1 || nq == 2);
-        uint32_t p = present ? (uint32_t)a.perm[rowbase + (size_t)ch * 64 + (u & 63)] : kAtNoKey;
+        const int ch = cw == 0 ? prev : (cw == 1 ? k0 + 1 : k0);
+        const bool present = cw == 0 ? has_prev != 0 : (cw == 2 || nq == 2);
+        pe[e] = present ? (uint32_t)__ldg(a.perm + rowbase + (size_t)ch * 64 + (u & 63)) : kAtNoKey;
+      }
+#pragma unroll
+      for (int e = 0; e < 6; ++e) {
+        const int u = lane + 32 * e;
+        uint32_t p = pe[e];
         if (p != kAtNoKey && p >= (uint32_t)a.L) {  // not a permutation of the row
           record_status(kErrBadKeys);
           p = 0;
@@ -277,28 +367,29 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
         // dQ = dS' (TMEM, 192 keys = 96 columns) . Qw (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 12; ++kk)
-          tc::mma_bf16_ts(tmem + kBwColDQ, tmem + kBwColS + kk * 8,
+          tc::mma_bf16_ts(tmem + kBwColDQ, tmem + kBwColDS + kk * 8,
                           tc::sdesc_sw128(sq + (kk >> 2) * kBwChunkBytes + (kk & 3) * 2048, 8192, 1024),
                           id_q, kk > 0);
         // key side: A = P^T / dS^T of one query chunk (two 64-key atoms,
-        // MN-major), B = that chunk's dO / q rows (MN-major), K = 64 queries
+        // MN-major), B = that chunk's dO / q rows (MN-major), K = 64 queries.
+        // q0 = columns 128..191 (dO rows 64..127), q1 = columns 64..127.
         const uint32_t p0 = tc::smem_u32(opP), d0 = tc::smem_u32(opD);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           tc::mma_bf16(tmem + kBwColDV1, tc::sdesc_sw128(p0 + kk * 2048, kBwChunkBytes, 1024),
-                       tc::sdesc_sw128(sdo + kk * 2048, 8192, 1024), id_k, kk > 0);
+                       tc::sdesc_sw128(sdo + kBwChunkBytes + kk * 2048, 8192, 1024), id_k, kk > 0);
           tc::mma_bf16(tmem + kBwColDK1, tc::sdesc_sw128(d0 + kk * 2048, kBwChunkBytes, 1024),
-                       tc::sdesc_sw128(sq + kBwChunkBytes + kk * 2048, 8192, 1024), id_k, kk > 0);
+                       tc::sdesc_sw128(sq + 2 * kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
+                       kk > 0);
         }
         if (nq == 2) {
           const uint32_t p1 = p0 + 2 * kBwChunkBytes, d1 = d0 + 2 * kBwChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             tc::mma_bf16(tmem + kBwColDV2, tc::sdesc_sw128(p1 + kk * 2048, kBwChunkBytes, 1024),
-                         tc::sdesc_sw128(sdo + kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
-                         kk > 0);
+                         tc::sdesc_sw128(sdo + kk * 2048, 8192, 1024), id_k, kk > 0);
             tc::mma_bf16(tmem + kBwColDK2, tc::sdesc_sw128(d1 + kk * 2048, kBwChunkBytes, 1024),
-                         tc::sdesc_sw128(sq + 2 * kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
+                         tc::sdesc_sw128(sq + kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
                          kk > 0);
           }
         }
@@ -308,10 +399,11 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
     __syncwarp();
   } else {
     // ------------------------------------------------ compute warpgroups
-    const int g = warp >> 2;            // window chunk qc + g of each row
-    const int m = tid & 127;            // query row = TMEM lane
-    const int qc = m >> 6, qi = m & 63;  // query chunk, row within it
-    const int wc = qc + g;              // this thread's window chunk
+    const int g = warp >> 2;            // 1: the w1 columns; 0: the row's other chunk
+    const int m = tid & 127;            // query row = TMEM lane = window column 64 + m
+    const int qb = m >= 64 ? 0 : 1;     // query chunk: q0 (k0) or q1 (k0+1)
+    const int qi = m & 63;              // K-row in that chunk's key-side operands
+    const int cb = g == 1 ? 128 : (qb == 0 ? 0 : 64);  // first window column of this thread
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t region = tmem + lane_off;
     for (uint32_t n = 0;; ++n) {
@@ -319,8 +411,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       const bool okf = at_wait(&S.full[s], (n / kBwSlots) & 1u, &S.abort);
       const BwInfo inf = S.info[s];
       if (bw_or(!okf || inf.done)) break;
-      const bool valid = qc < inf.nq;
-      const bool active = valid && (wc != 0 || inf.has_prev);
+      const bool valid = qb == 0 || inf.nq == 2;
+      const bool active = valid && (g == 1 || qb == 1 || inf.has_prev);
       const uint32_t ki = S.key[s][64 + m];
       const uint32_t lo = ki - ki % (uint32_t)a.L;
       const uint32_t span = a.causal ? (ki - lo) : (uint32_t)a.L;
@@ -332,20 +424,19 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       if (bw_or(!oks)) break;
       tc::fence_after_sync();
 
-      uint32_t dsq[32];  // dS scaled by the key normalisation, bf16 pairs
-      // P^T / dS^T operand row: query chunk qc, atom g (window chunk wc), K-row qi
-      uint8_t* prow = opP + qc * 2 * kBwChunkBytes + g * kBwChunkBytes;
-      uint8_t* drow = opD + qc * 2 * kBwChunkBytes + g * kBwChunkBytes;
+      // P^T / dS^T operand row: query chunk qb, atom g (w1 is atom 1), K-row qi
+      uint8_t* prow = opP + qb * 2 * kBwChunkBytes + g * kBwChunkBytes;
+      uint8_t* drow = opD + qb * 2 * kBwChunkBytes + g * kBwChunkBytes;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
-        const int u0 = 64 * wc + 16 * blk;  // first window column of the block
+        const int u0 = cb + 16 * blk;  // first window column of the block
         float sv[16], dp[16];
         tc::tmem_ld16(region + kBwColS + u0, sv);
         tc::tmem_ld16(region + kBwColDP + u0, dp);
         tc::tmem_ld_wait();
         tc::tmem_pin<16>(sv);
         tc::tmem_pin<16>(dp);
-        uint32_t pp[8], pd[8];
+        uint32_t pp[8], pd[8], dsq[8];  // P, dS / sqrt(d), dS / (|q_j| sqrt(d)): bf16 pairs
 #pragma unroll
         for (int jj = 0; jj < 16; jj += 4) {
           const uint4 k4 = *reinterpret_cast<const uint4*>(&S.key[s][u0 + jj]);
@@ -375,9 +466,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
           pp[jj / 2 + 1] = pack_bf16(pv[2], pv[3]);
           pd[jj / 2] = pack_bf16(dv[0], dv[1]);
           pd[jj / 2 + 1] = pack_bf16(dv[2], dv[3]);
-          dsq[8 * blk + jj / 2] = pack_bf16(qv[0], qv[1]);
-          dsq[8 * blk + jj / 2 + 1] = pack_bf16(qv[2], qv[3]);
+          dsq[jj / 2] = pack_bf16(qv[0], qv[1]);
+          dsq[jj / 2 + 1] = pack_bf16(qv[2], qv[3]);
         }
+        tc::tmem_st8(region + kBwColDS + u0 / 2, dsq);
         // 16-byte pieces 2blk, 2blk+1 of the 128-byte operand row
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -388,15 +480,11 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
               make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
         }
       }
-      // every lane's S and dP are read (both warpgroups): dS' may now go
-      // over S, with zeros for the window chunk outside this row's window
-      bw_or(false);
-      tc::tmem_st32(region + kBwColS + 32 * wc, dsq);
-      if (g != qc) {
+      if (g == 1) {  // zeros for the window chunk outside the row's window (w2 / w0)
         uint32_t z[32];
 #pragma unroll
         for (int x = 0; x < 32; ++x) z[x] = 0u;
-        tc::tmem_st32(region + kBwColS + (qc == 0 ? 64 : 0), z);
+        tc::tmem_st32(region + kBwColDS + (qb == 0 ? 32 : 0), z);
       }
       tc::tmem_st_wait();
       tc::fence_async_smem();  // P^T, dS^T rows -> tensor-core reads
@@ -406,25 +494,25 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       const bool oko = at_wait(&S.o_full, n & 1u, &S.abort);
       if (bw_or(!oko)) break;
       tc::fence_after_sync();
-      // drain: this warpgroup's 32 of the 64 columns of each accumulator
-      const uint32_t c0 = 32 * g;
+      // drain, merged per lane: lanes 64..127 hold the w1 token of column
+      // 64 + m, lanes 0..63 the w2 token of column 64 + m and the w0 token of
+      // column m; warpgroup 0 adds the dq rows, warpgroup 1 the dv rows
       const size_t bhL = (size_t)inf.bh * a.L;
-      {
-        const uint32_t p = S.pos[s][64 + m];
-        drain32(region + kBwColDQ + c0, a.dq_acc + (bhL + p) * 64 + c0, valid);
-      }
-      {
-        const uint32_t p = S.pos[s][m];  // keys [w0 ; w1]
-        const bool live = p != kAtNoKey;
-        const size_t t = (bhL + (live ? p : 0)) * 64 + c0;
-        drain32(region + kBwColDV1 + c0, a.dv_acc + t, live);
-        drain32(region + kBwColDK1 + c0, a.dk_acc + t, live);
-      }
-      if (inf.nq == 2) {
-        const uint32_t p = S.pos[s][64 + m];  // keys [w1 ; w2]
-        const size_t t = (bhL + p) * 64 + c0;
-        drain32(region + kBwColDV2 + c0, a.dv_acc + t, true);
-        drain32(region + kBwColDK2 + c0, a.dk_acc + t, true);
+      const bool two = inf.nq == 2;
+      const uint8_t* qrows = slots + (size_t)s * kBwSlotBytes;
+      const float inv_scale = 8.f / kLog2e;  // rn * 8 / log2(e) = 1 / |q|
+#pragma unroll 1
+      for (int rr = 0; rr < 2; ++rr) {  // at most two tokens per lane (warp-uniform)
+        // rr 0: column 64 + m (w1 for q0 lanes, w2 for q1 lanes); rr 1: w0, column m
+        const bool w1row = qb == 0;
+        if (rr == 0 ? (!w1row && !two) : (w1row || !inf.has_prev)) continue;
+        const uint32_t c = rr == 0 ? 64 + m : m;
+        // accumulators holding this token on this lane
+        const bool acc1 = rr == 1 || w1row;       // dV1 / dK1
+        const bool acc2 = rr == 0 && (!w1row || two);  // dV2 / dK2
+        float* dst = (g == 0 ? a.dq_acc : a.dv_acc) + (bhL + S.pos[s][c]) * 64;
+        if (g == 0) drain_dq(region, rr == 0, acc1, acc2, qrows, c, S.rn[s][c] * inv_scale, dst);
+        else drain_dv(region, acc1, acc2, dst);
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&S.tm_free);

@@ -392,7 +392,8 @@ attend_bwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V, const T
   }
 }
 
-// dQ = dq + (dkhat - khat (khat . dkhat)) / |q|,  dV = dv, cast to T.
+// dQ = dq + (dkhat - khat (khat . dkhat)) / |q|,  dV = dv, cast to T.  With
+// dk_acc null the projection is already inside dq (dQ = dq).
 template <typename T>
 __global__ void bwd_finalize_kernel(const T* __restrict__ Q, const float* __restrict__ dq_acc,
                                     const float* __restrict__ dk_acc,
@@ -400,6 +401,16 @@ __global__ void bwd_finalize_kernel(const T* __restrict__ Q, const float* __rest
                                     T* __restrict__ dQ, T* __restrict__ dV) {
   const size_t tok = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tok >= n_tok) return;
+  if (!dk_acc) {
+    for (int k = 0; k < kHeadDim; k += 8) {
+      float dq[8], dv[8];
+      load8(dq_acc + tok * kHeadDim + k, dq);
+      load8(dv_acc + tok * kHeadDim + k, dv);
+      store8(dQ + tok * kHeadDim + k, dq);
+      store8(dV + tok * kHeadDim + k, dv);
+    }
+    return;
+  }
   float q[kHeadDim], dk[kHeadDim];
   float ss = 0.f, proj = 0.f;
   for (int k = 0; k < kHeadDim; k += 8) {

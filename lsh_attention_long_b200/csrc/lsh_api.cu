@@ -340,15 +340,17 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   float* G = reinterpret_cast<float*>(w);
   float* rn = reinterpret_cast<float*>(w + tok_bytes);
   float* dq = reinterpret_cast<float*>(w + 2 * tok_bytes);
-  float* dk = reinterpret_cast<float*>(reinterpret_cast<char*>(dq) + acc_bytes);
-  float* dv = reinterpret_cast<float*>(reinterpret_cast<char*>(dk) + acc_bytes);
-  if (cudaMemsetAsync(dq, 0, 3 * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
+  float* dv = reinterpret_cast<float*>(reinterpret_cast<char*>(dq) + acc_bytes);
+  float* dk = reinterpret_cast<float*>(reinterpret_cast<char*>(dv) + acc_bytes);
+  // the tensor-core kernel projects dkhat into dq itself: no dk accumulator
+  const bool tc_path = attend_tc_supported(D);
+  if (cudaMemsetAsync(dq, 0, (tc_path ? 2 : 3) * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
   const T* q = static_cast<const T*>(Q);
   const unsigned tb = (unsigned)((D.n_tok + 255) / 256);
   lsh::bwd_dot_kernel<T><<<tb, 256, 0, st>>>(static_cast<const T*>(O), static_cast<const T*>(dO),
                                              D.n_tok, G);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  if (attend_tc_supported(D)) {
+  if (tc_path) {
     lsh::key_scale_kernel<<<tb, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(Q), D.n_tok,
                                               rn);
     if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
@@ -370,7 +372,6 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
     b.total_tiles = (long long)D.R * b.BH * b.n_tiles;
     b.inv_rounds = 1.f / (float)D.R;
     b.dq_acc = dq;
-    b.dk_acc = dk;
     b.dv_acc = dv;
     const size_t smem = lsh::attend_bwd_tc_smem_bytes();
     lsh_status s0 = allow_smem(lsh::attend_bwd_tc_kernel, smem);
@@ -388,8 +389,8 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
         1.f / (float)D.R, dq, dk, dv);
   }
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok, static_cast<T*>(dQ),
-                                                  static_cast<T*>(dV));
+  lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv, D.n_tok,
+                                                  static_cast<T*>(dQ), static_cast<T*>(dV));
   return last_launch();
 }
 
