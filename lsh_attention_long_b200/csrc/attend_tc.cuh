@@ -45,15 +45,16 @@
 // Two output modes:
 //   partial  every round's normalised o_r (fp32) and lse_r go to o_part /
 //            lse_r at original positions (the combine runs afterwards);
-//   online   rounds of a head are taken in order; each round folds its
-//            result into a running (max, sum, unnormalised output) per token
-//            kept in the workspace, and the last round writes O (bf16) and
-//            lse.  A tile of round r of a head waits (bounded spin) until
-//            every tile of round r-1 of that head is done (per-head tile
-//            counters); tickets are handed out in an order where that
-//            dependency always points to earlier tickets, so the scheme
-//            cannot deadlock.  Heads are taken in
-//            blocks sized so that a block's running state and q, v rows stay
+//   online   each round folds its result into a running (max, sum,
+//            unnormalised output) per token kept in the workspace; even
+//            rounds fold into one running state and odd rounds into a second,
+//            and online_merge_kernel joins the two into O (bf16) and lse.  A
+//            tile of round r of a head waits (bounded spin) until every tile
+//            of round r-2 of that head is done (per-head tile counters), so
+//            consecutive rounds of a head overlap; tickets are handed out in
+//            an order where that dependency always points to earlier
+//            tickets, so the scheme cannot deadlock.  Heads are taken in
+//            blocks sized so that a block's running states and q, v rows stay
 //            resident in L2 while its rounds run.
 #pragma once
 
@@ -102,10 +103,8 @@ struct AttnTcArgs {
   int online;
   float* o_part;     // partial mode
   float* lse_r;
-  float* acc_o;      // online mode: [n_tok][64] unnormalised output
-  float4* acc_ml;    // online mode: [n_tok] (running max, running sum, -, -)
-  __nv_bfloat16* O;  // online mode, last round
-  float* lse;
+  float* acc_o;      // online mode: [2][n_tok][64] unnormalised output (even, odd rounds)
+  float4* acc_ml;    // online mode: [2][n_tok] (running max, running sum, -, -)
   unsigned* counters;  // [BH][R] tiles done; then one ticket counter
 };
 
@@ -426,20 +425,29 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       }
       __syncwarp();
       // q and v rows, eight lanes per 128-byte row (coalesced per row): four
-      // rows per warp instruction instead of 32 scattered 16-byte pieces
-#pragma unroll 2
-      for (int i = 0; i < 48; ++i) {
-        const int u = 4 * i + (lane >> 3), c = lane & 7;
-        const int cw = u >> 6, row = u & 63;
-        uint8_t* qd = slot + cw * kAtChunkBytes + tc::sw128_offset(row, c);
-        uint8_t* vd = slot + (3 + cw) * kAtChunkBytes + tc::sw128_offset(row, c);
-        const uint32_t p = S.pos[s][u];
-        if (p != kAtNoKey) {
-          tc::cp_async16(tc::smem_u32(qd), Qbh + (size_t)p * 64 + c * 8);
-          tc::cp_async16(tc::smem_u32(vd), Vbh + (size_t)p * 64 + c * 8);
-        } else {
-          *reinterpret_cast<uint4*>(qd) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
+      // rows per warp instruction; lane group G takes window rows 48G..48G+47
+      // and reads their positions four at a time
+      {
+        const int G = lane >> 3, c = lane & 7;
+#pragma unroll 1
+        for (int i0 = 0; i0 < 48; i0 += 4) {
+          const uint4 p4 = *reinterpret_cast<const uint4*>(&S.pos[s][48 * G + i0]);
+          const uint32_t pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const int u = 48 * G + i0 + x;
+            const int cw = u >> 6, row = u & 63;
+            uint8_t* qd = slot + cw * kAtChunkBytes + tc::sw128_offset(row, c);
+            uint8_t* vd = qd + 3 * kAtChunkBytes;
+            const uint32_t p = pv[x];
+            if (p != kAtNoKey) {
+              tc::cp_async16(tc::smem_u32(qd), Qbh + (size_t)p * 64 + c * 8);
+              tc::cp_async16(tc::smem_u32(vd), Vbh + (size_t)p * 64 + c * 8);
+            } else {
+              *reinterpret_cast<uint4*>(qd) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4*>(vd) = make_uint4(0, 0, 0, 0);
+            }
+          }
         }
       }
       __syncwarp();
@@ -587,13 +595,14 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const AtInfo inf = S.info[s];
       if (wg_or(w, !okf || inf.done)) break;
 
-      if (a.online && inf.r > 0) {  // rounds of a head run in order
-        // every tile of round r-1 of this head must be folded in; the last
-        // (head, round) seen complete is cached so later tiles skip the load
+      if (a.online && inf.r >= 2) {
+        // every tile of round r-2 of this head (the same running state) must
+        // be folded in; the last (head, round) seen complete is cached so
+        // later tiles skip the load
         bool waited = true;
         if (!(S.dep_bh == inf.bh && S.dep_r == inf.r)) {
           if (m == 0) {
-            const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 1);
+            const unsigned* c = a.counters + (size_t)inf.bh * a.R + (inf.r - 2);
             const long long t0 = clock64();
             while (ld_acquire(c) < (unsigned)a.n_tiles) {
               if (*(volatile int*)&S.abort) { waited = false; break; }
@@ -614,7 +623,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
       const uint32_t ki = S.key[s][64 + m];
       const size_t tok = (size_t)inf.bh * a.L + S.pos[s][64 + m];
       const size_t bhL = (size_t)inf.bh * a.L;
-      const bool fold = a.online && inf.r > 0 && valid;  // uniform per warp
+      const bool fold = a.online && inf.r >= 2 && valid;  // uniform per warp
+      // this round's running state (online mode)
+      float* acc_o = a.acc_o + (size_t)(inf.r & 1) * n_tok * 64;
+      float4* acc_ml = a.acc_ml + (size_t)(inf.r & 1) * n_tok;
 
       // running state of this warp's 32 rows: staged by cp.async while the
       // softmax runs, sixteen lanes per 256-byte row
@@ -624,9 +636,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
           const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
           const size_t t2 = bhL + S.pos[s][64 + rr];
           tc::cp_async16(tc::smem_u32(wg_acc + (size_t)rr * 256 + ((q ^ (rr & 15)) << 4)),
-                         a.acc_o + t2 * 64 + 4 * q);
+                         acc_o + t2 * 64 + 4 * q);
         }
-        tc::cp_async16(tc::smem_u32(&ml_s[w * 128 + m]), a.acc_ml + tok);
+        tc::cp_async16(tc::smem_u32(&ml_s[w * 128 + m]), acc_ml + tok);
       }
       tc::cp_async_commit();
 
@@ -701,13 +713,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         eb = __expf(m_r - M);
         Lsum = ml.y * ea + l_r * eb;
       }
-      const bool last_round = inf.r + 1 == a.R;
-      const bool out_bf16 = a.online && last_round;
-      const float scale = !a.online ? 1.f / l_r : (last_round ? eb / Lsum : eb);
-      const float scale_acc = last_round ? ea / Lsum : ea;
+      const float scale = !a.online ? 1.f / l_r : eb;
+      const float scale_acc = ea;
       uint8_t* my_row = wg_acc + (size_t)m * 256;
       // O in two 32-column halves; the result goes back into this row's
-      // staging space (fp32, or bf16 for the final output)
+      // staging space (fp32)
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         float o[32];
@@ -735,57 +745,29 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             o[4 * q + 2] = fmaf(f.z, scale_acc, o[4 * q + 2]);
             o[4 * q + 3] = fmaf(f.w, scale_acc, o[4 * q + 3]);
           }
-          if (!out_bf16)
-            *reinterpret_cast<float4*>(piece) =
-                make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        }
-        if (out_bf16) {  // 64 B of bf16 per half: pieces 4hh .. 4hh+3 of a 128-B row
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 b;
-            b.x = pack_bf16(o[8 * q], o[8 * q + 1]);
-            b.y = pack_bf16(o[8 * q + 2], o[8 * q + 3]);
-            b.z = pack_bf16(o[8 * q + 4], o[8 * q + 5]);
-            b.w = pack_bf16(o[8 * q + 6], o[8 * q + 7]);
-            // bf16 piece 4hh+q takes the place of fp32 piece 4hh+q, which
-            // the first half (hh = 0) has already read; the pieces the
-            // second half still reads (8..15) are not touched
-            *reinterpret_cast<uint4*>(my_row + (((4 * hh + q) ^ (m & 15)) << 4)) = b;
-          }
+          *reinterpret_cast<float4*>(piece) =
+              make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         }
       }
       if (valid) {
         if (!a.online)
           a.lse_r[(size_t)inf.r * n_tok + tok] = lone ? kSelfScore : m_r + logf(l_r);
-        else if (!last_round)
-          __stcg(a.acc_ml + tok, make_float4(M, Lsum, 0.f, 0.f));
-        else if (a.lse)
-          a.lse[tok] = M + logf(Lsum);
+        else
+          __stcg(acc_ml + tok, make_float4(M, Lsum, 0.f, 0.f));
       }
       __syncwarp();
-      // the warp's 32 result rows to their original positions, coalesced
-      // per row: fp32 rows by sixteen lanes (256 B), bf16 rows by eight (128 B)
+      // the warp's 32 result rows (fp32) to their original positions,
+      // sixteen lanes per 256-byte row
       if (valid) {
-        if (!out_bf16) {
-          float* base = !a.online ? a.o_part + (size_t)inf.r * n_tok * 64 : a.acc_o;
+        float* base = !a.online ? a.o_part + (size_t)inf.r * n_tok * 64 : acc_o;
 #pragma unroll 2
-          for (int i = 0; i < 16; ++i) {
-            const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
-            const size_t t2 = bhL + S.pos[s][64 + rr];
-            const float4 f =
-                *reinterpret_cast<const float4*>(wg_acc + (size_t)rr * 256 + ((q ^ (rr & 15)) << 4));
-            if (!a.online) *reinterpret_cast<float4*>(base + t2 * 64 + 4 * q) = f;
-            else __stcg(reinterpret_cast<float4*>(base + t2 * 64 + 4 * q), f);
-          }
-        } else {
-#pragma unroll 2
-          for (int i = 0; i < 8; ++i) {
-            const int rr = wrow0 + 4 * i + (lane >> 3), q = lane & 7;
-            const size_t t2 = bhL + S.pos[s][64 + rr];
-            const uint4 b = *reinterpret_cast<const uint4*>(wg_acc + (size_t)rr * 256 +
-                                                            ((q ^ (rr & 15)) << 4));
-            *reinterpret_cast<uint4*>(a.O + t2 * 64 + 8 * q) = b;
-          }
+        for (int i = 0; i < 16; ++i) {
+          const int rr = wrow0 + 2 * i + (lane >> 4), q = lane & 15;
+          const size_t t2 = bhL + S.pos[s][64 + rr];
+          const float4 f =
+              *reinterpret_cast<const float4*>(wg_acc + (size_t)rr * 256 + ((q ^ (rr & 15)) << 4));
+          if (!a.online) *reinterpret_cast<float4*>(base + t2 * 64 + 4 * q) = f;
+          else __stcg(reinterpret_cast<float4*>(base + t2 * 64 + 4 * q), f);
         }
       }
       tc::mbar_arrive(&S.empty[s]);
@@ -804,7 +786,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             record_status(tc::kErrTimeout);
             *(volatile int*)&S.abort = 1;
           }
-          S.pub_bh[k] = last_round ? -1 : (int)inf.bh;  // the last round has no waiter
+          S.pub_bh[k] = inf.r + 2 < a.R ? (int)inf.bh : -1;  // rounds without a waiter
           S.pub_r[k] = inf.r;
           st_release_cta(&S.pub_seq[k], n + 1);
         }
@@ -814,6 +796,31 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 9) tc::tmem_dealloc(tmem, 512);
+}
+
+// O and lse from the running states of the even and the odd rounds (online
+// mode): M = max(M_0, M_1), L = sum_b L_b e^(M_b - M),
+// O = sum_b acc_b e^(M_b - M) / L, lse = M + ln L.  Eight threads per token.
+__global__ void online_merge_kernel(const float* __restrict__ acc_o,
+                                    const float4* __restrict__ acc_ml, int nbuf, size_t n_tok,
+                                    __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
+  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= n_tok * 8) return;
+  const size_t tok = g >> 3;
+  const int k = (int)(g & 7) * 8;
+  const float4 m0 = acc_ml[tok];
+  const float4 m1 = nbuf > 1 ? acc_ml[n_tok + tok] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+  const float M = fmaxf(m0.x, m1.x);
+  const float e0 = __expf(m0.x - M), e1 = nbuf > 1 ? __expf(m1.x - M) : 0.f;
+  const float Lsum = m0.y * e0 + m1.y * e1;
+  const float r = 1.f / Lsum;
+  float a0[8], a1[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+  load8(acc_o + tok * kHeadDim + k, a0);
+  if (nbuf > 1) load8(acc_o + (n_tok + tok) * kHeadDim + k, a1);
+#pragma unroll
+  for (int x = 0; x < 8; ++x) o[x] = (a0[x] * e0 + a1[x] * e1) * r;
+  store8(O + tok * kHeadDim + k, o);
+  if (lse && k == 0) lse[tok] = M + logf(Lsum);
 }
 
 }  // namespace lsh

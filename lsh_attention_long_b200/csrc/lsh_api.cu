@@ -88,9 +88,11 @@ size_t attend_fwd_ws_bytes(const Dims& D, bool has_o_part, bool has_lse_r, bool 
   if (attend_tc_supported(D)) {
     // counters, per-token key scale, then the running state or the partials
     const size_t base = counters_bytes(D) + align_up(D.n_tok * sizeof(float));
-    if (has_O && !has_o_part && !has_lse_r)  // online combine: running state per token
-      return base + align_up(D.n_tok * kHeadDim * sizeof(float)) +
-             align_up(D.n_tok * sizeof(float4));
+    if (has_O && !has_o_part && !has_lse_r) {  // online combine: running states per token
+      const size_t nbuf = D.R > 1 ? 2 : 1;     // even and odd rounds
+      return base + align_up(nbuf * D.n_tok * kHeadDim * sizeof(float)) +
+             align_up(nbuf * D.n_tok * sizeof(float4));
+    }
     const size_t all = (size_t)D.R * D.n_tok;  // every round's partials
     return base + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
            (has_lse_r ? 0 : align_up(all * sizeof(float)));
@@ -222,11 +224,12 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   a.n_tiles = (a.n_chunks + 1) / 2;
   a.tpi = a.n_tiles < 4 ? a.n_tiles : 4;
   a.ipr = (a.n_tiles + a.tpi - 1) / a.tpi;
-  // heads whose running state and q, v rows share L2 while their rounds
+  // heads whose running states and q, v rows share L2 while their rounds
   // run: enough items between dependent rounds to cover one wave of CTAs
-  const size_t per_head = (size_t)D.L * (kHeadDim * 4 + 8 + 2 * kHeadDim * 2);
+  const size_t nbuf = D.R > 1 ? 2 : 1;
+  const size_t per_head = (size_t)D.L * (nbuf * (kHeadDim * 4 + 16) + 2 * kHeadDim * 2);
   const int sms = num_sms();
-  long long hpb = (long long)((96ull << 20) / per_head);
+  long long hpb = (long long)((112ull << 20) / per_head);
   const long long want = (2LL * sms + a.ipr - 1) / a.ipr;
   if (hpb > want) hpb = want;
   if (hpb < 1) hpb = 1;
@@ -242,13 +245,11 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   w += align_up(D.n_tok * sizeof(float));
   a.acc_o = nullptr;
   a.acc_ml = nullptr;
-  a.O = static_cast<__nv_bfloat16*>(O);
-  a.lse = lse;
   a.o_part = o_part;
   a.lse_r = lse_r;
   if (online) {
     a.acc_o = reinterpret_cast<float*>(w);
-    w += align_up(D.n_tok * kHeadDim * sizeof(float));
+    w += align_up(nbuf * D.n_tok * kHeadDim * sizeof(float));
     a.acc_ml = reinterpret_cast<float4*>(w);
   } else {
     const size_t all = (size_t)D.R * D.n_tok;
@@ -267,9 +268,14 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   const long long grid = a.n_items < sms ? a.n_items : sms;
   lsh::attend_tc_kernel<<<(unsigned)grid, lsh::kAtThreads, smem, st>>>(a);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  if (!online && O) {
-    const size_t n = D.n_tok * 8;
-    lsh::combine_kernel<__nv_bfloat16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+  const size_t n8 = D.n_tok * 8;
+  if (online) {
+    lsh::online_merge_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
+        a.acc_o, a.acc_ml, (int)nbuf, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
+    return last_launch();
+  }
+  if (O) {
+    lsh::combine_kernel<__nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
         a.o_part, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
     return last_launch();
   }
