@@ -437,8 +437,17 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
         tc::tmem_pin<16>(sv);
         tc::tmem_pin<16>(dp);
         uint32_t pp[8], pd[8], dsq[8];  // P, dS / sqrt(d), dS / (|q_j| sqrt(d)): bf16 pairs
+        // the block's packed keys ascend: a row can have allowed columns in it
+        // only if [key[u0], key[u0+15]] meets [lo, lo + span) (or its own
+        // column is here and it is alone); a block no row of the warp uses is zero
+        const bool any = (active && S.key[s][u0 + 15] >= lo && S.key[s][u0] < lo + span) ||
+                         (lone && (uint32_t)(64 + m - u0) < 16u);
+        const bool skip = !__any_sync(0xffffffffu, any);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) { pp[x] = 0u; pd[x] = 0u; dsq[x] = 0u; }
 #pragma unroll
         for (int jj = 0; jj < 16; jj += 4) {
+          if (skip) break;
           const uint4 k4 = *reinterpret_cast<const uint4*>(&S.key[s][u0 + jj]);
           const float4 r4 = *reinterpret_cast<const float4*>(&S.rn[s][u0 + jj]);
           const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};

@@ -225,6 +225,43 @@ __device__ __forceinline__ void mask32(float* v, const uint32_t* kw, const float
   }
 }
 
+// P (bf16 pairs into pk) for 32 window columns and their sum into ls: a
+// column in the query's bucket and allowed gets exp2(s * r_j - ref2), any
+// other column 0.  With `scaled` the scores are already masked and scaled
+// (the exact route) and only ref2 is subtracted.  The block's packed keys are
+// ascending (a piece of the sorted row), so a row can only have allowed
+// columns in it if [kw[0], kw[31]] meets [lo, lo + span); when no row of the
+// warp does, the block is all zeros and its exponentials are skipped.
+__device__ __forceinline__ void softmax32(const float* v, const uint32_t* kw, const float* rw,
+                                          uint32_t lo, uint32_t span, uint32_t ki, bool active,
+                                          bool causal, bool scaled, float ref2, float* ls,
+                                          uint32_t* pk) {
+  const bool any = active && kw[31] >= lo && kw[0] < lo + span;  // lo + span <= nb * L < 2^31
+  if (!__any_sync(0xffffffffu, any)) {
+#pragma unroll
+    for (int x = 0; x < 16; ++x) pk[x] = 0u;
+    return;
+  }
+#pragma unroll
+  for (int jj = 0; jj < 32; jj += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(kw + jj);
+    const float4 r4 = *reinterpret_cast<const float4*>(rw + jj);
+    const uint32_t kj[4] = {k4.x, k4.y, k4.z, k4.w};
+    const float rj[4] = {r4.x, r4.y, r4.z, r4.w};
+    float p[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      bool in = active && (kj[x] - lo) < span;
+      if (!causal) in = in && kj[x] != ki;
+      const float t = scaled ? v[jj + x] - ref2 : fmaf(v[jj + x], rj[x], -ref2);
+      p[x] = ex2((scaled || in) ? t : -INFINITY);
+    }
+    ls[(jj >> 2) & 3] += (p[0] + p[1]) + (p[2] + p[3]);
+    pk[jj / 2] = pack_bf16(p[0], p[1]);
+    pk[jj / 2 + 1] = pack_bf16(p[2], p[3]);
+  }
+}
+
 // Exact route for rows with a large score bound: writes the masked scores
 // back over S and returns the row maximum (log2 units; 0 if all masked).
 // Out of line: rarely taken, kept out of the hot loop's instruction cache.
@@ -670,17 +707,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
         float v[32];
         tc::tmem_ld32(region + qc * 64 + 32 * c, v);
         tc::tmem_ld_wait();
-        if (!exact)
-          mask32(v, &S.key[s][kc * 64 + 32 * (c & 1)], &S.rn[s][kc * 64 + 32 * (c & 1)], lo,
-                 span, ki, valid && (kc != 0 || inf.has_prev), a.causal != 0);
+        tc::tmem_pin<32>(v);
         uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float p0 = ex2(v[2 * x] - ref2);
-          const float p1 = ex2(v[2 * x + 1] - ref2);
-          ls[x & 3] += p0 + p1;
-          pk[x] = pack_bf16(p0, p1);
-        }
+        softmax32(v, &S.key[s][kc * 64 + 32 * (c & 1)], &S.rn[s][kc * 64 + 32 * (c & 1)], lo, span,
+                  ki, valid && (kc != 0 || inf.has_prev), a.causal != 0, exact, ref2, ls, pk);
         tc::tmem_st16(region + kc * 32 + 16 * (c & 1), pk);
       }
       {
