@@ -53,6 +53,8 @@ def parse_args():
     p.add_argument("--workload", default=HEADLINE)
     p.add_argument("--no-extras", action="store_true",
                    help="headline only: skip fwd+bwd, e2e and the CPU baseline")
+    p.add_argument("--ref-seconds", type=float, default=150.0,
+                   help="--impl reference: CPU seconds of oracle sampling over all steps")
     return p.parse_args()
 
 
@@ -79,6 +81,13 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def aggregate_tokens_per_s(world: int, tokens_per_rank_step: int, steps: int,
+                           max_ms: float) -> float:
+    """Whole-job throughput: every rank runs its own copy of the workload
+    (weak scaling), timed by the slowest rank."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
 def max_over_ranks(x: float, world: int) -> float:
@@ -258,8 +267,9 @@ def run_ours(args, world, rank):
         raise RuntimeError("device status error in the timed region")
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
-    launches_per_step = 1 + 1 + (2 if R > 1 else 1)
-    value = world * B * Lx * args.steps / (total_ms / 1e3)
+    # hash_tc, sort_rows, then key_scale + attend_tc + online_merge
+    launches_per_step = 1 + 1 + 3
+    value = aggregate_tokens_per_s(world, B * Lx, args.steps, total_ms)
 
     peaks, peak_kind = load_peaks()
     work = stage_work(w)
@@ -347,7 +357,7 @@ def run_e2e(args, w, world):
     ms = max_over_ranks(ms, world)
     bi = sum(host[k].numel() * host[k].element_size() for k in ("Q", "V", "rot"))
     bo = O_host.numel() * O_host.element_size()
-    return {"value": round(world * w.B * w.L * steps / (ms / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(aggregate_tokens_per_s(world, w.B * w.L, steps, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
@@ -396,7 +406,7 @@ def run_fwd_bwd(args, w, world):
     if L.lsh_device_status() != 0:
         raise RuntimeError("device status error in fwd+bwd")
     tot = max_over_ranks(fwd + bwd, world)
-    return {"value": round(world * w.B * w.L * steps / (tot / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(aggregate_tokens_per_s(world, w.B * w.L, steps, tot), 1), "unit": "tokens/s",
             "ms_fwd": round(fwd / steps, 4), "ms_bwd": round(bwd / steps, 4), "steps": steps,
             "config": {"B": w.B, "H": w.H, "L": w.L, "n_buckets": w.n_buckets,
                        "n_rounds": w.n_rounds, "chunk": w.chunk, "causal": w.causal}}
@@ -488,11 +498,14 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     s = OracleSampler(w)
-    # a few minutes in all: about 150 s of sampling over warm-up + timed steps
-    per_step = 150.0 / (args.warmup + args.steps)
-    probe, _ = s.step(256, 4)
+    # a few minutes in all: about --ref-seconds of sampling over warm-up + timed steps
+    per_step = args.ref_seconds / (args.warmup + args.steps)
+    max_chunks = w.L // w.chunk
+    probe_tok, probe_chunks = min(256, w.L), min(4, max_chunks)
+    probe, _ = s.step(probe_tok, probe_chunks)
     scale = max(1.0, min(32.0, per_step / max(probe, 1e-3)))
-    n_tok, n_chunks = int(256 * scale), max(1, int(4 * scale))
+    n_tok = min(int(probe_tok * scale), w.L)
+    n_chunks = min(max(1, int(probe_chunks * scale)), max_chunks)
     full = []
     for i in range(args.warmup + args.steps):
         _, f = s.step(n_tok, n_chunks)
