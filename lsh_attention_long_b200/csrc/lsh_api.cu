@@ -191,16 +191,33 @@ lsh_status hash_launch(const Dims& D, const void* Q, const void* rot, uint32_t* 
 
 lsh_status sort_launch(const Dims& D, const uint32_t* keys, int32_t* perm, cudaStream_t st) {
   const size_t budget = 200 * 1024;
-  int nwarps = (int)(budget / ((size_t)D.nb * sizeof(uint32_t)));
+  const size_t hist = (size_t)D.nb * sizeof(uint32_t);
+  const size_t rows = (size_t)D.R * D.B * D.H;
+  // two CTAs per row (a cluster) when the rows alone would leave most SMs
+  // idle; the pair exchanges per-bucket totals, one more histogram of memory
+  const int P = (rows * 2 <= (size_t)num_sms() && D.L >= 4096 && 2 * hist <= budget) ? 2 : 1;
+  int nwarps = (int)((budget - (P > 1 ? hist : 0)) / hist);
   nwarps = nwarps > 32 ? 32 : nwarps;
-  const int by_len = (D.L + 127) / 128;  // at least 4 steps of 32 per warp
+  const int by_len = (D.L / P + 127) / 128;  // at least 4 steps of 32 per warp
   nwarps = nwarps > by_len ? by_len : nwarps;
   if (nwarps < 1) nwarps = 1;
-  const size_t smem = (size_t)nwarps * D.nb * sizeof(uint32_t);
+  const size_t smem = (size_t)(nwarps + (P > 1 ? 1 : 0)) * hist;
   lsh_status st0 = allow_smem(lsh::sort_rows_kernel, smem);
   if (st0 != LSH_OK) return st0;
-  const unsigned rows = (unsigned)((size_t)D.R * D.B * D.H);
-  lsh::sort_rows_kernel<<<rows, nwarps * 32, smem, st>>>(keys, perm, D.L, D.nb);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * P));
+  cfg.blockDim = dim3((unsigned)(nwarps * 32));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lsh::sort_rows_kernel, keys, perm, D.L, D.nb) != cudaSuccess)
+    return LSH_ERR_CUDA;
   return last_launch();
 }
 

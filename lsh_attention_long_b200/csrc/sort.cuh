@@ -5,17 +5,22 @@
 // order is (bucket, position); since a row's keys arrive in position order,
 // a stable counting sort on the bucket produces it.
 //
-// One CTA per row.  Each warp owns a contiguous segment of the row and a
+// A row is sorted by one thread-block cluster of P CTAs (P = 1 or 2), CTA c
+// taking the c-th part of the row.  Each warp owns a contiguous segment and a
 // private histogram in shared memory, so counting needs no atomics:
 //   pass 1  per 32-token step, __match_any_sync groups equal buckets and the
 //           group leader adds the group size to the warp's histogram;
-//   scan    bucket-major, warp-minor exclusive prefix sums turn the
-//           histograms into each warp's first output slot per bucket;
+//   scan    per-bucket totals of every CTA of the cluster meet through
+//           distributed shared memory; bucket-major, CTA-minor, warp-minor
+//           exclusive prefix sums give each warp's first output slot per
+//           bucket;
 //   pass 2  the same walk again; a token's slot is its warp's offset for the
 //           bucket plus its rank among equal-bucket lanes of lower index.
-// Warps, steps and lanes visit positions in increasing order, so equal
+// CTAs, warps, steps and lanes visit positions in increasing order, so equal
 // buckets keep position order: the sort is stable.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 
@@ -36,18 +41,26 @@ __device__ __forceinline__ uint32_t checked_bucket(const uint32_t* k, int t, int
 
 __global__ void __launch_bounds__(1024)
 sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, int L, int nb) {
-  extern __shared__ uint32_t cnt[];  // [nwarps][nb]
+  namespace cg = cooperative_groups;
+  extern __shared__ uint32_t cnt[];  // [nwarps][nb], then (P > 1) this CTA's totals [nb]
   __shared__ uint32_t warp_sums[32];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int P = (int)cluster.num_blocks(), crank = (int)cluster.block_rank();
   const int nwarps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t* k = keys + (size_t)blockIdx.x * L;
-  int32_t* out = perm + (size_t)blockIdx.x * L;
+  const size_t row = blockIdx.x / P;
+  const uint32_t* k = keys + row * L;
+  int32_t* out = perm + row * L;
+  uint32_t* tot = cnt + (size_t)nwarps * nb;
 
   for (int e = threadIdx.x; e < nwarps * nb; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
 
-  const int seg = (((L + nwarps - 1) / nwarps) + 31) & ~31;
-  const int begin = min(L, w * seg), end = min(L, begin + seg);
+  // this CTA's part of the row, then this warp's segment of it
+  const int part = (((L + P - 1) / P) + 31) & ~31;
+  const int cbeg = min(L, crank * part), cend = min(L, cbeg + part);
+  const int seg = ((((cend - cbeg) + nwarps - 1) / nwarps) + 31) & ~31;
+  const int begin = min(cend, cbeg + w * seg), end = min(cend, begin + seg);
   uint32_t* my = cnt + (size_t)w * nb;
   bool bad = false;
 
@@ -61,12 +74,32 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   if (bad) record_status(kErrBadKeys);
   __syncthreads();
 
-  // scan: each thread owns a contiguous run of buckets
+  // this CTA's totals per bucket, visible to the cluster (a lone CTA sums
+  // its histograms in place)
+  if (P > 1)
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      uint32_t s0 = 0;
+      for (int ww = 0; ww < nwarps; ++ww) s0 += cnt[ww * nb + b];
+      tot[b] = s0;
+    }
+  cluster.sync();
+  auto total = [&](int c, int b) -> uint32_t {  // CTA c's tokens of bucket b
+    if (P == 1) {
+      uint32_t s0 = 0;
+      for (int ww = 0; ww < nwarps; ++ww) s0 += cnt[ww * nb + b];
+      return s0;
+    }
+    return cluster.map_shared_rank(tot, c)[b];
+  };
+
+  // scan: each thread owns a contiguous run of buckets; a bucket's slots
+  // start after every smaller bucket of the row, then after the earlier
+  // CTAs' tokens of the same bucket
   const int per = (nb + blockDim.x - 1) / blockDim.x;
   const int b0 = min(nb, threadIdx.x * per), b1 = min(nb, b0 + per);
   uint32_t local = 0;
   for (int b = b0; b < b1; ++b)
-    for (int ww = 0; ww < nwarps; ++ww) local += cnt[ww * nb + b];
+    for (int c = 0; c < P; ++c) local += total(c, b);
   uint32_t incl = local;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -86,13 +119,22 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   }
   __syncthreads();
   uint32_t running = incl - local + (w > 0 ? warp_sums[w - 1] : 0);
-  for (int b = b0; b < b1; ++b)
+  for (int b = b0; b < b1; ++b) {
+    uint32_t all = 0, before = 0;
+    for (int c = 0; c < P; ++c) {
+      const uint32_t x = total(c, b);
+      all += x;
+      if (c < crank) before += x;
+    }
+    uint32_t r = running + before;
     for (int ww = 0; ww < nwarps; ++ww) {
       const uint32_t c = cnt[ww * nb + b];
-      cnt[ww * nb + b] = running;
-      running += c;
+      cnt[ww * nb + b] = r;
+      r += c;
     }
-  __syncthreads();
+    running += all;
+  }
+  cluster.sync();  // every CTA has read the others' totals
 
   // pass 2: stable scatter of positions
   for (int base = begin; base < end; base += 32) {
