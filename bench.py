@@ -53,6 +53,9 @@ def parse_args():
     p.add_argument("--workload", default=HEADLINE)
     p.add_argument("--no-extras", action="store_true",
                    help="headline only: skip fwd+bwd, e2e and the CPU baseline")
+    p.add_argument("--fwd-bwd", action="store_true",
+                   help="only the forward + backward measurement of --workload (a "
+                        "diagnostic line, not the headline)")
     p.add_argument("--ref-seconds", type=float, default=150.0,
                    help="--impl reference: CPU seconds of oracle sampling over all steps")
     return p.parse_args()
@@ -380,7 +383,7 @@ def run_fwd_bwd(args, w, world):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    steps = max(3, args.steps // 4)
+    steps = max(1, args.steps) if args.fwd_bwd else max(3, args.steps // 4)
 
     def step():
         e[0].record(stream)
@@ -542,6 +545,12 @@ def main():
     try:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA device for --impl ours")
+        if args.fwd_bwd:
+            res = {"workload": args.workload,
+                   "fwd_bwd": run_fwd_bwd(args, W.WORKLOADS[args.workload], world)}
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_ours(args, world, rank)
         if rank == 0 and not args.no_extras and world == 1:
             res["cpu_baseline"] = run_cpu_baseline(W.WORKLOADS[args.workload])
