@@ -416,8 +416,14 @@ def run_fwd_bwd(args, w, world):
 
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-# for the kernel as it stands, keyed by (stage, workload); None until taken.
-TRAFFIC = {}
+# for the kernel as it stands, keyed by (stage, workload); absent until taken.
+# From one ncu capture of the timed step of `bench.py --steps 1 --warmup 1
+# --no-extras`; to be cleared whenever the kernel changes.
+TRAFFIC = {
+    ("attend", "fwd_bf16_L65536"): 1084709000 + 989513472,
+    ("hash", "fwd_bf16_L65536"): 67665000 + 4091648,
+    ("sort", "fwd_bf16_L65536"): 19975000 + 3175936,
+}
 
 
 # ---------------------------------------------------------------------------
