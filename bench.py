@@ -56,6 +56,9 @@ def parse_args():
     p.add_argument("--fwd-bwd", action="store_true",
                    help="only the forward + backward measurement of --workload (a "
                         "diagnostic line, not the headline)")
+    p.add_argument("--recall", action="store_true",
+                   help="recall of LSH attention against full attention on the clustered "
+                        "L=16384 workload, over rounds and bucket counts (a report)")
     p.add_argument("--ref-seconds", type=float, default=150.0,
                    help="--impl reference: CPU seconds of oracle sampling over all steps")
     return p.parse_args()
@@ -415,6 +418,106 @@ def run_fwd_bwd(args, w, world):
                        "n_rounds": w.n_rounds, "chunk": w.chunk, "causal": w.causal}}
 
 
+# ---------------------------------------------------------------------------
+# recall against full attention (a report; the pages give no number for it)
+# ---------------------------------------------------------------------------
+
+def attended_mask(keys, perm, L: int, chunk: int, causal: bool, rows, b: int, h: int):
+    """[len(rows), L] bool: the keys that query positions `rows` of (b, h)
+    attend to in any round.  Per round the window is the query's chunk of the
+    sorted row and the previous chunk (chunk 0 wraps to the last; a single
+    chunk is its own window once); a key counts when it is in the query's
+    bucket, is not the query itself and, if causal, is at an earlier
+    position.  keys, perm: [R, B, H, L] (packed keys bucket * L + position)."""
+    R = keys.shape[0]
+    dev = keys.device
+    nch = L // chunk
+    S = rows.numel()
+    mask = torch.zeros((S, L), dtype=torch.bool, device=dev)
+    offs = torch.arange(chunk, device=dev)
+    for r in range(R):
+        k_r = keys[r, b, h].to(torch.int64) & 0xFFFFFFFF  # original order
+        p_r = perm[r, b, h].to(torch.int64)               # sorted slot -> position
+        inv = torch.empty_like(p_r)
+        inv[p_r] = torch.arange(L, device=dev)
+        ck = inv[rows] // chunk
+        if nch > 1:
+            prev = (ck - 1) % nch
+            win = torch.cat([prev[:, None] * chunk + offs, ck[:, None] * chunk + offs], 1)
+        else:
+            win = ck[:, None] * chunk + offs
+        tok = p_r[win]
+        ok = (k_r[tok] // L == (k_r[rows] // L)[:, None]) & (tok != rows[:, None])
+        if causal:
+            ok &= tok < rows[:, None]
+        qi = torch.arange(S, device=dev)[:, None].expand_as(tok)
+        mask[qi[ok], tok[ok]] = True
+    return mask
+
+
+def full_attention_recall(Q, keys, perm, chunk: int, causal: bool, rows, b: int, h: int):
+    """Per query: the share of full shared-QK attention's probability mass
+    (softmax of q_i . khat_j / sqrt(d) over every other key, earlier ones if
+    causal) that falls on keys LSH attention sees in some round.  fp64.
+    Queries with no key at all (the first position, causal) are dropped."""
+    q = Q[b, h].to(torch.float64)
+    L, d = q.shape
+    n = q.norm(dim=1, keepdim=True)
+    khat = torch.where(n > 0, q / torch.where(n > 0, n, torch.ones_like(n)), torch.zeros_like(q))
+    s = (q[rows] @ khat.T) / math.sqrt(d)
+    cols = torch.arange(L, device=q.device)[None, :]
+    allowed = cols != rows[:, None]
+    if causal:
+        allowed &= cols < rows[:, None]
+    s = s.masked_fill(~allowed, float("-inf"))
+    keep = allowed.any(1)
+    p = torch.softmax(s[keep], dim=1)
+    seen = attended_mask(keys, perm, L, chunk, causal, rows, b, h)[keep]
+    return (p * seen).sum(1)
+
+
+def run_recall(args):
+    """Recall against full attention over rounds (R = 1, 2, 4, 8 at nb = 256)
+    and bucket counts (nb = 64, 256, 1024 at R = 4) on the clustered
+    L = 16384 workload, with the forward's time for each setting."""
+    import lsh_attention_long_b200 as L
+    L.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    base = W.WORKLOADS["fwd_bf16_L16384_clustered"]
+    inp = W.make_inputs(base)
+    Q, V = inp["Q"].to(dev), inp["V"].to(dev)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(7)
+    rows = torch.randperm(base.L, generator=g)[:4096].sort().values.to(dev)
+    out = []
+    for R, nb in [(1, 256), (2, 256), (4, 256), (8, 256), (4, 64), (4, 1024)]:
+        rot = W.gaussian((R, base.d, nb // 2), 1, Q.dtype).to(dev)
+        res = L.lsh_forward(Q, V, rot, nb, base.chunk, base.causal)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for _ in range(3):
+            L.lsh_forward(Q, V, rot, nb, base.chunk, base.causal, out=res)
+        ev[0].record()
+        for _ in range(10):
+            L.lsh_forward(Q, V, rot, nb, base.chunk, base.causal, out=res)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / 10
+        rec = torch.cat([full_attention_recall(Q, res["keys"], res["perm"], base.chunk,
+                                               base.causal, rows, b, 0) for b in range(base.B)])
+        out.append({"n_rounds": R, "n_buckets": nb, "chunk": base.chunk,
+                    "recall_mean": round(float(rec.mean()), 4),
+                    "recall_p10": round(float(rec.quantile(0.1)), 4),
+                    "fwd_ms": round(ms, 4),
+                    "tokens_per_s": round(base.B * base.L / (ms / 1e3), 1)})
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error in the recall sweep")
+    return {"report": "recall vs full attention", "workload": base.name,
+            "sample": "4096 query positions (seed 7) of head 0 in each batch element; fp64 "
+                      "full attention over every other key",
+            "sweep": out}
+
+
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the kernel as it stands, keyed by (stage, workload); absent until taken.
 # From one ncu capture of the timed step of `bench.py --steps 1 --warmup 1
@@ -551,6 +654,10 @@ def main():
     try:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py needs a CUDA device for --impl ours")
+        if args.recall:
+            if rank == 0:
+                print(json.dumps(run_recall(args)), flush=True)
+            return
         if args.fwd_bwd:
             res = {"workload": args.workload,
                    "fwd_bwd": run_fwd_bwd(args, W.WORKLOADS[args.workload], world)}

@@ -213,6 +213,15 @@ def test_backward_workload_L16384(oracle):
     check_bwd(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal, heads=(1, 2))
 
 
+def test_backward_L65536_one_head(oracle):
+    """The backward at the headline size (8 rounds, 1024 buckets), one head
+    against the oracle."""
+    w = W.WORKLOADS["fwd_bf16_L65536"]
+    inp = W.make_inputs(w)
+    inp["dO"] = W.gaussian(tuple(inp["Q"].shape), 2, inp["Q"].dtype)
+    check_bwd(oracle, inp, w.n_buckets, w.chunk, w.causal, heads=(0, 5))
+
+
 # ---------------------------------------------------------------------------
 # edge cases of the ABI on the device
 # ---------------------------------------------------------------------------

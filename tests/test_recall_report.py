@@ -1,0 +1,80 @@
+"""The recall report's window enumeration and recall figure (CPU).
+
+`bench.py --recall` measures how much of full shared-QK attention's
+probability mass LSH attention can see ("Reformer explainer",
+akshathtiwari.co.in/blog/reformer: more hash rounds raise the chance that
+similar tokens share a bucket).  The pages print no recall value, so the
+report is unpinned as a number; these tests pin the computation itself:
+a single bucket and a single chunk must see everything (recall 1), and the
+attended sets must equal a brute-force enumeration over the oracle's keys
+and sort.
+"""
+
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _keys_perm(oracle, Q, nb, R, seed):
+    rng = np.random.default_rng(seed)
+    rot = rng.standard_normal((R, Q.shape[-1], max(nb // 2, 1)))
+    keys, _, _ = oracle.lsh_hash(Q, rot, nb)
+    perm = oracle.lsh_sort(keys)
+    return (torch.from_numpy(keys.astype(np.int64)), torch.from_numpy(perm.astype(np.int64)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_one_bucket_one_chunk_sees_everything(oracle, causal):
+    rng = np.random.default_rng(0)
+    L = 96
+    Q = rng.standard_normal((1, 1, L, 64))
+    keys, perm = _keys_perm(oracle, Q, 1, 2, 1)
+    rows = torch.arange(L)
+    rec = bench.full_attention_recall(torch.from_numpy(Q), keys, perm, L, causal, rows, 0, 0)
+    np.testing.assert_allclose(rec.numpy(), 1.0, rtol=0, atol=1e-12)
+    assert rec.numel() == (L - 1 if causal else L)  # causal: position 0 has no key
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("L,chunk,nb,R", [(256, 32, 8, 2), (128, 64, 4, 3), (64, 64, 4, 1)])
+def test_attended_sets_match_brute_force(oracle, causal, L, chunk, nb, R):
+    rng = np.random.default_rng(L + nb)
+    Q = rng.standard_normal((1, 2, L, 64))
+    keys, perm = _keys_perm(oracle, Q, nb, R, L)
+    rows = torch.arange(0, L, 3)
+    h = 1
+    got = bench.attended_mask(keys, perm, L, chunk, causal, rows, 0, h).numpy()
+    nch = L // chunk
+    want = np.zeros_like(got)
+    for qi, i in enumerate(rows.tolist()):
+        for r in range(R):
+            k = keys[r, 0, h].numpy() & 0xFFFFFFFF
+            p = perm[r, 0, h].numpy()
+            slot = int(np.nonzero(p == i)[0][0])
+            c = slot // chunk
+            chunks = [c] if nch == 1 else [(c - 1) % nch, c]
+            for cc in chunks:
+                for j in p[cc * chunk:(cc + 1) * chunk]:
+                    if j == i or k[j] // L != k[i] // L or (causal and j > i):
+                        continue
+                    want[qi, j] = True
+    assert np.array_equal(got, want)
+
+
+def test_recall_is_a_share_of_the_mass(oracle):
+    rng = np.random.default_rng(5)
+    L = 256
+    Q = rng.standard_normal((1, 1, L, 64))
+    keys, perm = _keys_perm(oracle, Q, 16, 2, 9)
+    rec = bench.full_attention_recall(torch.from_numpy(Q), keys, perm, 32, False,
+                                      torch.arange(L), 0, 0).numpy()
+    assert np.all(rec >= 0.0) and np.all(rec <= 1.0 + 1e-12)
+    assert 0.0 < rec.mean() < 1.0
