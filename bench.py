@@ -491,7 +491,7 @@ def run_recall(args):
     rows = torch.randperm(base.L, generator=g)[:4096].sort().values.to(dev)
     out = []
     for R, nb in [(1, 256), (2, 256), (4, 256), (8, 256), (4, 64), (4, 1024)]:
-        rot = W.gaussian((R, base.d, nb // 2), 1, Q.dtype).to(dev)
+        rot = W.rotations(R, base.d, nb, 1, Q.dtype).to(dev)
         res = L.lsh_forward(Q, V, rot, nb, base.chunk, base.causal)
         torch.cuda.synchronize()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
