@@ -69,6 +69,35 @@ def test_attended_sets_match_brute_force(oracle, causal, L, chunk, nb, R):
     assert np.array_equal(got, want)
 
 
+def test_topk_recall_one_bucket_one_chunk_is_one(oracle):
+    rng = np.random.default_rng(3)
+    L = 128
+    Q = rng.standard_normal((1, 1, L, 64))
+    keys, perm = _keys_perm(oracle, Q, 1, 1, 2)
+    rec = bench.full_attention_recall(torch.from_numpy(Q), keys, perm, L, False,
+                                      torch.arange(L), 0, 0, topk=16)
+    np.testing.assert_allclose(rec.numpy(), 1.0, rtol=0, atol=0)
+
+
+def test_topk_recall_counts_the_top_keys(oracle):
+    # top-k recall equals the share of each query's k best keys in its
+    # attended set, computed here directly from the mask and the scores
+    rng = np.random.default_rng(4)
+    L, k = 256, 8
+    Q = rng.standard_normal((1, 1, L, 64))
+    keys, perm = _keys_perm(oracle, Q, 16, 2, 6)
+    rows = torch.arange(L)
+    got = bench.full_attention_recall(torch.from_numpy(Q), keys, perm, 32, False, rows, 0, 0,
+                                      topk=k).numpy()
+    mask = bench.attended_mask(keys, perm, L, 32, False, rows, 0, 0).numpy()
+    q = Q[0, 0]
+    khat = q / np.linalg.norm(q, axis=1, keepdims=True)
+    s = q @ khat.T
+    np.fill_diagonal(s, -np.inf)
+    want = np.array([mask[i, np.argsort(-s[i])[:k]].mean() for i in range(L)])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
 def test_recall_is_a_share_of_the_mass(oracle):
     rng = np.random.default_rng(5)
     L = 256
