@@ -136,6 +136,22 @@ LSH_API lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void
                        uint32_t* keys, int32_t* buckets, int32_t* perm, void* O, float* lse,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* Whole forward from host memory: Q, V [B,H,L,d] and rot [R,d,n_buckets/2]
+ * (dtype) are host buffers; O [B,H,L,d] (dtype) and lse [B,H,L] fp32 (or
+ * NULL) are written to host buffers.  Page-locked host buffers let the
+ * copies run asynchronously: the heads are processed in groups, and the
+ * host-to-device copy of one group, the kernels of the next and the
+ * device-to-host copy of the one before overlap (two internal streams, made
+ * once per device; every step is ordered before the end of the work on
+ * `stream`, so synchronising `stream` covers the copies too).  Same
+ * arithmetic as lsh_forward, head by head.  ws is device scratch of at least
+ * lsh_forward_host_ws_size() bytes, owned by the caller; nothing is
+ * allocated.  Keys and permutations are not returned. */
+LSH_API size_t lsh_forward_host_ws_size(const lsh_shape* shape);
+LSH_API lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V,
+                            const void* rot, void* O, float* lse, void* ws, size_t ws_bytes,
+                            void* stream);
+
 /* Backward of steps 3-5 with buckets and permutations held constant.
  * Given the forward's O [B,H,L,d] and lse [B,H,L] and the upstream gradient
  * dO [B,H,L,d], writes dQ and dV [B,H,L,d] in dtype.  dQ includes the path

@@ -523,6 +523,153 @@ lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void* V, con
   return lsh_attend_fwd(shape, Q, V, keys, perm, nullptr, nullptr, O, lse, ws, ws_bytes, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Forward from host buffers, pipelined over groups of heads
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// Heads per group: at least three groups when there are heads enough, so
+// that copies in, kernels and copies out of neighbouring groups overlap.
+int host_group_heads(const Dims& D) {
+  const int BH = D.B * D.H;
+  const int groups = BH >= 4 ? 4 : BH;
+  return (BH + groups - 1) / groups;
+}
+
+// One group's device buffers: Q, V, O, lse, keys, perm, the forward workspace.
+struct HostGroupLayout {
+  size_t q, v, o, lse, keys, perm, ws, ws_bytes, total;
+};
+
+HostGroupLayout host_group_layout(const Dims& D, int G) {
+  Dims g = D;
+  g.B = 1;
+  g.H = G;
+  g.n_tok = (size_t)G * D.L;
+  const size_t elt = D.dtype == LSH_BF16 ? 2 : 4;
+  HostGroupLayout l;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off += align_up(bytes); return at; };
+  l.q = take(g.n_tok * D.d * elt);
+  l.v = take(g.n_tok * D.d * elt);
+  l.o = take(g.n_tok * D.d * elt);
+  l.lse = take(g.n_tok * sizeof(float));
+  l.keys = take((size_t)D.R * g.n_tok * sizeof(uint32_t));
+  l.perm = take((size_t)D.R * g.n_tok * sizeof(int32_t));
+  l.ws_bytes = fwd_ws_bytes(g);
+  l.ws = take(l.ws_bytes);
+  l.total = off;
+  return l;
+}
+
+size_t rot_bytes(const Dims& D) {
+  return D.nb > 1 ? (size_t)D.R * D.d * (D.nb / 2) * (D.dtype == LSH_BF16 ? 2 : 4) : 0;
+}
+
+// Two copy streams and the events of the pipeline, made once per device.
+struct HostPipe {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {}, rot_done = nullptr;
+  bool ready = false;
+};
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxDevices];
+
+HostPipe* host_pipe() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe& p = g_pipe[dev];
+  if (!p.ready) {
+    bool ok = cudaStreamCreateWithFlags(&p.up, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.down, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.rot_done, cudaEventDisableTiming) == cudaSuccess;
+    for (int b = 0; b < 2 && ok; ++b)
+      ok = cudaEventCreateWithFlags(&p.in_done[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.comp_done[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.out_done[b], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;
+    p.ready = true;
+  }
+  return &p;
+}
+
+}  // namespace
+
+size_t lsh_forward_host_ws_size(const lsh_shape* shape) {
+  Dims D;
+  if (check_shape(shape, &D) != LSH_OK || D.empty) return 0;
+  const HostGroupLayout l = host_group_layout(D, host_group_heads(D));
+  return align_up(rot_bytes(D)) + 2 * l.total;
+}
+
+lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V, const void* rot,
+                            void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  lsh_status s = check_shape(shape, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Q || !V || !O || (D.nb > 1 && !rot) || !ws) return LSH_ERR_INVALID_ARG;
+  if (misaligned(ws)) return LSH_ERR_INVALID_ARG;
+  const int G = host_group_heads(D);
+  const HostGroupLayout l = host_group_layout(D, G);
+  if (ws_bytes < align_up(rot_bytes(D)) + 2 * l.total) return LSH_ERR_WORKSPACE;
+  HostPipe* p = host_pipe();
+  if (!p) return LSH_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  void* rot_d = base;
+  char* buf[2] = {base + align_up(rot_bytes(D)), base + align_up(rot_bytes(D)) + l.total};
+  const size_t elt = D.dtype == LSH_BF16 ? 2 : 4;
+  const size_t head_elems = (size_t)D.L * D.d;
+  const int BH = D.B * D.H;
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // the copy streams start after the work already on `stream`
+  if (!ok(cudaEventRecord(p->rot_done, st)) || !ok(cudaStreamWaitEvent(p->up, p->rot_done, 0)))
+    return LSH_ERR_CUDA;
+  if (rot_bytes(D) &&
+      !ok(cudaMemcpyAsync(rot_d, rot, rot_bytes(D), cudaMemcpyHostToDevice, p->up)))
+    return LSH_ERR_CUDA;
+  const int n_groups = (BH + G - 1) / G;
+  for (int i = 0; i < n_groups; ++i) {
+    const int b = i & 1;
+    const int h0 = i * G, gh = BH - h0 < G ? BH - h0 : G;
+    char* d = buf[b];
+    // copies in: after the copies out of the group that used this buffer
+    if (i >= 2 && !ok(cudaStreamWaitEvent(p->up, p->out_done[b], 0))) return LSH_ERR_CUDA;
+    if (!ok(cudaMemcpyAsync(d + l.q, static_cast<const char*>(Q) + h0 * head_elems * elt,
+                            gh * head_elems * elt, cudaMemcpyHostToDevice, p->up)) ||
+        !ok(cudaMemcpyAsync(d + l.v, static_cast<const char*>(V) + h0 * head_elems * elt,
+                            gh * head_elems * elt, cudaMemcpyHostToDevice, p->up)) ||
+        !ok(cudaEventRecord(p->in_done[b], p->up)))
+      return LSH_ERR_CUDA;
+    // kernels on `stream`
+    if (!ok(cudaStreamWaitEvent(st, p->in_done[b], 0))) return LSH_ERR_CUDA;
+    lsh_shape gs = *shape;
+    gs.B = 1;
+    gs.H = gh;
+    s = lsh_forward(&gs, d + l.q, d + l.v, rot_d, reinterpret_cast<uint32_t*>(d + l.keys),
+                    nullptr, reinterpret_cast<int32_t*>(d + l.perm), d + l.o,
+                    reinterpret_cast<float*>(d + l.lse), d + l.ws, l.ws_bytes, st);
+    if (s != LSH_OK) return s;
+    if (!ok(cudaEventRecord(p->comp_done[b], st))) return LSH_ERR_CUDA;
+    // copies out
+    if (!ok(cudaStreamWaitEvent(p->down, p->comp_done[b], 0)) ||
+        !ok(cudaMemcpyAsync(static_cast<char*>(O) + h0 * head_elems * elt, d + l.o,
+                            gh * head_elems * elt, cudaMemcpyDeviceToHost, p->down)))
+      return LSH_ERR_CUDA;
+    if (lse && !ok(cudaMemcpyAsync(lse + (size_t)h0 * D.L, d + l.lse, gh * D.L * sizeof(float),
+                                   cudaMemcpyDeviceToHost, p->down)))
+      return LSH_ERR_CUDA;
+    if (!ok(cudaEventRecord(p->out_done[b], p->down))) return LSH_ERR_CUDA;
+  }
+  // the end of the work on `stream` waits for the last copies out
+  for (int b = 0; b < 2 && b < n_groups; ++b)
+    if (!ok(cudaStreamWaitEvent(st, p->out_done[b], 0))) return LSH_ERR_CUDA;
+  return LSH_OK;
+}
+
 lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const void* V, const void* O,
                           const void* dO, const uint32_t* keys, const int32_t* perm,
                           const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,

@@ -24,7 +24,8 @@ STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "L
           7: "LSH_ERR_SCRATCH_LIMIT"}
 
 EXPORTS = ("lsh_workspace_size", "lsh_hash", "lsh_sort", "lsh_attend_fwd", "lsh_combine",
-           "lsh_forward", "lsh_attend_bwd", "lsh_device_status", "lsh_status_string")
+           "lsh_forward", "lsh_forward_host", "lsh_forward_host_ws_size", "lsh_attend_bwd",
+           "lsh_device_status", "lsh_status_string")
 
 
 class LshError(RuntimeError):
@@ -59,6 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsh_attend_fwd": ([S, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "lsh_combine": ([S, P, P, P, P, P], ctypes.c_int),
         "lsh_forward": ([S, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
+        "lsh_forward_host_ws_size": ([S], sz),
+        "lsh_forward_host": ([S, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "lsh_attend_bwd": ([S, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "lsh_device_status": ([P], ctypes.c_int),
         "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -203,6 +206,33 @@ def lsh_forward(Q, V, rot, n_buckets: int, chunk: int, causal: bool, *, out=None
           _ptr(rot) if n_buckets > 1 else None, _ptr(o["keys"]), _ptr(o.get("buckets")),
           _ptr(o["perm"]), _ptr(o["O"]), _ptr(o["lse"]), _ptr(ws), ws.numel(), _stream(stream))
     return o
+
+
+def forward_host_workspace(shape: Shape, device) -> torch.Tensor:
+    """Device scratch for lsh_forward_host on this shape."""
+    n = load_library().lsh_forward_host_ws_size(ctypes.byref(shape))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def lsh_forward_host(Q, V, rot, n_buckets: int, chunk: int, causal: bool, *, O=None, lse=None,
+                     ws=None, device=None, stream=None):
+    """Whole forward from host tensors (page-locked for overlapped copies):
+    returns host O [B,H,L,d] and lse [B,H,L].  The library pipelines the
+    copies and kernels over groups of heads; the call returns once they are
+    queued on ``stream`` (synchronise it before reading O)."""
+    B, H, L, d = _qshape(Q)
+    R = rot.shape[0]
+    shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    if O is None:
+        O = torch.empty_like(Q, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, pin_memory=True)
+    if ws is None:
+        ws = forward_host_workspace(shape, device or torch.device("cuda", torch.cuda.current_device()))
+    _call("lsh_forward_host", ctypes.byref(shape), _ptr(Q), _ptr(V),
+          _ptr(rot) if n_buckets > 1 else None, _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+          _stream(stream))
+    return O, lse
 
 
 def lsh_attend_bwd(Q, V, O, dO, keys, perm, lse, n_buckets: int, chunk: int, causal: bool, *,

@@ -161,6 +161,23 @@ def test_workload_L65536_as_benchmarked(oracle):
     print(f"near ties in the 4096-token sample: {ties}")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,Lx,nb,R,causal", [(2, 3, 1024, 16, 2, True),
+                                                 (1, 1, 512, 8, 3, False),
+                                                 (1, 8, 4096, 64, 2, True)])
+def test_host_buffer_forward_equals_device_forward(dtype, B, H, Lx, nb, R, causal):
+    """lsh_forward_host (pinned host buffers, head groups pipelined through
+    the device) gives exactly lsh_forward's O and lse."""
+    inp = W.make_random(B, H, Lx, 64, nb, R, dtype, seed=Lx + H)
+    host = {k: inp[k].pin_memory() for k in ("Q", "V", "rot")}
+    ref = L.lsh_forward(*(host[k].cuda() for k in ("Q", "V", "rot")), nb, 64, causal)
+    O, lse = L.lsh_forward_host(host["Q"], host["V"], host["rot"], nb, 64, causal)
+    torch.cuda.synchronize()
+    _check_status()
+    assert torch.equal(O, ref["O"].cpu())
+    assert torch.equal(lse, ref["lse"].cpu())
+
+
 # ---------------------------------------------------------------------------
 # backward
 # ---------------------------------------------------------------------------

@@ -88,6 +88,24 @@ def test_null_and_misaligned_pointers_are_rejected(lib):
     assert lib.lsh_hash(None, fake, fake, fake, None, None) == 1
 
 
+def test_host_forward_checks_arguments_before_any_copy(lib):
+    s = _shape(B=1, H=4, L=1024, n_buckets=16, n_rounds=2)
+    host = ctypes.c_void_p(4096)  # never dereferenced: every call below fails its checks first
+    need = lib.lsh_forward_host_ws_size(ctypes.byref(s))
+    # two head groups in flight: at least twice one group's q, v, o and keys
+    assert need >= 2 * 2 * (1024 * 64 * 2 * 3 + 2 * 1024 * 8)
+    assert lib.lsh_forward_host(ctypes.byref(s), None, host, host, host, None, host, need,
+                                None) == 1
+    assert lib.lsh_forward_host(ctypes.byref(s), host, host, host, host, None, None, need,
+                                None) == 1
+    assert lib.lsh_forward_host(ctypes.byref(s), host, host, host, host, None,
+                                ctypes.c_void_p(4096), need - 1, None) == 4  # LSH_ERR_WORKSPACE
+    empty = _shape(B=0)
+    assert lib.lsh_forward_host(ctypes.byref(empty), None, None, None, None, None, None, 0,
+                                None) == 0
+    assert lib.lsh_forward_host_ws_size(ctypes.byref(empty)) == 0
+
+
 def test_empty_shapes_are_no_ops(lib):
     for kw in (dict(B=0), dict(H=0), dict(L=0)):
         s = _shape(**kw)
