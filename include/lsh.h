@@ -146,7 +146,11 @@ LSH_API lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void
  * `stream`, so synchronising `stream` covers the copies too).  Same
  * arithmetic as lsh_forward, head by head.  ws is device scratch of at least
  * lsh_forward_host_ws_size() bytes, owned by the caller; nothing is
- * allocated.  Keys and permutations are not returned. */
+ * allocated.  Keys and permutations are not returned.  The internal streams
+ * and events are shared by every call on a device: calls from several host
+ * threads take turns to enqueue their work (a per-device lock), and the
+ * copies of all calls on a device run in call order on those streams.  Calls
+ * that run at the same time need separate ws and output buffers. */
 LSH_API size_t lsh_forward_host_ws_size(const lsh_shape* shape);
 LSH_API lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V,
                             const void* rot, void* O, float* lse, void* ws, size_t ws_bytes,

@@ -572,6 +572,9 @@ struct HostPipe {
   cudaStream_t up = nullptr, down = nullptr;
   cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {}, rot_done = nullptr;
   bool ready = false;
+  // held while one call enqueues its copies, waits and kernels, so that the
+  // events of concurrent calls from several host threads do not interleave
+  std::mutex enqueue;
 };
 std::mutex g_pipe_mutex;
 HostPipe g_pipe[kMaxDevices];
@@ -617,6 +620,7 @@ lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V
   if (ws_bytes < align_up(rot_bytes(D)) + 2 * l.total) return LSH_ERR_WORKSPACE;
   HostPipe* p = host_pipe();
   if (!p) return LSH_ERR_CUDA;
+  std::lock_guard<std::mutex> hold(p->enqueue);
   cudaStream_t st = as_stream(stream);
   char* base = static_cast<char*>(ws);
   void* rot_d = base;
