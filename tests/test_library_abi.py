@@ -66,6 +66,8 @@ def test_status_strings(lib):
     (dict(d=32), 2), (dict(chunk=48), 1), (dict(n_buckets=3), 1), (dict(n_buckets=0), 1),
     (dict(n_rounds=0), 1), (dict(dtype=7), 1), (dict(chunk=128, L=256), 2),
     (dict(B=-1), 1), (dict(n_buckets=65536), 2), (dict(L=1 << 20, n_buckets=4096), 2),
+    (dict(B=1, H=4096, n_rounds=16), 2),                        # 65 536 rows > 65 535
+    (dict(B=1, H=512, L=65536, n_buckets=2, n_rounds=64), 2),   # B*H*L*R = 2^31
 ])
 def test_invalid_shapes_are_rejected_before_launch(lib, kw, expect):
     s = _shape(**kw)
