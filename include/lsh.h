@@ -139,11 +139,14 @@ LSH_API lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void
 /* Whole forward from host memory: Q, V [B,H,L,d] and rot [R,d,n_buckets/2]
  * (dtype) are host buffers; O [B,H,L,d] (dtype) and lse [B,H,L] fp32 (or
  * NULL) are written to host buffers.  Page-locked host buffers let the
- * copies run asynchronously: the heads are processed in groups, and the
- * host-to-device copy of one group, the kernels of the next and the
- * device-to-host copy of the one before overlap (two internal streams, made
- * once per device; every step is ordered before the end of the work on
- * `stream`, so synchronising `stream` covers the copies too).  Same
+ * copies run asynchronously: the heads are processed in groups (the last
+ * group split in two), rotating through three device buffer sets, and the
+ * host-to-device copy of one group, the kernels of the one before and the
+ * device-to-host copy of the one before that overlap; a group's hashing and
+ * sorting start once its Q has arrived, while its V is still in flight (two
+ * internal streams, made once per device; every step is ordered before the
+ * end of the work on `stream`, so synchronising `stream` covers the copies
+ * too).  Same
  * arithmetic as lsh_forward, head by head.  ws is device scratch of at least
  * lsh_forward_host_ws_size() bytes, owned by the caller; nothing is
  * allocated.  Keys and permutations are not returned.  The internal streams

@@ -537,6 +537,21 @@ int host_group_heads(const Dims& D) {
   return (BH + groups - 1) / groups;
 }
 
+// Heads of the group that starts at head h0.  Groups hold G heads, except the
+// last G heads, which form two groups of half the size: what runs after the
+// last copy in (its kernels and its copy out) is then half as long.
+int host_group_size(int BH, int G, int h0) {
+  const int tail = BH < G ? BH : G;
+  const int tail_start = BH - tail;
+  if (h0 < tail_start) return (tail_start - h0) < G ? tail_start - h0 : G;
+  if (h0 == tail_start && tail >= 2) return (tail + 1) / 2;
+  return BH - h0;
+}
+
+// Device buffer sets the groups rotate through: with three, the copy in of
+// group i+1 never waits for the copy out of group i-1.
+constexpr int kHostBufs = 3;
+
 // One group's device buffers: Q, V, O, lse, keys, perm, the forward workspace.
 struct HostGroupLayout {
   size_t q, v, o, lse, keys, perm, ws, ws_bytes, total;
@@ -570,7 +585,8 @@ size_t rot_bytes(const Dims& D) {
 // Two copy streams and the events of the pipeline, made once per device.
 struct HostPipe {
   cudaStream_t up = nullptr, down = nullptr;
-  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {}, rot_done = nullptr;
+  cudaEvent_t q_done[kHostBufs] = {}, v_done[kHostBufs] = {}, comp_done[kHostBufs] = {},
+              out_done[kHostBufs] = {}, rot_done = nullptr;
   bool ready = false;
   // held while one call enqueues its copies, waits and kernels, so that the
   // events of concurrent calls from several host threads do not interleave
@@ -588,8 +604,9 @@ HostPipe* host_pipe() {
     bool ok = cudaStreamCreateWithFlags(&p.up, cudaStreamNonBlocking) == cudaSuccess &&
               cudaStreamCreateWithFlags(&p.down, cudaStreamNonBlocking) == cudaSuccess &&
               cudaEventCreateWithFlags(&p.rot_done, cudaEventDisableTiming) == cudaSuccess;
-    for (int b = 0; b < 2 && ok; ++b)
-      ok = cudaEventCreateWithFlags(&p.in_done[b], cudaEventDisableTiming) == cudaSuccess &&
+    for (int b = 0; b < kHostBufs && ok; ++b)
+      ok = cudaEventCreateWithFlags(&p.q_done[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.v_done[b], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&p.comp_done[b], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&p.out_done[b], cudaEventDisableTiming) == cudaSuccess;
     if (!ok) return nullptr;
@@ -604,7 +621,7 @@ size_t lsh_forward_host_ws_size(const lsh_shape* shape) {
   Dims D;
   if (check_shape(shape, &D) != LSH_OK || D.empty) return 0;
   const HostGroupLayout l = host_group_layout(D, host_group_heads(D));
-  return align_up(rot_bytes(D)) + 2 * l.total;
+  return align_up(rot_bytes(D)) + kHostBufs * l.total;
 }
 
 lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V, const void* rot,
@@ -617,14 +634,13 @@ lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V
   if (misaligned(ws)) return LSH_ERR_INVALID_ARG;
   const int G = host_group_heads(D);
   const HostGroupLayout l = host_group_layout(D, G);
-  if (ws_bytes < align_up(rot_bytes(D)) + 2 * l.total) return LSH_ERR_WORKSPACE;
+  if (ws_bytes < align_up(rot_bytes(D)) + kHostBufs * l.total) return LSH_ERR_WORKSPACE;
   HostPipe* p = host_pipe();
   if (!p) return LSH_ERR_CUDA;
   std::lock_guard<std::mutex> hold(p->enqueue);
   cudaStream_t st = as_stream(stream);
-  char* base = static_cast<char*>(ws);
-  void* rot_d = base;
-  char* buf[2] = {base + align_up(rot_bytes(D)), base + align_up(rot_bytes(D)) + l.total};
+  char* base = static_cast<char*>(ws) + align_up(rot_bytes(D));
+  void* rot_d = ws;
   const size_t elt = D.dtype == LSH_BF16 ? 2 : 4;
   const size_t head_elems = (size_t)D.L * D.d;
   const int BH = D.B * D.H;
@@ -635,41 +651,51 @@ lsh_status lsh_forward_host(const lsh_shape* shape, const void* Q, const void* V
   if (rot_bytes(D) &&
       !ok(cudaMemcpyAsync(rot_d, rot, rot_bytes(D), cudaMemcpyHostToDevice, p->up)))
     return LSH_ERR_CUDA;
-  const int n_groups = (BH + G - 1) / G;
-  for (int i = 0; i < n_groups; ++i) {
-    const int b = i & 1;
-    const int h0 = i * G, gh = BH - h0 < G ? BH - h0 : G;
-    char* d = buf[b];
-    // copies in: after the copies out of the group that used this buffer
-    if (i >= 2 && !ok(cudaStreamWaitEvent(p->up, p->out_done[b], 0))) return LSH_ERR_CUDA;
-    if (!ok(cudaMemcpyAsync(d + l.q, static_cast<const char*>(Q) + h0 * head_elems * elt,
-                            gh * head_elems * elt, cudaMemcpyHostToDevice, p->up)) ||
-        !ok(cudaMemcpyAsync(d + l.v, static_cast<const char*>(V) + h0 * head_elems * elt,
-                            gh * head_elems * elt, cudaMemcpyHostToDevice, p->up)) ||
-        !ok(cudaEventRecord(p->in_done[b], p->up)))
-      return LSH_ERR_CUDA;
-    // kernels on `stream`
-    if (!ok(cudaStreamWaitEvent(st, p->in_done[b], 0))) return LSH_ERR_CUDA;
+  int i = 0;
+  for (int h0 = 0; h0 < BH; ++i) {
+    const int b = i % kHostBufs;
+    const int gh = host_group_size(BH, G, h0);
+    char* d = base + (size_t)b * l.total;
     lsh_shape gs = *shape;
     gs.B = 1;
     gs.H = gh;
-    s = lsh_forward(&gs, d + l.q, d + l.v, rot_d, reinterpret_cast<uint32_t*>(d + l.keys),
-                    nullptr, reinterpret_cast<int32_t*>(d + l.perm), d + l.o,
-                    reinterpret_cast<float*>(d + l.lse), d + l.ws, l.ws_bytes, st);
+    const size_t bytes = gh * head_elems * elt;
+    // copies in, after the copy out of the group that last used this buffer
+    // set; q first, so that hashing and sorting overlap the copy of v
+    if (i >= kHostBufs && !ok(cudaStreamWaitEvent(p->up, p->out_done[b], 0)))
+      return LSH_ERR_CUDA;
+    if (!ok(cudaMemcpyAsync(d + l.q, static_cast<const char*>(Q) + h0 * head_elems * elt, bytes,
+                            cudaMemcpyHostToDevice, p->up)) ||
+        !ok(cudaEventRecord(p->q_done[b], p->up)) ||
+        !ok(cudaMemcpyAsync(d + l.v, static_cast<const char*>(V) + h0 * head_elems * elt, bytes,
+                            cudaMemcpyHostToDevice, p->up)) ||
+        !ok(cudaEventRecord(p->v_done[b], p->up)))
+      return LSH_ERR_CUDA;
+    // kernels on `stream`: the same calls as lsh_forward
+    uint32_t* keys = reinterpret_cast<uint32_t*>(d + l.keys);
+    int32_t* perm = reinterpret_cast<int32_t*>(d + l.perm);
+    if (!ok(cudaStreamWaitEvent(st, p->q_done[b], 0))) return LSH_ERR_CUDA;
+    s = lsh_hash(&gs, d + l.q, rot_d, keys, nullptr, st);
+    if (s == LSH_OK) s = lsh_sort(&gs, keys, perm, d + l.ws, l.ws_bytes, st);
+    if (s != LSH_OK) return s;
+    if (!ok(cudaStreamWaitEvent(st, p->v_done[b], 0))) return LSH_ERR_CUDA;
+    s = lsh_attend_fwd(&gs, d + l.q, d + l.v, keys, perm, nullptr, nullptr, d + l.o,
+                       reinterpret_cast<float*>(d + l.lse), d + l.ws, l.ws_bytes, st);
     if (s != LSH_OK) return s;
     if (!ok(cudaEventRecord(p->comp_done[b], st))) return LSH_ERR_CUDA;
     // copies out
     if (!ok(cudaStreamWaitEvent(p->down, p->comp_done[b], 0)) ||
-        !ok(cudaMemcpyAsync(static_cast<char*>(O) + h0 * head_elems * elt, d + l.o,
-                            gh * head_elems * elt, cudaMemcpyDeviceToHost, p->down)))
+        !ok(cudaMemcpyAsync(static_cast<char*>(O) + h0 * head_elems * elt, d + l.o, bytes,
+                            cudaMemcpyDeviceToHost, p->down)))
       return LSH_ERR_CUDA;
     if (lse && !ok(cudaMemcpyAsync(lse + (size_t)h0 * D.L, d + l.lse, gh * D.L * sizeof(float),
                                    cudaMemcpyDeviceToHost, p->down)))
       return LSH_ERR_CUDA;
     if (!ok(cudaEventRecord(p->out_done[b], p->down))) return LSH_ERR_CUDA;
+    h0 += gh;
   }
   // the end of the work on `stream` waits for the last copies out
-  for (int b = 0; b < 2 && b < n_groups; ++b)
+  for (int b = 0; b < kHostBufs && b < i; ++b)
     if (!ok(cudaStreamWaitEvent(st, p->out_done[b], 0))) return LSH_ERR_CUDA;
   return LSH_OK;
 }

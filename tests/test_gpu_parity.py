@@ -164,7 +164,8 @@ def test_workload_L65536_as_benchmarked(oracle):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,H,Lx,nb,R,causal", [(2, 3, 1024, 16, 2, True),
                                                  (1, 1, 512, 8, 3, False),
-                                                 (1, 8, 4096, 64, 2, True)])
+                                                 (1, 8, 4096, 64, 2, True),
+                                                 (1, 5, 2048, 32, 2, False)])
 def test_host_buffer_forward_equals_device_forward(dtype, B, H, Lx, nb, R, causal):
     """lsh_forward_host (pinned host buffers, head groups pipelined through
     the device) gives exactly lsh_forward's O and lse."""
@@ -302,6 +303,27 @@ def test_tensor_core_hash_exact_ties_take_lowest_index():
     # p_3 == -p_2: z_3 ties z_{half+2} and z_2 ties z_{half+3}; the lower index wins
     assert not np.isin(b, [half + 2, half + 3]).any()
     assert np.isin(b, [0, half, 2, 3]).any()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_zero_queries(oracle, dtype):
+    """Rows of Q that are exactly zero: bucket 0 (every entry of [p ; -p] is
+    zero, the first index wins), a zero unit key (scores 0 against them), and
+    no gradient through the normalisation of a zero row."""
+    inp = W.make_random(1, 2, 320, 64, 16, 2, dtype, seed=91, backward=True)
+    zero = [0, 5, 63, 64, 77, 200, 201, 319]
+    inp["Q"][0, 0, zero] = 0
+    inp["Q"][0, 1, 100:164] = 0          # a whole chunk's worth of zero rows
+    check_all(oracle, inp, 16, 64, True)
+    check_bwd(oracle, inp, 16, 64, True)
+    _, buckets = L.lsh_hash(inp["Q"].cuda(), inp["rot"].cuda(), 16)
+    assert (buckets[:, 0, 0, zero] == 0).all()
+
+
+def test_largest_row_count(oracle):
+    """n_rounds * B * H = 65 535 rows, the most the launch grid takes."""
+    inp = W.make_random(1, 4369, 64, 64, 4, 15, torch.bfloat16, seed=5)
+    check_all(oracle, inp, 4, 64, False, heads=(0, 4368))
 
 
 @pytest.mark.parametrize("causal", [True, False])
