@@ -311,6 +311,8 @@ def run_ours(args, world, rank):
                    "causal": w.causal, "l2": "flushed between timed steps (256 MB memset)",
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
         "roofline": roof, "stages": stages,
+        # the same rate counted in (batch, head, position, round) units
+        "head_token_rounds_per_s": round(value * H * R, 1),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
