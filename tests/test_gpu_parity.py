@@ -116,6 +116,9 @@ CASES = [
     (1, 1, 256, 1024, 1, 64, False),  # more buckets than tokens: lone tokens
     (1, 2, 64, 4, 1, 4, True),        # tiny chunks
     (1, 1, 512, 32768, 1, 64, True),  # the largest bucket count
+    (1, 2, 384, 8, 5, 64, True),      # five rounds: three fold into one running state, two into the other
+    (2, 1, 256, 4, 8, 64, False),     # eight rounds, non-causal
+    (1, 1, 256, 96, 2, 64, True),     # nb/2 = 48, not a power of two: CUDA-core hash
 ]
 
 
@@ -216,6 +219,8 @@ BWD_CASES = [
     (1, 2, 64, 4, 1, 4, True),
     (2, 2, 1024, 64, 3, 64, False),   # sixteen chunks, several tiles per row
     (1, 2, 1088, 32, 2, 64, True),    # seventeen chunks: last tile has one query chunk
+    (1, 1, 256, 1, 2, 64, False),     # one bucket, non-causal
+    (1, 2, 384, 8, 5, 64, True),      # five rounds
 ]
 
 
