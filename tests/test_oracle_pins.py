@@ -9,6 +9,7 @@ repeated rounds) and finite differences of the forward.
 """
 
 import math
+import os
 
 import numpy as np
 import pytest
@@ -98,6 +99,22 @@ def test_hash_exact_ties_take_the_lowest_index(oracle):
     _, b2, tie2 = oracle.lsh_hash(Q, rot2, 4)
     assert np.array_equal(b2[0, 0, 0], np.where(p0 >= 0, 0, 1))
     assert np.all(tie2 == 1)
+
+
+def test_hash_hand_worked_axis_sectors(oracle):
+    """The worked example in tests/golden/hash_axis_sectors.txt: with the
+    identity as rotation, each bucket is a signed coordinate axis, derived by
+    hand (including the lowest-index rule on exact ties)."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "hash_axis_sectors.txt")
+    rows = [line.split() for line in open(path) if line.strip() and not line.startswith("#")]
+    for d in sorted({int(r[0]) for r in rows}):
+        sel = [r for r in rows if int(r[0]) == d]
+        X = np.array([[float(v) for v in r[1:1 + d]] for r in sel])
+        want = np.array([int(r[1 + d]) for r in sel])
+        L = len(sel)
+        keys, buckets, _ = oracle.lsh_hash(X[None, None], np.eye(d)[None], 2 * d)
+        np.testing.assert_array_equal(buckets[0, 0, 0], want)
+        np.testing.assert_array_equal(keys[0, 0, 0], want * L + np.arange(L))
 
 
 def test_hash_one_bucket_ignores_rotation(oracle):
