@@ -267,6 +267,29 @@ def test_brute_force_bucket_mates(oracle, L, chunk, nb, R, causal):
     np.testing.assert_allclose(out["lse"], lse, rtol=1e-12, atol=1e-9)
 
 
+@pytest.mark.parametrize("chunk,causal", [(2, False), (2, True), (1, False), (1, True)])
+def test_hand_worked_bucket_pairs(oracle, chunk, causal):
+    """tests/golden/attention_pairs.txt: every query has at most one
+    bucket-mate in its window, so the output is that mate's value exactly,
+    or the token's own value with lse = -1e5 when causality masks the mate."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "attention_pairs.txt")
+    rows = [line.split() for line in open(path) if line.strip() and not line.startswith("#")]
+    L = len(rows)
+    Q = np.array([[float(r[1]), float(r[2])] for r in rows])[None, None]
+    V = np.array([[i, 10.0 + i] for i in range(L)])[None, None]
+    out = oracle.lsh_forward(Q, V, np.eye(2)[None], 4, chunk, causal)
+    for i, r in enumerate(rows):
+        mate = r[5] if chunk == 1 else (r[4] if causal else r[3])
+        if mate == "self":
+            np.testing.assert_array_equal(out["O"][0, 0, i], V[0, 0, i])
+            assert out["lse"][0, 0, i] == -1e5
+        else:
+            j = int(mate)
+            np.testing.assert_array_equal(out["O"][0, 0, i], V[0, 0, j])
+            s_ij = Q[0, 0, i] @ Q[0, 0, j] / (np.linalg.norm(Q[0, 0, j]) * math.sqrt(2))
+            assert abs(out["lse"][0, 0, i] - s_ij) < 1e-12
+
+
 def test_constant_values_give_constant_output(oracle):
     rng = _rng(9)
     Q = rng.standard_normal((1, 2, 64, 64))
