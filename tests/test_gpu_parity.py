@@ -325,6 +325,38 @@ def test_zero_queries(oracle, dtype):
     assert (buckets[:, 0, 0, zero] == 0).all()
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("chunk,causal", [(2, False), (2, True), (1, False)])
+def test_hand_worked_bucket_pairs_on_the_device(dtype, chunk, causal):
+    """The hand-worked example of tests/golden/attention_pairs.txt, padded
+    from d = 2 to d = 64 with zeros (the rotation's two columns are the first
+    two axes): each output is one named token's value (up to fp32 rounding)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "attention_pairs.txt")
+    rows = [line.split() for line in open(path) if line.strip() and not line.startswith("#")]
+    n = len(rows)
+    Q = torch.zeros(1, 1, n, 64)
+    Q[0, 0, :, 0] = torch.tensor([float(r[1]) for r in rows])
+    Q[0, 0, :, 1] = torch.tensor([float(r[2]) for r in rows])
+    V = torch.zeros(1, 1, n, 64)
+    V[0, 0, :, 0] = torch.arange(n, dtype=torch.float32)
+    V[0, 0, :, 1] = 10 + torch.arange(n, dtype=torch.float32)
+    rot = torch.zeros(1, 64, 2)
+    rot[0, 0, 0] = rot[0, 1, 1] = 1
+    Q, V, rot = (t.to(dtype).cuda() for t in (Q, V, rot))
+    out = L.lsh_forward(Q, V, rot, 4, chunk, causal)
+    torch.cuda.synchronize()
+    _check_status()
+    O, lse = out["O"].float().cpu(), out["lse"].cpu()
+    for i, r in enumerate(rows):
+        mate = r[5] if chunk == 1 else (r[4] if causal else r[3])
+        j = i if mate == "self" else int(mate)
+        # the mate's weight is p / p in fp32: equal to 1 up to rounding
+        assert torch.allclose(O[0, 0, i], V[0, 0, j].float().cpu(), rtol=0, atol=1e-5)
+        if mate == "self":
+            assert abs(lse[0, 0, i].item() + 1e5) < 0.05
+
+
 def test_largest_row_count(oracle):
     """n_rounds * B * H = 65 535 rows, the most the launch grid takes."""
     inp = W.make_random(1, 4369, 64, 64, 4, 15, torch.bfloat16, seed=5)
