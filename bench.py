@@ -598,6 +598,20 @@ class OracleSampler:
                 f"(B*H*L*R hashes, B*H*R rows, B*H*R*L/c chunks); single-threaded fp64")
 
 
+def host_cpu() -> dict:
+    """The host's CPU model name and logical core count, for the baseline lines."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 def run_cpu_baseline(w):
     """The oracle as it stands on one whole head (b=0, h=0) of the workload:
     hash, sort, attention and combine for all rounds, scaled by B*H."""
@@ -612,7 +626,7 @@ def run_cpu_baseline(w):
     sec = time.perf_counter() - t0
     full = sec * w.B * w.H
     return {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": 1,
-            "kind": "oracle",
+            "kind": "oracle", **host_cpu(),
             "sample": f"one head (b=0, h=0) of {w.name}, all {w.n_rounds} rounds, full "
                       f"L={w.L}: hash, sort, attention, combine in {sec:.1f} s single-threaded "
                       f"fp64; scaled by B*H={w.B * w.H} to the whole step"}
@@ -641,7 +655,7 @@ def run_cpu_baseline_threads(w):
         sec = time.perf_counter() - t0
     full = sec * BH / n
     return {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": n,
-            "kind": "oracle",
+            "kind": "oracle", **host_cpu(),
             "sample": f"{n} of the {BH} heads of {w.name}, one per thread, all {w.n_rounds} "
                       f"rounds, full L={w.L}: hash, sort, attention, combine in {sec:.1f} s "
                       f"fp64; scaled by {BH}/{n} to the whole step"}
@@ -677,7 +691,7 @@ def run_reference(args, world, rank):
                    "n_buckets": w.n_buckets, "n_rounds": w.n_rounds, "chunk": w.chunk,
                    "causal": w.causal},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, **host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -37,5 +37,6 @@ def test_baseline_records():
     many = bench.run_cpu_baseline_threads(w)
     for r in (one, many):
         assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+        assert r["nproc"] >= r["cores"] and r["cpu_model"]
     assert one["cores"] == 1
     assert 1 <= many["cores"] <= w.B * w.H
