@@ -107,9 +107,47 @@ def _call(name: str, *args):
 
 
 def _qshape(Q: torch.Tensor):
-    if Q.dim() != 4:
-        raise ValueError("Q must be [B, H, L, d]")
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a [B, H, L, d] tensor")
     return tuple(Q.shape)
+
+
+def _validate(specs, device=None):
+    """Checks (name, tensor, shape, dtype, on_device) entries before any call:
+    the library takes plain pointers, so a wrong size, type or memory space
+    would otherwise reach the kernels.  Shapes and types are checked for every
+    entry first, then where each tensor lives (CUDA tensors on one device;
+    host tensors for the host-buffer forward).  None tensors are skipped."""
+    for name, t, shape, dtype, _ in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for name, t, _, _, on_device in specs:
+        if t is None:
+            continue
+        if on_device and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not on_device and t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+        if on_device:
+            if device is None:
+                device = t.device
+            elif t.device != device:
+                raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _rot_spec(rot, R, d, n_buckets, dtype, on_device=True):
+    """The rotation is read only when n_buckets > 1: [R, d, n_buckets/2]."""
+    if n_buckets > 1:
+        return ("rot", rot, (R, d, n_buckets // 2), dtype, on_device)
+    return ("rot", None, None, None, on_device)
 
 
 def lsh_workspace_size(shape: Shape) -> int:
@@ -126,6 +164,10 @@ def lsh_hash(Q, rot, n_buckets: int, *, keys=None, buckets=None, want_buckets=Tr
     B, H, L, d = _qshape(Q)
     R = rot.shape[0]
     shape = make_shape(B, H, L, d, n_buckets, R, 1, False, Q.dtype)
+    rows = (R, B, H, L)
+    _validate([("Q", Q, None, None, True), _rot_spec(rot, R, d, n_buckets, Q.dtype),
+               ("keys", keys, rows, torch.int32, True),
+               ("buckets", buckets, rows, torch.int32, True)])
     if keys is None:
         keys = torch.empty((R, B, H, L), dtype=torch.int32, device=Q.device)
     if buckets is None and want_buckets:
@@ -137,8 +179,12 @@ def lsh_hash(Q, rot, n_buckets: int, *, keys=None, buckets=None, want_buckets=Tr
 
 def lsh_sort(keys, n_buckets: int, *, perm=None, stream=None):
     """Step 2: perm [R,B,H,L] i32 (original position at each sorted slot)."""
+    if not isinstance(keys, torch.Tensor) or keys.dim() != 4:
+        raise ValueError("keys must be a [R, B, H, L] tensor")
     R, B, H, L = keys.shape
     shape = make_shape(B, H, L, 64, n_buckets, R, 1, False, torch.float32)
+    _validate([("keys", keys, None, torch.int32, True),
+               ("perm", perm, (R, B, H, L), torch.int32, True)])
     if perm is None:
         perm = torch.empty_like(keys, dtype=torch.int32)
     _call("lsh_sort", ctypes.byref(shape), _ptr(keys), _ptr(perm), None, 0, _stream(stream))
@@ -152,6 +198,13 @@ def lsh_attend_fwd(Q, V, keys, perm, n_buckets: int, chunk: int, causal: bool, *
     B, H, L, d = _qshape(Q)
     R = keys.shape[0]
     shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    rows = (R, B, H, L)
+    _validate([("Q", Q, None, None, True), ("V", V, Q.shape, Q.dtype, True),
+               ("keys", keys, rows, torch.int32, True), ("perm", perm, rows, torch.int32, True),
+               ("o_part", o_part, rows + (d,), torch.float32, True),
+               ("lse_r", lse_r, rows, torch.float32, True),
+               ("O", O, Q.shape, Q.dtype, True), ("lse", lse, (B, H, L), torch.float32, True),
+               ("ws", ws, None, None, True)])
     if combine:
         if O is None:
             O = torch.empty_like(Q)
@@ -173,8 +226,13 @@ def lsh_attend_fwd(Q, V, keys, perm, n_buckets: int, chunk: int, causal: bool, *
 
 def lsh_combine(o_part, lse_r, dtype: torch.dtype, *, O=None, lse=None, stream=None):
     """Step 5 alone: O [B,H,L,d] in dtype and lse [B,H,L] fp32."""
+    if not isinstance(o_part, torch.Tensor) or o_part.dim() != 5:
+        raise ValueError("o_part must be a [R, B, H, L, d] tensor")
     R, B, H, L, d = o_part.shape
     shape = make_shape(B, H, L, d, 2, R, 1, False, dtype)
+    _validate([("o_part", o_part, None, torch.float32, True),
+               ("lse_r", lse_r, (R, B, H, L), torch.float32, True),
+               ("O", O, (B, H, L, d), dtype, True), ("lse", lse, (B, H, L), torch.float32, True)])
     if O is None:
         O = torch.empty((B, H, L, d), dtype=dtype, device=o_part.device)
     if lse is None:
@@ -193,6 +251,15 @@ def lsh_forward(Q, V, rot, n_buckets: int, chunk: int, causal: bool, *, out=None
     R = rot.shape[0]
     shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
     o = dict(out or {})
+    rows = (R, B, H, L)
+    _validate([("Q", Q, None, None, True), ("V", V, Q.shape, Q.dtype, True),
+               _rot_spec(rot, R, d, n_buckets, Q.dtype),
+               ("out['keys']", o.get("keys"), rows, torch.int32, True),
+               ("out['perm']", o.get("perm"), rows, torch.int32, True),
+               ("out['buckets']", o.get("buckets"), rows, torch.int32, True),
+               ("out['O']", o.get("O"), Q.shape, Q.dtype, True),
+               ("out['lse']", o.get("lse"), (B, H, L), torch.float32, True),
+               ("ws", ws, None, None, True)])
     dev = Q.device
     o.setdefault("keys", torch.empty((R, B, H, L), dtype=torch.int32, device=dev))
     o.setdefault("perm", torch.empty((R, B, H, L), dtype=torch.int32, device=dev))
@@ -223,6 +290,10 @@ def lsh_forward_host(Q, V, rot, n_buckets: int, chunk: int, causal: bool, *, O=N
     B, H, L, d = _qshape(Q)
     R = rot.shape[0]
     shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    _validate([("Q", Q, None, None, False), ("V", V, Q.shape, Q.dtype, False),
+               _rot_spec(rot, R, d, n_buckets, Q.dtype, on_device=False),
+               ("O", O, Q.shape, Q.dtype, False), ("lse", lse, (B, H, L), torch.float32, False),
+               ("ws", ws, None, None, True)])
     if O is None:
         O = torch.empty_like(Q, pin_memory=True)
     if lse is None:
@@ -241,6 +312,13 @@ def lsh_attend_bwd(Q, V, O, dO, keys, perm, lse, n_buckets: int, chunk: int, cau
     B, H, L, d = _qshape(Q)
     R = keys.shape[0]
     shape = make_shape(B, H, L, d, n_buckets, R, chunk, causal, Q.dtype)
+    rows = (R, B, H, L)
+    _validate([("Q", Q, None, None, True), ("V", V, Q.shape, Q.dtype, True),
+               ("O", O, Q.shape, Q.dtype, True), ("dO", dO, Q.shape, Q.dtype, True),
+               ("keys", keys, rows, torch.int32, True), ("perm", perm, rows, torch.int32, True),
+               ("lse", lse, (B, H, L), torch.float32, True),
+               ("dQ", dQ, Q.shape, Q.dtype, True), ("dV", dV, Q.shape, Q.dtype, True),
+               ("ws", ws, None, None, True)])
     if dQ is None:
         dQ = torch.empty_like(Q)
     if dV is None:
