@@ -109,7 +109,7 @@ LSH_API lsh_status lsh_hash(const lsh_shape* shape, const void* Q, const void* r
 LSH_API lsh_status lsh_sort(const lsh_shape* shape, const uint32_t* keys, int32_t* perm, void* ws,
                     size_t ws_bytes, void* stream);
 
-/* Steps 3-5 (gather -> chunk attention -> scatter, fused combine).
+/* Steps 3-5 (gather -> chunk attention -> scatter, with the combine).
  * Q, V: [B,H,L,d]; keys, perm: from lsh_hash / lsh_sort.
  * o_part: [R,B,H,L,d] fp32 or NULL; lse_r: [R,B,H,L] fp32 or NULL.
  * O: [B,H,L,d] in dtype, or NULL to skip the combine (then o_part and lse_r
@@ -179,17 +179,30 @@ LSH_API lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const v
  * a plugin inside another runtime's execution phase, or a latency-critical
  * loop where an allocation would synchronise the device.  This call takes
  * the same inputs and outputs as lsh_attend_fwd with O given (Q, V, keys,
- * perm -> O, lse) but no workspace: the per-round partials of rounds
- * 0..R-2 live in a scratch array of LSH_STATIC_SCRATCH_BYTES (64 MiB) that
- * the library defines at file scope in device memory.  Every GPU that loads
- * the library holds that array until the process exits.  It allocates
- * nothing itself: no cudaMalloc, no cudaFree, no allocating library call.
- *   - Capacity: (n_rounds - 1) * B * H * L * (d + 1) * 4 bytes must not
- *     exceed LSH_STATIC_SCRATCH_BYTES, else LSH_ERR_SCRATCH_LIMIT is
- *     returned before any launch.  One round (n_rounds == 1) needs none.
+ * perm -> O, lse) but no workspace: the attention's scratch lives in an
+ * array of LSH_STATIC_SCRATCH_BYTES (64 MiB) that the library defines at
+ * file scope in device memory.  Every GPU that loads the library holds that
+ * array until the process exits.  It allocates nothing itself: no
+ * cudaMalloc, no cudaFree, no allocating library call.
+ *   - Capacity.  With n = B * H * L tokens, and every part below rounded up
+ *     to a multiple of 256 bytes, the scratch a call needs is
+ *       tensor-core path (dtype LSH_BF16 and chunk == 64):
+ *         (n_rounds * B * H + 1) * 4   tile and ticket counters
+ *       + n * 4                        per-token key scales
+ *       + k * n * 256 + k * n * 16     running (output, max, sum) states,
+ *                                      k = 2 if n_rounds > 1, else 1;
+ *       so about 276 bytes per token for one round and 548 for more;
+ *       CUDA-core path (every other supported case):
+ *         (n_rounds - 1) * n * d * 4 + (n_rounds - 1) * n * 4
+ *                                      partials of rounds 0 .. n_rounds-2,
+ *       none for one round.
+ *     A call whose need exceeds LSH_STATIC_SCRATCH_BYTES returns
+ *     LSH_ERR_SCRATCH_LIMIT before any launch.
  *   - Set-up: the first call on a device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
- *     that first call outside any stream capture.
+ *     that first call outside any stream capture.  The cached address
+ *     belongs to the device's primary context as it was then: after
+ *     cudaDeviceReset the process must not call this entry point again.
  *   - Sharing: all calls in the process on a device use the same array and
  *     it keeps whatever the last call left there.  Every element a call reads
  *     is written earlier in the same call, so nothing needs clearing, but

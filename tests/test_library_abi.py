@@ -134,3 +134,42 @@ def test_missing_library_fails_loudly(tmp_path):
             mod.load_library(str(tmp_path / "absent.so"))
     finally:
         mod._lib = saved
+
+
+def _align(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("Lx,R,chunk,dtype,need", [
+    # tensor-core path (bf16, chunk 64), one round: counters, key scales, one
+    # running state of 256 + 16 B per token
+    (243136, 1, 64, 1, _align(8) + _align(243136 * 4) + _align(243136 * 272)),
+    (243200, 1, 64, 1, _align(8) + _align(243200 * 4) + _align(243200 * 272)),
+    # CUDA-core path (f32), two rounds: one round of fp32 partials (256 + 4 B)
+    (258048, 2, 64, 0, _align(258048 * 256) + _align(258048 * 4)),
+    (258112, 2, 64, 0, _align(258112 * 256) + _align(258112 * 4)),
+    # the same L=16384 x 8 heads, R=2 problem on each path: 71 MB on the
+    # tensor-core path, 34 MB on the CUDA-core path (chunk 32)
+    (8 * 16384, 2, 64, 1, _align(3 * 4) + _align(131072 * 4) + _align(2 * 131072 * 272)),
+    (8 * 16384, 2, 32, 1, _align(131072 * 256) + _align(131072 * 4)),
+])
+def test_static_scratch_limit_follows_the_path(lib, Lx, R, chunk, dtype, need):
+    """lsh_attend_fwd_static refuses exactly the problems whose need, on the
+    path they take, exceeds its 64 MiB array.  An accepted problem goes on to
+    look up the array, which fails on a machine without a GPU (LSH_ERR_CUDA),
+    so it is probed only there."""
+    P = ctypes.c_void_p
+    lib.lsh_attend_fwd_static.argtypes = [ctypes.POINTER(Shape), P, P, P, P, P, P, P]
+    lib.lsh_attend_fwd_static.restype = ctypes.c_int
+    s = _shape(B=1, H=1, L=Lx, n_buckets=2, n_rounds=R, chunk=chunk, dtype=dtype)
+    fake = ctypes.c_void_p(256)
+    limit = 64 << 20
+    if need > limit:
+        assert lib.lsh_attend_fwd_static(ctypes.byref(s), fake, fake, fake, fake, fake, None,
+                                         None) == 7
+        return
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("an accepted problem would launch on these placeholder pointers")
+    assert lib.lsh_attend_fwd_static(ctypes.byref(s), fake, fake, fake, fake, fake, None,
+                                     None) == 3

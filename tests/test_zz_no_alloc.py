@@ -4,16 +4,17 @@ Some callers cannot allocate device memory when they run attention: a host
 framework whose planner owns every buffer, a plugin executing inside another
 runtime, or a latency-critical loop where cudaMalloc would synchronise the
 device.  For them the library keeps its scratch in a built-in device array of
-fixed size; this test calls that entry point through the C ABI and checks it
-against lsh_attend_fwd with a caller-provided workspace, on two calls in a
-row (different inputs), plus the size limit.
+fixed size.  These tests call that entry point through the C ABI and check it
+against lsh_attend_fwd with a caller-provided workspace on two calls in a row
+that take the same kernel path (the second call finds the first one's state
+in the shared array), and check the size limit with the need of the path a
+case actually takes.
 
 The file is named so that pytest collects it last.
 """
 
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -24,6 +25,22 @@ from lsh_attention_long_b200.lsh import Shape
 pytestmark = pytest.mark.gpu
 
 STATIC_BYTES = 64 << 20
+
+
+def _align(x):
+    return (x + 255) // 256 * 256
+
+
+def static_need(B, H, Lx, R, chunk, dtype):
+    """Scratch bytes the header documents for lsh_attend_fwd_static."""
+    n = B * H * Lx
+    if dtype == torch.bfloat16 and chunk == 64:  # tensor-core path
+        k = 2 if R > 1 else 1
+        return (_align((R * B * H + 1) * 4) + _align(n * 4) + _align(k * n * 256)
+                + _align(k * n * 16))
+    if R == 1:  # CUDA-core path
+        return 0
+    return _align((R - 1) * n * 64 * 4) + _align((R - 1) * n * 4)
 
 
 @pytest.fixture(scope="module")
@@ -43,45 +60,55 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _run_static(lib, Q, V, keys, perm, nb, chunk, causal):
-    B, H, Lx, d = Q.shape
-    shape = L.make_shape(B, H, Lx, d, nb, keys.shape[0], chunk, causal, Q.dtype)
+def _call_static(lib, shape, Q, V, keys, perm, O, lse):
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.lsh_attend_fwd_static(ctypes.byref(shape), _p(Q), _p(V), _p(keys), _p(perm),
+                                     _p(O), _p(lse), stream)
+
+
+def _same_as_workspace_call(lib, B, H, Lx, nb, R, chunk, causal, dtype, seed):
+    """Runs both entry points on one problem; their O and lse must be equal
+    bit for bit (the same kernels, only the scratch differs)."""
+    assert static_need(B, H, Lx, R, chunk, dtype) <= STATIC_BYTES
+    inp = W.make_random(B, H, Lx, 64, nb, R, dtype, seed=seed)
+    Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
+    keys, _ = L.lsh_hash(Q, rot, nb, want_buckets=False)
+    perm = L.lsh_sort(keys, nb)
+    O_ref, lse_ref, _, _ = L.lsh_attend_fwd(Q, V, keys, perm, nb, chunk, causal)
+    shape = L.make_shape(B, H, Lx, 64, nb, R, chunk, causal, Q.dtype)
     O = torch.full_like(Q, float("nan"))
     lse = torch.full((B, H, Lx), float("nan"), dtype=torch.float32, device=Q.device)
-    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    rc = lib.lsh_attend_fwd_static(ctypes.byref(shape), _p(Q), _p(V), _p(keys), _p(perm), _p(O),
-                                   _p(lse), stream)
+    rc = _call_static(lib, shape, Q, V, keys, perm, O, lse)
     assert rc == 0, L.lsh.STATUS.get(rc, rc)
-    return O, lse
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
+    assert torch.equal(O, O_ref)
+    assert torch.equal(lse, lse_ref)
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_static_scratch_matches_workspace_entry_point(lib, dtype):
-    cases = [  # two calls in a row on different problems; the second reuses the array
-        (2, 4, 1024, 64, 4, 64, True, 11),
-        (1, 3, 320, 16, 3, 32, False, 12),
-    ]
-    tol = 2e-2 if dtype == torch.bfloat16 else 2e-3
-    for B, H, Lx, nb, R, chunk, causal, seed in cases:
-        inp = W.make_random(B, H, Lx, 64, nb, R, dtype, seed=seed)
-        Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
-        keys, _ = L.lsh_hash(Q, rot, nb, want_buckets=False)
-        perm = L.lsh_sort(keys, nb)
-        O_ref, lse_ref, _, _ = L.lsh_attend_fwd(Q, V, keys, perm, nb, chunk, causal)
-        O, lse = _run_static(lib, Q, V, keys, perm, nb, chunk, causal)
-        torch.cuda.synchronize()
-        assert L.lsh_device_status() == 0
-        np.testing.assert_allclose(O.float().cpu().numpy(), O_ref.float().cpu().numpy(),
-                                   rtol=0, atol=tol)
-        np.testing.assert_allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), rtol=1e-6, atol=tol)
+@pytest.mark.parametrize("dtype,chunk2", [(torch.bfloat16, 64), (torch.float32, 32)])
+def test_static_scratch_matches_workspace_entry_point(lib, dtype, chunk2):
+    """Two calls in a row on one path: a larger problem leaves its running
+    states (tensor-core path) or partials (CUDA-core path) in the shared
+    array, then a smaller one must not read any of them."""
+    _same_as_workspace_call(lib, 2, 4, 2048, 64, 4, 64, True, dtype, seed=11)
+    _same_as_workspace_call(lib, 1, 3, 320, 16, 3, chunk2, False, dtype, seed=12)
 
 
-def test_static_scratch_rejects_problems_beyond_its_size(lib):
-    # (R-1) * B*H*L * 65 floats: 1 * 8*8*4096 * 260 B = 68 MB > 64 MiB
-    B, H, Lx, R = 8, 8, 4096, 2
-    shape = L.make_shape(B, H, Lx, 64, 64, R, 64, True, torch.bfloat16)
+def test_static_scratch_capacity_follows_the_path(lib):
+    """B=1 H=8 L=16384 R=2: the tensor-core path (bf16, chunk 64) needs about
+    71 MB and is refused; the CUDA-core path (f32, or bf16 with chunk 32)
+    needs 34 MB and runs.  One round in bf16 needs 36 MB and runs; one round
+    at L=65536 needs 145 MB and is refused."""
     fake = ctypes.c_void_p(256)  # never dereferenced: the size check fails first
-    rc = lib.lsh_attend_fwd_static(ctypes.byref(shape), fake, fake, fake, fake, fake, None, None)
-    assert rc == 7
+    refused = [(1, 8, 16384, 2, 64, torch.bfloat16), (1, 8, 65536, 1, 64, torch.bfloat16)]
+    for B, H, Lx, R, chunk, dtype in refused:
+        assert static_need(B, H, Lx, R, chunk, dtype) > STATIC_BYTES
+        shape = L.make_shape(B, H, Lx, 64, 64, R, chunk, True, dtype)
+        rc = lib.lsh_attend_fwd_static(ctypes.byref(shape), fake, fake, fake, fake, fake, None,
+                                       None)
+        assert rc == 7
     assert lib.lsh_status_string(7).startswith(b"problem exceeds")
-    assert (R - 1) * B * H * Lx * 65 * 4 > STATIC_BYTES
+    _same_as_workspace_call(lib, 1, 8, 16384, 64, 2, 64, True, torch.float32, seed=21)
+    _same_as_workspace_call(lib, 1, 8, 16384, 64, 2, 32, True, torch.bfloat16, seed=22)
+    _same_as_workspace_call(lib, 1, 8, 16384, 64, 1, 64, True, torch.bfloat16, seed=23)
