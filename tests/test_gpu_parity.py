@@ -8,6 +8,9 @@ failure; near ties (top two rotated projections within 1e-5 relative) are
 counted and reported.
 """
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -18,6 +21,26 @@ from lsh_attention_long_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 TOL = {torch.float32: 2e-3, torch.bfloat16: 2e-2}
+# host threads for the oracle over independent (b, h) heads; its C routines
+# release the GIL
+WORKERS = max(1, min(16, os.cpu_count() or 1))
+
+
+def _pmap(fn, items):
+    with ThreadPoolExecutor(max_workers=WORKERS) as ex:
+        return list(ex.map(fn, items))
+
+
+def _heads(B, H):
+    return [(b, h) for b in range(B) for h in range(H)]
+
+
+def _err(got, ref, atol, rtol=0.0):
+    """(largest |got - ref|, whether every element is within atol + rtol |ref|)."""
+    if got.size == 0:
+        return 0.0, True
+    d = np.abs(got.astype(np.float64) - ref)
+    return float(d.max()), bool((d <= atol + rtol * np.abs(ref)).all())
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -58,6 +81,68 @@ def check_hash(oracle, Q, rot, nb, keys, buckets, sample=None):
     bad = (gb != ob) & (tie == 0)
     assert not bad.any(), f"{int(bad.sum())} bucket mismatches outside near ties"
     return int(tie.sum())
+
+
+def hash_every_token(oracle, Q, rot, nb, keys):
+    """Every token's bucket id in every round against the oracle, head by
+    head over host threads.  Returns the near-tie count and how many near
+    ties the GPU resolved the other way; any other mismatch fails."""
+    Qn, rotn = _np(Q), _np(rot)
+    B, H, Ln = Qn.shape[:3]
+    kk = keys.cpu().numpy().view(np.uint32)
+    gb = (kk // np.uint32(Ln)).astype(np.int64)
+    assert np.array_equal(kk % np.uint32(Ln),
+                          np.broadcast_to(np.arange(Ln, dtype=np.uint32), kk.shape))
+
+    def one(bh):
+        b, h = bh
+        _, ob, tie = oracle.lsh_hash(Qn[b:b + 1, h:h + 1], rotn, nb)
+        diff = gb[:, b:b + 1, h:h + 1] != ob
+        return int((diff & (tie == 0)).sum()), int(tie.sum()), int((diff & (tie != 0)).sum())
+
+    res = _pmap(one, _heads(B, H))
+    bad = sum(r[0] for r in res)
+    assert bad == 0, f"{bad} bucket mismatches outside near ties"
+    return sum(r[1] for r in res), sum(r[2] for r in res)
+
+
+def attention_every_head(oracle, Q, V, keys, perm, chunk, causal, O, lse, o_part=None,
+                         lse_r=None):
+    """O and lse (and, when given, the per-round o_part and lse_r) of every
+    (b, h) head against the oracle fed the GPU's keys and permutations, head
+    by head over host threads.  Returns the largest error of each output."""
+    tol = TOL[Q.dtype]
+    Qn, Vn = _np(Q), _np(V)
+    keys_np = keys.cpu().numpy().view(np.uint32)
+    perm_np = perm.cpu().numpy()
+    gO, glse = _np(O), _np(lse)
+    gop = None if o_part is None else _np(o_part)
+    glr = None if lse_r is None else _np(lse_r)
+
+    def one(bh):
+        b, h = bh
+        op, lr = oracle.lsh_attend_fwd(Qn[b:b + 1, h:h + 1], Vn[b:b + 1, h:h + 1],
+                                       keys_np[:, b:b + 1, h:h + 1],
+                                       perm_np[:, b:b + 1, h:h + 1], chunk, causal)
+        Oo, lo = oracle.lsh_combine(op, lr)
+        e = {"O": _err(gO[b, h], Oo[0, 0], tol), "lse": _err(glse[b, h], lo[0, 0], tol, 1e-6)}
+        if gop is not None:
+            e["o_part"] = _err(gop[:, b, h], op[:, 0, 0], tol)
+            e["lse_r"] = _err(glr[:, b, h], lr[:, 0, 0], tol, 1e-6)
+        return bh, e
+
+    return _collect(_pmap(one, _heads(*Qn.shape[:2])))
+
+
+def _collect(per_head):
+    """Largest error per output over heads; fails naming the first head out
+    of tolerance."""
+    worst = {}
+    for bh, e in per_head:
+        for k, (m, ok) in e.items():
+            assert ok, f"{k} of head {bh} differs from the oracle by {m}"
+            worst[k] = max(worst.get(k, 0.0), m)
+    return worst
 
 
 def run_steps(inp, nb, chunk, causal):
@@ -129,39 +214,54 @@ def test_small_shapes(oracle, dtype, B, H, Lx, nb, R, chunk, causal):
     check_all(oracle, inp, nb, chunk, causal)
 
 
-def test_workload_fwd_f32_L1024(oracle):
+def test_workload_fwd_f32_L1024(oracle, parity_record):
     w = W.WORKLOADS["fwd_f32_L1024"]
-    check_all(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal)
+    g = check_all(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal)
+    ties, flips = hash_every_token(oracle, g["Q"], g["rot"], w.n_buckets, g["keys"])
+    worst = attention_every_head(oracle, g["Q"], g["V"], g["keys"], g["perm"], w.chunk, w.causal,
+                                 g["O"], g["lse"], g["o_part"], g["lse_r"])
+    parity_record.append({"workload": w.name, "heads": 1, "tokens_hashed": w.L,
+                          "near_ties": ties, "near_tie_flips": flips, "rows_sorted": 1,
+                          "max_abs": worst, "tol": TOL[torch.float32]})
 
 
-@pytest.mark.parametrize("name,head", [("fwd_bf16_L4096", (5, 3)),
-                                       ("fwd_bf16_L16384_clustered", (1, 6))])
-def test_workload_bf16(oracle, name, head):
+@pytest.mark.parametrize("name", ["fwd_bf16_L4096", "fwd_bf16_L16384_clustered"])
+def test_workload_bf16_every_head(oracle, parity_record, name):
+    """Every step of the forward on every (b, h) head of the workload: bucket
+    ids of every token, permutations of every row, per-round partials and the
+    combined O and lse."""
     w = W.WORKLOADS[name]
-    check_all(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal, heads=head)
+    g = run_steps(W.make_inputs(w), w.n_buckets, w.chunk, w.causal)
+    ties, flips = hash_every_token(oracle, g["Q"], g["rot"], w.n_buckets, g["keys"])
+    keys_np = g["keys"].cpu().numpy().view(np.uint32)
+    assert np.array_equal(g["perm"].cpu().numpy(), oracle.lsh_sort(keys_np))
+    worst = attention_every_head(oracle, g["Q"], g["V"], g["keys"], g["perm"], w.chunk, w.causal,
+                                 g["O"], g["lse"], g["o_part"], g["lse_r"])
+    parity_record.append({"workload": name, "heads": w.B * w.H, "tokens_hashed": w.B * w.H * w.L,
+                          "near_ties": ties, "near_tie_flips": flips, "rows_sorted":
+                          w.n_rounds * w.B * w.H, "max_abs": worst, "tol": TOL[g["Q"].dtype]})
 
 
-def test_workload_L65536_as_benchmarked(oracle):
-    """The benchmarked forward (one lsh_forward call) at full size; hash on a
-    sample of tokens, sort on every row, attention on one sampled head."""
+def test_workload_L65536_as_benchmarked(oracle, parity_record):
+    """The benchmarked forward (one lsh_forward call, the online combine) at
+    full size: every token's bucket ids in all 8 rounds, every row's
+    permutation, O and lse of all 8 heads."""
     w = W.WORKLOADS["fwd_bf16_L65536"]
     inp = W.make_inputs(w)
     Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
     out = L.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal, want_buckets=True)
     torch.cuda.synchronize()
     _check_status()
-    ties = check_hash(oracle, Q, rot, w.n_buckets, out["keys"], out["buckets"], sample=4096)
+    assert torch.equal(out["keys"] // w.L, out["buckets"])
+    ties, flips = hash_every_token(oracle, Q, rot, w.n_buckets, out["keys"])
     keys_np = out["keys"].cpu().numpy().view(np.uint32)
     assert np.array_equal(out["perm"].cpu().numpy(), oracle.lsh_sort(keys_np))
-    h = 3
-    o_part, lse_r = oracle.lsh_attend_fwd(_np(Q)[:, h:h + 1], _np(V)[:, h:h + 1],
-                                          keys_np[:, :, h:h + 1],
-                                          out["perm"].cpu().numpy()[:, :, h:h + 1],
-                                          w.chunk, w.causal)
-    O, lse = oracle.lsh_combine(o_part, lse_r)
-    np.testing.assert_allclose(_np(out["O"])[:, h:h + 1], O, rtol=0, atol=2e-2)
-    np.testing.assert_allclose(_np(out["lse"])[:, h:h + 1], lse, rtol=1e-6, atol=2e-2)
-    print(f"near ties in the 4096-token sample: {ties}")
+    worst = attention_every_head(oracle, Q, V, out["keys"], out["perm"], w.chunk, w.causal,
+                                 out["O"], out["lse"])
+    parity_record.append({"workload": w.name, "heads": w.B * w.H,
+                          "tokens_hashed": w.B * w.H * w.L, "near_ties": ties,
+                          "near_tie_flips": flips, "rows_sorted": w.n_rounds * w.B * w.H,
+                          "max_abs": worst, "tol": 2e-2})
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -209,6 +309,37 @@ def check_bwd(oracle, inp, nb, chunk, causal, heads=None):
     np.testing.assert_allclose(gQ, rQ, rtol=0, atol=tol)
 
 
+def check_bwd_every_head(oracle, w, inp):
+    """Forward and backward of a full-size workload, every (b, h) head: the
+    hash of every token, every row's permutation, O and lse, dQ and dV."""
+    Q, V, rot, dO = (inp[k].cuda() for k in ("Q", "V", "rot", "dO"))
+    out = L.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal)
+    dQ, dV = L.lsh_attend_bwd(Q, V, out["O"], dO, out["keys"], out["perm"], out["lse"],
+                              w.n_buckets, w.chunk, w.causal)
+    torch.cuda.synchronize()
+    _check_status()
+    ties, flips = hash_every_token(oracle, Q, rot, w.n_buckets, out["keys"])
+    keys_np = out["keys"].cpu().numpy().view(np.uint32)
+    perm_np = out["perm"].cpu().numpy()
+    assert np.array_equal(perm_np, oracle.lsh_sort(keys_np))
+    worst = attention_every_head(oracle, Q, V, out["keys"], out["perm"], w.chunk, w.causal,
+                                 out["O"], out["lse"])
+    tol = TOL[Q.dtype]
+    Qn, Vn, dOn, gQ, gV = (_np(t) for t in (Q, V, dO, dQ, dV))
+
+    def one(bh):
+        b, h = bh
+        rQ, rV = oracle.lsh_attend_bwd(Qn[b:b + 1, h:h + 1], Vn[b:b + 1, h:h + 1],
+                                       dOn[b:b + 1, h:h + 1], keys_np[:, b:b + 1, h:h + 1],
+                                       perm_np[:, b:b + 1, h:h + 1], w.chunk, w.causal)
+        return bh, {"dQ": _err(gQ[b, h], rQ[0, 0], tol), "dV": _err(gV[b, h], rV[0, 0], tol)}
+
+    worst.update(_collect(_pmap(one, _heads(w.B, w.H))))
+    return {"heads": w.B * w.H, "tokens_hashed": w.B * w.H * w.L, "near_ties": ties,
+            "near_tie_flips": flips, "rows_sorted": w.n_rounds * w.B * w.H, "max_abs": worst,
+            "tol": tol}
+
+
 BWD_CASES = [
     (1, 3, 320, 16, 2, 64, True),
     (2, 1, 96, 6, 3, 32, False),
@@ -231,18 +362,20 @@ def test_backward_small_shapes(oracle, dtype, B, H, Lx, nb, R, chunk, causal):
     check_bwd(oracle, inp, nb, chunk, causal)
 
 
-def test_backward_workload_L16384(oracle):
+def test_backward_workload_L16384_every_head(oracle, parity_record):
     w = W.WORKLOADS["fwdbwd_bf16_L16384"]
-    check_bwd(oracle, W.make_inputs(w), w.n_buckets, w.chunk, w.causal, heads=(1, 2))
+    rec = check_bwd_every_head(oracle, w, W.make_inputs(w))
+    parity_record.append({"workload": w.name + " (fwd+bwd)", **rec})
 
 
-def test_backward_L65536_one_head(oracle):
-    """The backward at the headline size (8 rounds, 1024 buckets), one head
-    against the oracle."""
+def test_backward_L65536_every_head(oracle, parity_record):
+    """The backward at the headline size (8 rounds, 1024 buckets), every head
+    against the oracle, with dO ~ N(0, 1) from seed 2."""
     w = W.WORKLOADS["fwd_bf16_L65536"]
     inp = W.make_inputs(w)
     inp["dO"] = W.gaussian(tuple(inp["Q"].shape), 2, inp["Q"].dtype)
-    check_bwd(oracle, inp, w.n_buckets, w.chunk, w.causal, heads=(0, 5))
+    rec = check_bwd_every_head(oracle, w, inp)
+    parity_record.append({"workload": w.name + " (fwd+bwd)", **rec})
 
 
 # ---------------------------------------------------------------------------
