@@ -44,6 +44,15 @@
 //   - near tie: the top two entries z1 >= z2 of [p ; -p] satisfy
 //     z1 - z2 <= 1e-5 * |z1|.
 //
+// Also here: the chunked position-wise feed-forward that sits beside LSH
+// attention in a Reformer layer ("Reformer explainer": a chunked feed-forward
+// with the reversible layers; "Reformer Language Models (Korean)", its
+// Reformer overview: feed-forward activations can dominate memory, so the
+// feed-forward runs in chunks to cut peak memory).  Readings taken: the
+// standard Transformer feed-forward y = W2 relu(W1 x + b1) + b2 at every
+// position; chunking evaluates `chunk` positions at a time, so the hidden
+// activation exists for one chunk only, and does not change the result.
+//
 // Parity pins for every function live in tests/test_oracle_pins.py.
 
 #include <algorithm>
@@ -368,6 +377,90 @@ int oracle_lsh_attend_bwd(int B, int H, int L, int d, int n_rounds, int chunk, i
         }
       }
     }
+  return 0;
+}
+
+// Chunked feed-forward, forward.  X [T, d_model], W1 [d_ff, d_model],
+// b1 [d_ff], W2 [d_model, d_ff], b2 [d_model] -> Y [T, d_model].  Positions
+// are taken `chunk` at a time; for each chunk the hidden activation
+//   h[t, j] = max(0, b1[j] + sum_k W1[j, k] X[t, k])
+// is formed, then
+//   Y[t, i] = b2[i] + sum_j W2[i, j] h[t, j].
+// Returns 0, or 1 on an invalid argument.
+int oracle_ffn_forward(int T, int d_model, int d_ff, int chunk, const double* X, const double* W1,
+                       const double* b1, const double* W2, const double* b2, double* Y) {
+  if (T < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return 1;
+  std::vector<double> h((size_t)chunk * d_ff);
+  for (int c0 = 0; c0 < T; c0 += chunk) {
+    const int n = std::min(chunk, T - c0);
+    for (int t = 0; t < n; ++t) {
+      const double* x = X + (size_t)(c0 + t) * d_model;
+      for (int j = 0; j < d_ff; ++j) {
+        double a = b1[j];
+        for (int k = 0; k < d_model; ++k) a += W1[(size_t)j * d_model + k] * x[k];
+        h[(size_t)t * d_ff + j] = a > 0.0 ? a : 0.0;
+      }
+    }
+    for (int t = 0; t < n; ++t) {
+      double* y = Y + (size_t)(c0 + t) * d_model;
+      for (int i = 0; i < d_model; ++i) {
+        double s = b2[i];
+        for (int j = 0; j < d_ff; ++j) s += W2[(size_t)i * d_ff + j] * h[(size_t)t * d_ff + j];
+        y[i] = s;
+      }
+    }
+  }
+  return 0;
+}
+
+// Chunked feed-forward, backward: gradients of sum(dY * Y) with respect to
+// X, W1, b1, W2, b2 (the weight and bias gradients summed over every
+// position).  Per chunk the pre-activation a = b1 + W1 x and h = max(0, a)
+// are recomputed, then
+//   dW2[i, j] += dY[t, i] h[t, j],   db2[i] += dY[t, i],
+//   dh[t, j] = sum_i W2[i, j] dY[t, i],   da = dh where a > 0, else 0,
+//   dW1[j, k] += da[t, j] X[t, k],   db1[j] += da[t, j],
+//   dX[t, k] = sum_j W1[j, k] da[t, j].
+// The derivative of max(0, a) at a = 0 is taken as 0.
+int oracle_ffn_backward(int T, int d_model, int d_ff, int chunk, const double* X, const double* W1,
+                        const double* b1, const double* W2, const double* dY, double* dX,
+                        double* dW1, double* db1, double* dW2, double* db2) {
+  if (T < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return 1;
+  std::fill(dW1, dW1 + (size_t)d_ff * d_model, 0.0);
+  std::fill(db1, db1 + d_ff, 0.0);
+  std::fill(dW2, dW2 + (size_t)d_model * d_ff, 0.0);
+  std::fill(db2, db2 + d_model, 0.0);
+  std::vector<double> a((size_t)d_ff), h((size_t)d_ff), da((size_t)d_ff);
+  for (int c0 = 0; c0 < T; c0 += chunk) {
+    const int n = std::min(chunk, T - c0);
+    for (int t = 0; t < n; ++t) {
+      const double* x = X + (size_t)(c0 + t) * d_model;
+      const double* dy = dY + (size_t)(c0 + t) * d_model;
+      for (int j = 0; j < d_ff; ++j) {
+        double s = b1[j];
+        for (int k = 0; k < d_model; ++k) s += W1[(size_t)j * d_model + k] * x[k];
+        a[j] = s;
+        h[j] = s > 0.0 ? s : 0.0;
+      }
+      for (int i = 0; i < d_model; ++i) {
+        db2[i] += dy[i];
+        for (int j = 0; j < d_ff; ++j) dW2[(size_t)i * d_ff + j] += dy[i] * h[j];
+      }
+      for (int j = 0; j < d_ff; ++j) {
+        double dh = 0.0;
+        for (int i = 0; i < d_model; ++i) dh += W2[(size_t)i * d_ff + j] * dy[i];
+        da[j] = a[j] > 0.0 ? dh : 0.0;
+        db1[j] += da[j];
+        for (int k = 0; k < d_model; ++k) dW1[(size_t)j * d_model + k] += da[j] * x[k];
+      }
+      double* dx = dX + (size_t)(c0 + t) * d_model;
+      for (int k = 0; k < d_model; ++k) {
+        double s = 0.0;
+        for (int j = 0; j < d_ff; ++j) s += W1[(size_t)j * d_model + k] * da[j];
+        dx[k] = s;
+      }
+    }
+  }
   return 0;
 }
 

@@ -48,9 +48,12 @@ def _load():
         lib.oracle_lsh_attend_fwd_range.argtypes = [I, I, I, I, I, I, I, P, P, P, P, I, I, P, P]
         lib.oracle_lsh_combine.argtypes = [I, I, I, I, I, P, P, P, P]
         lib.oracle_lsh_attend_bwd.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P]
+        lib.oracle_ffn_forward.argtypes = [I, I, I, I, P, P, P, P, P, P]
+        lib.oracle_ffn_backward.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P, P]
         for f in (lib.oracle_lsh_hash, lib.oracle_lsh_sort, lib.oracle_lsh_attend_fwd,
                   lib.oracle_lsh_attend_fwd_range,
-                  lib.oracle_lsh_combine, lib.oracle_lsh_attend_bwd):
+                  lib.oracle_lsh_combine, lib.oracle_lsh_attend_bwd, lib.oracle_ffn_forward,
+                  lib.oracle_ffn_backward):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -166,3 +169,30 @@ def lsh_forward(Q, V, rot, n_buckets: int, chunk: int, causal: bool):
     O, lse = lsh_combine(o_part, lse_r)
     return {"keys": keys, "buckets": buckets, "near_tie": tie, "perm": perm,
             "o_part": o_part, "lse_r": lse_r, "O": O, "lse": lse}
+
+
+def ffn_forward(X, W1, b1, W2, b2, chunk: int):
+    """Chunked feed-forward: X [T, d_model] -> Y [T, d_model] float64."""
+    X, W1, b1, W2, b2 = (_f64(a) for a in (X, W1, b1, W2, b2))
+    T, d_model = X.shape
+    d_ff = W1.shape[0]
+    Y = np.zeros((T, d_model))
+    rc = _load().oracle_ffn_forward(T, d_model, d_ff, chunk, _ptr(X), _ptr(W1), _ptr(b1),
+                                    _ptr(W2), _ptr(b2), _ptr(Y))
+    _check(rc, "oracle_ffn_forward")
+    return Y
+
+
+def ffn_backward(X, W1, b1, W2, dY, chunk: int):
+    """Gradients of sum(dY * Y) -> dX, dW1, db1, dW2, db2 (float64)."""
+    X, W1, b1, W2, dY = (_f64(a) for a in (X, W1, b1, W2, dY))
+    T, d_model = X.shape
+    d_ff = W1.shape[0]
+    dX = np.zeros_like(X)
+    dW1, db1 = np.zeros_like(W1), np.zeros(d_ff)
+    dW2, db2 = np.zeros_like(W2), np.zeros(d_model)
+    rc = _load().oracle_ffn_backward(T, d_model, d_ff, chunk, _ptr(X), _ptr(W1), _ptr(b1),
+                                     _ptr(W2), _ptr(dY), _ptr(dX), _ptr(dW1), _ptr(db1),
+                                     _ptr(dW2), _ptr(db2))
+    _check(rc, "oracle_ffn_backward")
+    return dX, dW1, db1, dW2, db2

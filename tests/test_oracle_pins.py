@@ -421,3 +421,100 @@ def test_chunk_range_restricts_the_full_computation(oracle):
     np.testing.assert_array_equal(l[mask], full_l[mask])
     np.testing.assert_array_equal(o[mask], full_o[mask])
     assert np.all(l[~mask] == 0) and np.all(o[~mask] == 0)
+
+
+# ---------------------------------------------------------------------------
+# chunked feed-forward (the companion op of LSH attention in a Reformer layer)
+# ---------------------------------------------------------------------------
+
+def _ffn_golden():
+    path = os.path.join(os.path.dirname(__file__), "golden", "ffn_small.txt")
+    vals = {}
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            name, *nums = line.split()
+            vals[name] = np.array([float(x) for x in nums])
+    shapes = {"W1": (3, 2), "b1": (3,), "W2": (2, 3), "b2": (2,), "X": (3, 2), "Y": (3, 2),
+              "dY": (3, 2), "dX": (3, 2), "dW1": (3, 2), "db1": (3,), "dW2": (2, 3),
+              "db2": (2,)}
+    return {k: vals[k].reshape(s) for k, s in shapes.items()}
+
+
+def test_ffn_hand_worked_example(oracle):
+    g = _ffn_golden()
+    for chunk in (1, 2, 3):
+        Y = oracle.ffn_forward(g["X"], g["W1"], g["b1"], g["W2"], g["b2"], chunk)
+        np.testing.assert_array_equal(Y, g["Y"])
+        dX, dW1, db1, dW2, db2 = oracle.ffn_backward(g["X"], g["W1"], g["b1"], g["W2"], g["dY"],
+                                                     chunk)
+        for got, name in ((dX, "dX"), (dW1, "dW1"), (db1, "db1"), (dW2, "dW2"), (db2, "db2")):
+            np.testing.assert_array_equal(got, g[name], err_msg=name)
+
+
+def test_ffn_identity_weights_give_relu(oracle):
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((37, 8))
+    I = np.eye(8)
+    Y = oracle.ffn_forward(X, I, np.zeros(8), I, np.zeros(8), 5)
+    np.testing.assert_array_equal(Y, np.maximum(X, 0.0))
+
+
+def test_ffn_zero_second_layer_gives_its_bias(oracle):
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((9, 4))
+    b2 = rng.standard_normal(4)
+    Y = oracle.ffn_forward(X, rng.standard_normal((16, 4)), rng.standard_normal(16),
+                           np.zeros((4, 16)), b2, 4)
+    np.testing.assert_array_equal(Y, np.broadcast_to(b2, Y.shape))
+
+
+def test_ffn_chunking_does_not_change_the_result(oracle):
+    rng = np.random.default_rng(3)
+    T, dm, dff = 50, 16, 64
+    X, W1, b1 = rng.standard_normal((T, dm)), rng.standard_normal((dff, dm)), rng.standard_normal(dff)
+    W2, b2 = rng.standard_normal((dm, dff)), rng.standard_normal(dm)
+    dY = rng.standard_normal((T, dm))
+    whole = oracle.ffn_forward(X, W1, b1, W2, b2, T)
+    gw = oracle.ffn_backward(X, W1, b1, W2, dY, T)
+    for chunk in (1, 7, 16, 49):
+        np.testing.assert_array_equal(oracle.ffn_forward(X, W1, b1, W2, b2, chunk), whole)
+        for a, b in zip(oracle.ffn_backward(X, W1, b1, W2, dY, chunk), gw):
+            np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-12)
+
+
+def test_ffn_matches_library_matmuls(oracle):
+    rng = np.random.default_rng(4)
+    T, dm, dff = 33, 24, 96
+    X, W1, b1 = rng.standard_normal((T, dm)), rng.standard_normal((dff, dm)), rng.standard_normal(dff)
+    W2, b2 = rng.standard_normal((dm, dff)), rng.standard_normal(dm)
+    ref = np.maximum(X @ W1.T + b1, 0.0) @ W2.T + b2
+    np.testing.assert_allclose(oracle.ffn_forward(X, W1, b1, W2, b2, 8), ref, rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_ffn_backward_matches_finite_differences(oracle):
+    rng = np.random.default_rng(5)
+    T, dm, dff = 6, 5, 7
+    X, W1, b1 = rng.standard_normal((T, dm)), rng.standard_normal((dff, dm)), rng.standard_normal(dff)
+    W2, b2 = rng.standard_normal((dm, dff)), rng.standard_normal(dm)
+    dY = rng.standard_normal((T, dm))
+    grads = dict(zip(("X", "W1", "b1", "W2", "b2"),
+                     oracle.ffn_backward(X, W1, b1, W2, dY, 4)))
+    params = {"X": X, "W1": W1, "b1": b1, "W2": W2, "b2": b2}
+    eps = 1e-6
+
+    def loss():
+        return float((dY * oracle.ffn_forward(params["X"], params["W1"], params["b1"],
+                                              params["W2"], params["b2"], 4)).sum())
+
+    for name, p in params.items():
+        num = np.zeros_like(p)
+        for idx in np.ndindex(p.shape):
+            keep = p[idx]
+            p[idx] = keep + eps
+            up = loss()
+            p[idx] = keep - eps
+            down = loss()
+            p[idx] = keep
+            num[idx] = (up - down) / (2 * eps)
+        np.testing.assert_allclose(grads[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
