@@ -196,3 +196,64 @@ def ffn_backward(X, W1, b1, W2, dY, chunk: int):
                                      _ptr(dW2), _ptr(db2))
     _check(rc, "oracle_ffn_backward")
     return dX, dW1, db1, dW2, db2
+
+
+# ---------------------------------------------------------------------------
+# reversible residual block around LSH attention (composition of the above)
+# ---------------------------------------------------------------------------
+
+def _heads(x, H):
+    """[B, L, H*d] (token-major) -> [B, H, L, d]."""
+    B, L, D = x.shape
+    return np.ascontiguousarray(x.reshape(B, L, H, D // H).transpose(0, 2, 1, 3))
+
+
+def _tokens(x):
+    """[B, H, L, d] -> [B, L, H*d]."""
+    B, H, L, d = x.shape
+    return np.ascontiguousarray(x.transpose(0, 2, 1, 3).reshape(B, L, H * d))
+
+
+def rev_attention(x, keys, perm, H, chunk, causal):
+    """F(x): LSH attention with the token's own features as query (= key)
+    and value, head by head: [B, L, H*d] -> [B, L, H*d], buckets given."""
+    q = _heads(_f64(x), H)
+    o_part, lse_r = lsh_attend_fwd(q, q, keys, perm, chunk, causal)
+    O, _ = lsh_combine(o_part, lse_r)
+    return _tokens(O)
+
+
+def rev_forward(X1, X2, rot, n_buckets, H, chunk, causal, W1, b1, W2, b2, ffn_chunk):
+    """Reversible block (RevNet residuals, as the Reformer abstract and the
+    explainer describe): Y1 = X1 + F(X2), Y2 = X2 + G(Y1), with F = LSH
+    attention of X2 and G the chunked feed-forward.  Returns Y1, Y2 and the
+    keys and permutations of X2's hash, which the backward holds constant."""
+    X1, X2 = _f64(X1), _f64(X2)
+    B, L, D = X2.shape
+    keys, _, _ = lsh_hash(_heads(X2, H), rot, n_buckets)
+    perm = lsh_sort(keys)
+    Y1 = X1 + rev_attention(X2, keys, perm, H, chunk, causal)
+    Y2 = X2 + ffn_forward(Y1.reshape(B * L, D), W1, b1, W2, b2, ffn_chunk).reshape(B, L, D)
+    return Y1, Y2, keys, perm
+
+
+def rev_backward(Y1, Y2, dY1, dY2, keys, perm, H, chunk, causal, W1, b1, W2, b2, ffn_chunk):
+    """Backward of the reversible block from its outputs alone: the inputs
+    are recomputed (X2 = Y2 - G(Y1), X1 = Y1 - F(X2)), not stored.  With the
+    buckets held constant:
+      dY1' = dY1 + G'(Y1)^T dY2,   dX2 = dY2 + F'(X2)^T dY1',   dX1 = dY1',
+    and the feed-forward's weight and bias gradients.  F'(x)^T g is the sum
+    of the attention's query and value gradients (both are x).
+    Returns X1, X2, dX1, dX2, dW1, db1, dW2, db2."""
+    Y1, Y2, dY1, dY2 = (_f64(a) for a in (Y1, Y2, dY1, dY2))
+    B, L, D = Y1.shape
+    T = B * L
+    X2 = Y2 - ffn_forward(Y1.reshape(T, D), W1, b1, W2, b2, ffn_chunk).reshape(B, L, D)
+    gY1, dW1, db1, dW2, db2 = ffn_backward(Y1.reshape(T, D), W1, b1, W2, dY2.reshape(T, D),
+                                           ffn_chunk)
+    dY1p = dY1 + gY1.reshape(B, L, D)
+    X1 = Y1 - rev_attention(X2, keys, perm, H, chunk, causal)
+    q = _heads(X2, H)
+    dQ, dV = lsh_attend_bwd(q, q, _heads(dY1p, H), keys, perm, chunk, causal)
+    dX2 = dY2 + _tokens(dQ + dV)
+    return X1, X2, dY1p, dX2, dW1, db1, dW2, db2

@@ -518,3 +518,67 @@ def test_ffn_backward_matches_finite_differences(oracle):
             p[idx] = keep
             num[idx] = (up - down) / (2 * eps)
         np.testing.assert_allclose(grads[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+# ---------------------------------------------------------------------------
+# reversible residual block (Y1 = X1 + F(X2), Y2 = X2 + G(Y1); F = LSH
+# attention of X2 with its buckets held constant, G = chunked feed-forward)
+# ---------------------------------------------------------------------------
+
+def _rev_case(seed, B=1, L=16, H=1, d=64, dff=32, nb=4, R=2):
+    rng = np.random.default_rng(seed)
+    D = H * d
+    return dict(X1=rng.standard_normal((B, L, D)), X2=rng.standard_normal((B, L, D)),
+                rot=rng.standard_normal((R, d, nb // 2)), nb=nb, H=H,
+                W1=rng.standard_normal((dff, D)) / np.sqrt(D), b1=0.1 * rng.standard_normal(dff),
+                W2=rng.standard_normal((D, dff)) / np.sqrt(dff), b2=0.1 * rng.standard_normal(D),
+                dY1=rng.standard_normal((B, L, D)), dY2=rng.standard_normal((B, L, D)))
+
+
+def test_reversible_block_reconstructs_its_inputs(oracle):
+    """The RevNet property: the backward recovers X1 and X2 from Y1 and Y2."""
+    c = _rev_case(1, L=64, H=2)
+    Y1, Y2, keys, perm = oracle.rev_forward(c["X1"], c["X2"], c["rot"], c["nb"], c["H"], 8, True,
+                                            c["W1"], c["b1"], c["W2"], c["b2"], 16)
+    X1, X2 = oracle.rev_backward(Y1, Y2, c["dY1"][:, :64], c["dY2"][:, :64], keys, perm,
+                                 c["H"], 8, True, c["W1"], c["b1"], c["W2"], c["b2"], 16)[:2]
+    np.testing.assert_allclose(X1, c["X1"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(X2, c["X2"], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_reversible_block_gradients_match_finite_differences(oracle, causal):
+    """Gradients of sum(dY1 * Y1 + dY2 * Y2), buckets held at those of the
+    unperturbed X2, against central differences in fp64."""
+    c = _rev_case(2 + causal)
+    chunk, fchunk = 4, 8
+    Y1, Y2, keys, perm = oracle.rev_forward(c["X1"], c["X2"], c["rot"], c["nb"], c["H"], chunk,
+                                            causal, c["W1"], c["b1"], c["W2"], c["b2"], fchunk)
+    got = dict(zip(("X1", "X2", "dX1", "dX2", "W1", "b1", "W2", "b2"),
+                   oracle.rev_backward(Y1, Y2, c["dY1"], c["dY2"], keys, perm, c["H"], chunk,
+                                       causal, c["W1"], c["b1"], c["W2"], c["b2"], fchunk)))
+    grads = {"X1": got["dX1"], "X2": got["dX2"], "W1": got["W1"], "b1": got["b1"],
+             "W2": got["W2"], "b2": got["b2"]}
+    p = {k: c[k].copy() for k in ("X1", "X2", "W1", "b1", "W2", "b2")}
+    B, L, D = p["X1"].shape
+
+    def loss():
+        y1 = p["X1"] + oracle.rev_attention(p["X2"], keys, perm, c["H"], chunk, causal)
+        y2 = p["X2"] + oracle.ffn_forward(y1.reshape(B * L, D), p["W1"], p["b1"], p["W2"],
+                                          p["b2"], fchunk).reshape(B, L, D)
+        return float((c["dY1"] * y1).sum() + (c["dY2"] * y2).sum())
+
+    rng = np.random.default_rng(7)
+    eps = 1e-6
+    for name, arr in p.items():
+        flat = arr.reshape(-1)
+        for idx in rng.choice(flat.size, size=min(24, flat.size), replace=False):
+            keep = flat[idx]
+            flat[idx] = keep + eps
+            up = loss()
+            flat[idx] = keep - eps
+            down = loss()
+            flat[idx] = keep
+            num = (up - down) / (2 * eps)
+            ana = grads[name].reshape(-1)[idx]
+            assert abs(ana - num) <= 1e-6 * max(1.0, abs(num)), (name, idx, ana, num)
