@@ -3,12 +3,15 @@
 
 Headline: forward tokens/s (B*L per second, all heads and 8 hash rounds) on
 the L=65536 workload (B=1, H=8, d=64, n_buckets=1024, n_rounds=8, chunk=64,
-causal, bf16), one step = hash -> sort -> chunk attention with the fused
-round combine, inputs resident in HBM, L2 flushed (256 MB memset) between
-timed steps.  Also reported: fwd+bwd tokens/s (L=16384 workload and an
-L=65536 variant), the same forward end to end from pinned host buffers, per
-stage times, the roofline of the dominant kernel, clocks, and the CPU
-oracle timed on the host cores.
+causal, bf16), one step = hash -> sort -> chunk attention -> round combine,
+inputs resident in HBM, L2 flushed (256 MB memset) between timed steps.
+Also reported: fwd+bwd tokens/s with the backward's roofline (L=16384
+workload and an L=65536 variant), the same forward end to end from pinned
+host buffers, per-stage times, the roofline of the dominant kernel, every
+other workload's forward with its roofline, recall against full attention
+over rounds and bucket counts, the chunked feed-forward's positions/s with
+its tensor roofline, clocks, and the CPU oracle timed on the host cores
+(with a parity record of the head it recomputes).
 
 ``--impl reference`` times the CPU oracle (the reference arm) on a bounded
 sample of the same workload.  Under torchrun every rank runs the full
@@ -59,6 +62,12 @@ def parse_args():
     p.add_argument("--recall", action="store_true",
                    help="recall of LSH attention against full attention on the clustered "
                         "L=16384 workload, over rounds and bucket counts (a report)")
+    p.add_argument("--shard", choices=["none", "heads"], default="none",
+                   help="heads: split one problem's B*H heads over the ranks (strong "
+                        "scaling) instead of a replica per rank")
+    p.add_argument("--gather", action="store_true",
+                   help="with --shard heads: all-gather O and lse to every rank inside "
+                        "the timed step")
     p.add_argument("--ref-seconds", type=float, default=150.0,
                    help="--impl reference: CPU seconds of oracle sampling over all steps")
     return p.parse_args()
@@ -197,6 +206,11 @@ def stage_work(w: W.Workload):
         "attend": {"bytes": tr * (2 * d * s + 8) + 2 * n_tok * (R - 1) * (4 * d + 4)
                    + n_tok * (d * s + 4),
                    "flops": tr * 8 * w.chunk * d},
+        # per token-round: perm and key, q, v and dO rows, lse and G, three
+        # fp32 accumulator rows read and written once; per token: the dQ, dV
+        # writes and the O, dO reads of G = dO . O, spread over R rounds
+        "bwd": {"bytes": tr * (4 + 4 + 3 * d * s + 8 + 3 * 4 * d) + n_tok * (2 * d * s + 3 * 4 * d),
+                "flops": tr * 20 * w.chunk * d},
     }
 
 
@@ -217,14 +231,37 @@ def device_inputs(w: W.Workload, dev):
     return {k: v.to(dev) for k, v in inp.items()}
 
 
-def run_ours(args, world, rank):
+def roofline_of(w: W.Workload, stage: str, ms: float, peaks, peak_kind, traffic=None):
+    """The roofline line of one stage: algorithmic work of one launch over its
+    measured time, against the stage's binding peak."""
+    work = stage_work(w)[stage]
+    sec = ms / 1e3
+    if stage == "hash" and w.dtype == "bf16" and w.n_buckets >= 256:
+        tfs = work["flops"] / sec / 1e12
+        return {"bound": "tensor", "kernel": stage, "achieved": round(tfs, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tfs / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "peak_source": peak_kind}
+    gbs = work["bytes"] / sec / 1e9
+    return {"bound": "hbm", "kernel": stage, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+            "peak_source": peak_kind}
+
+
+def time_forward(w: W.Workload, steps: int, warmup: int, world: int, sample_clocks: bool = False,
+                 inputs=None, after_step=None):
+    """hash -> sort -> attend (with the combine) on device-resident inputs, L2
+    flushed before each step; CUDA events per stage on the launching stream.
+    `inputs` (device Q, V, rot) replaces the workload's own, e.g. one rank's
+    heads of it; `after_step(O, lse)` runs inside each timed step, after the
+    attention (its time counts with the attention's).
+    Returns (total ms over the steps, per-stage ms per step, clocks, outputs)."""
     import lsh_attention_long_b200 as L
-    L.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = W.WORKLOADS[args.workload]
-    t = device_inputs(w, dev)
+    t = inputs if inputs is not None else device_inputs(w, dev)
     Q, V, rot = t["Q"], t["V"], t["rot"]
-    R, B, H, Lx = w.n_rounds, w.B, w.H, w.L
+    R, Lx = w.n_rounds, w.L
+    B, H = Q.shape[:2]
     shape = L.make_shape(B, H, Lx, w.d, w.n_buckets, R, w.chunk, w.causal, Q.dtype)
     ws = L.workspace(shape, dev)
     keys = torch.empty((R, B, H, Lx), dtype=torch.int32, device=dev)
@@ -233,6 +270,7 @@ def run_ours(args, world, rank):
     lse = torch.empty((B, H, Lx), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
 
     def step():
         L.lsh_hash(Q, rot, w.n_buckets, keys=keys, want_buckets=False)
@@ -240,9 +278,10 @@ def run_ours(args, world, rank):
         L.lsh_sort(keys, w.n_buckets, perm=perm)
         ev[2].record(stream)
         L.lsh_attend_fwd(Q, V, keys, perm, w.n_buckets, w.chunk, w.causal, O=O, lse=lse, ws=ws)
+        if after_step is not None:
+            after_step(O, lse)
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         ev[0].record(stream)
         step()
@@ -250,13 +289,12 @@ def run_ours(args, world, rank):
     torch.cuda.synchronize()
     if L.lsh_device_status() != 0:
         raise RuntimeError("device status error during warm-up")
-
     stage_ms = {"hash": 0.0, "sort": 0.0, "attend": 0.0}
     total_ms = 0.0
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        for _ in range(args.steps):
+    with ClockSampler(dev.index) if sample_clocks else _NoClocks() as clocks:
+        for _ in range(steps):
             flush.zero_()
             ev[0].record(stream)
             step()
@@ -272,56 +310,188 @@ def run_ours(args, world, rank):
     if L.lsh_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
     total_ms = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms / args.steps
-    # hash_tc, sort_rows, then key_scale + attend_tc + online_merge
-    launches_per_step = 1 + 1 + 3
-    value = aggregate_tokens_per_s(world, B * Lx, args.steps, total_ms)
+    per_stage = {k: v / steps for k, v in stage_ms.items()}
+    del flush, ws
+    return total_ms, per_stage, clocks.summary(), {"keys": keys, "perm": perm, "O": O, "lse": lse}
 
-    peaks, peak_kind = load_peaks()
+
+class _NoClocks:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+    def summary(self):
+        return None
+
+
+def stage_lines(w: W.Workload, per_stage: dict, peaks) -> dict:
     work = stage_work(w)
-    stages = {}
-    for name, ms in stage_ms.items():
-        sec = ms / args.steps / 1e3
+    out = {}
+    for name, ms in per_stage.items():
+        sec = ms / 1e3
         gbs = work[name]["bytes"] / sec / 1e9
         tfs = work[name]["flops"] / sec / 1e12
-        stages[name] = {"ms": round(ms / args.steps, 4), "GB_s": round(gbs, 1),
-                        "TFLOP_s": round(tfs, 2),
-                        "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
-                        "tensor_frac": round(tfs / peaks["bf16_tflops"], 4)}
-    dom = max(stage_ms, key=stage_ms.get)
-    bound = "tensor" if dom == "hash" and w.dtype == "bf16" and w.n_buckets >= 256 else "hbm"
-    traffic = TRAFFIC.get((dom, w.name))
-    if bound == "hbm":
-        roof = {"bound": "hbm", "kernel": dom, "achieved": stages[dom]["GB_s"],
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": stages[dom]["hbm_frac"],
-                "traffic": traffic, "peak_source": peak_kind}
-    else:
-        roof = {"bound": "tensor", "kernel": dom, "achieved": stages[dom]["TFLOP_s"],
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": stages[dom]["tensor_frac"], "traffic": traffic,
-                "peak_source": peak_kind}
+        out[name] = {"ms": round(ms, 4), "GB_s": round(gbs, 1), "TFLOP_s": round(tfs, 2),
+                     "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "tensor_frac": round(tfs / peaks["bf16_tflops"], 4)}
+    return out
+
+
+def workload_config(w: W.Workload) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+            "n_buckets": w.n_buckets, "n_rounds": w.n_rounds, "chunk": w.chunk,
+            "causal": w.causal}
+
+
+def run_ours(args, world, rank):
+    import lsh_attention_long_b200 as L
+    L.load_library()
+    w = W.WORKLOADS[args.workload]
+    total_ms, per_stage, clocks, outs = time_forward(w, args.steps, args.warmup, world,
+                                                     sample_clocks=True)
+    ms_per_step = total_ms / args.steps
+    # hash_tc, sort_rows, then key_scale + attend_tc + combine
+    launches_per_step = 1 + 1 + 3
+    value = aggregate_tokens_per_s(world, w.B * w.L, args.steps, total_ms)
+    peaks, peak_kind = load_peaks()
+    stages = stage_lines(w, per_stage, peaks)
+    dom = max(per_stage, key=per_stage.get)
+    roof = roofline_of(w, dom, per_stage[dom], peaks, peak_kind, TRAFFIC.get((dom, w.name)))
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian Q, V, rotations)",
-        "config": {"workload": w.name, "B": B, "H": H, "L": Lx, "d": w.d,
-                   "n_buckets": w.n_buckets, "n_rounds": R, "chunk": w.chunk,
-                   "causal": w.causal, "l2": "flushed between timed steps (256 MB memset)",
-                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "config": workload_config(w),
+        "l2": "flushed between timed steps (256 MB memset)",
+        "parallelism": f"replicas x{world} (independent problems per GPU)",
         "roofline": roof, "stages": stages,
         # the same rate counted in (batch, head, position, round) units
-        "head_token_rounds_per_s": round(value * H * R, 1),
+        "head_token_rounds_per_s": round(value * w.H * w.n_rounds, 1),
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clocks,
     }
     if not args.no_extras:
         result["e2e"] = run_e2e(args, w, world)
         result["fwd_bwd"] = {BWD_WORKLOAD: run_fwd_bwd(args, W.WORKLOADS[BWD_WORKLOAD], world),
                              "fwd_bf16_L65536+bwd": run_fwd_bwd(args, w, world)}
-    del flush, ws
+        result["workloads"] = run_other_workloads(args, w, world, peaks, peak_kind)
+        result["recall"] = run_recall(args)
+        result["ffn"] = run_ffn(args, world)
+    # the head the CPU baseline recomputes, for its parity record
+    result["_head0"] = {k: v[:, :1, :1].cpu() if k in ("keys", "perm") else v[:1, :1].cpu()
+                        for k, v in outs.items()}
     return result
+
+
+def run_sharded(args, world, rank):
+    """One problem (the workload) split over the ranks by (batch, head): rank
+    k runs hash -> sort -> attend on its contiguous slice of the B*H heads;
+    no data-path collective, unless --gather all-gathers O and lse inside the
+    timed step.  value = the whole problem's tokens per second, timed by the
+    slowest rank (strong scaling: the total work is fixed)."""
+    import lsh_attention_long_b200 as L
+    from lsh_attention_long_b200 import shard
+    L.load_library()
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    full = W.make_inputs(w)
+    h0, h1 = shard.head_range(w.B * w.H, world, rank)
+    t = {"Q": shard.head_slice(full["Q"], world, rank).contiguous().to(dev),
+         "V": shard.head_slice(full["V"], world, rank).contiguous().to(dev),
+         "rot": full["rot"].to(dev)}
+    after = None
+    if args.gather:
+        def after(O, lse):
+            shard.all_gather_heads(O, w.B, w.H, world, rank)
+            shard.all_gather_heads(lse, w.B, w.H, world, rank)
+    total_ms, per_stage, clocks, _ = time_forward(w, args.steps, args.warmup, world,
+                                                  sample_clocks=True, inputs=t, after_step=after)
+    value = w.B * w.L * args.steps / (total_ms / 1e3)
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian Q, V, rotations)", "config": workload_config(w),
+        "l2": "flushed between timed steps (256 MB memset)",
+        "parallelism": f"(batch, head) shards of one problem over {world} ranks; rank 0 holds "
+                       f"heads [{h0}, {h1}) of {w.B * w.H}"
+                       + ("; O and lse all-gathered in the timed step" if args.gather else ""),
+        "stages_rank0": {k: round(v, 4) for k, v in per_stage.items()},
+        "gpu_launches": 5 * args.steps, "clocks": clocks,
+    }
+
+
+def run_ffn(args, world):
+    """The chunked feed-forward (65 536 positions, 512 -> 2048 -> 512, chunks
+    of 8192) on device-resident inputs, L2 flushed between steps: positions
+    per second and the tensor-pipe roofline of its two products (4 * T *
+    d_model * d_ff flops per step)."""
+    import lsh_attention_long_b200 as L
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.FFN_WORKLOADS["ffn_bf16_L65536"]
+    t = {k: v.to(dev) for k, v in W.ffn_inputs(w.tokens, w.d_model, w.d_ff).items()}
+    Y = torch.empty_like(t["X"])
+    ws = L.ffn_workspace(w.tokens, w.d_model, w.d_ff, w.chunk, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(5, args.steps // 2)
+
+    def step():
+        L.lsh_ffn_forward(t["X"], t["W1"], t["b1"], t["W2"], t["b2"], w.chunk, Y=Y, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+    barrier(world)
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error in the feed-forward")
+    ms = max_over_ranks(ms, world) / steps
+    peaks, peak_kind = load_peaks()
+    tfs = 4.0 * w.tokens * w.d_model * w.d_ff / (ms / 1e3) / 1e12
+    del flush, ws
+    return {"value": round(world * w.tokens / (ms / 1e3), 1), "unit": "positions/s",
+            "ms_per_step": round(ms, 4), "steps": steps, "config": w.describe(),
+            "launches_per_step": 2 * (w.tokens // w.chunk),
+            "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (both products)",
+                         "achieved": round(tfs, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tfs / peaks["bf16_tflops"], 4),
+                         "traffic": TRAFFIC.get(("ffn", w.name)), "peak_source": peak_kind}}
+
+
+def run_other_workloads(args, headline, world, peaks, peak_kind):
+    """Forward tokens/s and the dominant stage's roofline of every other
+    workload (the small fp32 one, L=4096, the clustered L=16384 and the
+    fwd+bwd workload's forward), timed as the headline."""
+    out = {}
+    steps = max(5, args.steps // 2)
+    for name, w in W.WORKLOADS.items():
+        if name == headline.name:
+            continue
+        total_ms, per_stage, _, _ = time_forward(w, steps, max(3, args.warmup), world)
+        dom = max(per_stage, key=per_stage.get)
+        out[name] = {"value": round(aggregate_tokens_per_s(world, w.B * w.L, steps, total_ms), 1),
+                     "unit": "tokens/s", "ms_per_step": round(total_ms / steps, 4),
+                     "steps": steps, "config": workload_config(w),
+                     "stages": stage_lines(w, per_stage, peaks),
+                     "roofline": roofline_of(w, dom, per_stage[dom], peaks, peak_kind,
+                                             TRAFFIC.get((dom, name)))}
+    return out
 
 
 def run_e2e(args, w, world):
@@ -411,10 +581,14 @@ def run_fwd_bwd(args, w, world):
     if L.lsh_device_status() != 0:
         raise RuntimeError("device status error in fwd+bwd")
     tot = max_over_ranks(fwd + bwd, world)
+    peaks, peak_kind = load_peaks()
     return {"value": round(aggregate_tokens_per_s(world, w.B * w.L, steps, tot), 1), "unit": "tokens/s",
             "ms_fwd": round(fwd / steps, 4), "ms_bwd": round(bwd / steps, 4), "steps": steps,
-            "config": {"B": w.B, "H": w.H, "L": w.L, "n_buckets": w.n_buckets,
-                       "n_rounds": w.n_rounds, "chunk": w.chunk, "causal": w.causal}}
+            "config": workload_config(w),
+            # the backward call (G = dO . O, key scales, the tensor-core kernel,
+            # the cast) against HBM with the survey's algorithmic bytes
+            "roofline_bwd": roofline_of(w, "bwd", bwd / steps, peaks, peak_kind,
+                                        TRAFFIC.get(("bwd", w.name)))}
 
 
 # ---------------------------------------------------------------------------
@@ -536,7 +710,6 @@ def run_recall(args):
 # From one ncu capture of the timed step of `bench.py --steps 1 --warmup 1
 # --no-extras`; to be cleared whenever the kernel changes.
 TRAFFIC = {
-    ("attend", "fwd_bf16_L65536"): 1084709000 + 989513472,
     ("hash", "fwd_bf16_L65536"): 67665000 + 4091648,
     ("sort", "fwd_bf16_L65536"): 19975000 + 3175936,
 }
@@ -612,24 +785,47 @@ def host_cpu() -> dict:
     return {"cpu_model": model, "nproc": os.cpu_count()}
 
 
-def run_cpu_baseline(w):
+def run_cpu_baseline(w, head0=None):
     """The oracle as it stands on one whole head (b=0, h=0) of the workload:
-    hash, sort, attention and combine for all rounds, scaled by B*H."""
+    hash, sort, attention and combine for all rounds, scaled by B*H.  With the
+    GPU's outputs for that head (head0), the oracle's results also give a
+    parity record outside the timed region: near ties among the head's hashes,
+    bucket ids and permutations that differ, and the largest errors of O and
+    lse (the oracle's attention fed the GPU's keys and permutations)."""
     from oracle import oracle as cpu_oracle
     cpu_oracle.build()
+    import numpy as np
     inp = W.make_inputs(w)
     Q = inp["Q"][:1, :1].float().numpy()
     V = inp["V"][:1, :1].float().numpy()
     rot = inp["rot"].float().numpy()
     t0 = time.perf_counter()
-    cpu_oracle.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal)
+    ref = cpu_oracle.lsh_forward(Q, V, rot, w.n_buckets, w.chunk, w.causal)
     sec = time.perf_counter() - t0
     full = sec * w.B * w.H
-    return {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": 1,
-            "kind": "oracle", **host_cpu(),
-            "sample": f"one head (b=0, h=0) of {w.name}, all {w.n_rounds} rounds, full "
-                      f"L={w.L}: hash, sort, attention, combine in {sec:.1f} s single-threaded "
-                      f"fp64; scaled by B*H={w.B * w.H} to the whole step"}
+    res = {"value": round(w.B * w.L / full, 3), "unit": "tokens/s", "cores": 1,
+           "kind": "oracle", **host_cpu(),
+           "sample": f"one head (b=0, h=0) of {w.name}, all {w.n_rounds} rounds, full "
+                     f"L={w.L}: hash, sort, attention, combine in {sec:.1f} s single-threaded "
+                     f"fp64; scaled by B*H={w.B * w.H} to the whole step"}
+    if head0 is not None:
+        keys = head0["keys"].numpy().view(np.uint32)
+        perm = head0["perm"].numpy()
+        gb = keys // np.uint32(w.L)
+        tie = ref["near_tie"] != 0
+        diff = gb != ref["buckets"]
+        o_part, lse_r = cpu_oracle.lsh_attend_fwd(Q, V, keys, perm, w.chunk, w.causal)
+        O, lse = cpu_oracle.lsh_combine(o_part, lse_r)
+        res["parity_head0"] = {
+            "tokens_hashed": int(keys.size), "near_ties": int(tie.sum()),
+            "bucket_mismatch_outside_near_ties": int((diff & ~tie).sum()),
+            "near_tie_flips": int((diff & tie).sum()),
+            "perm_equal_to_oracle_sort_of_gpu_keys": bool(np.array_equal(perm,
+                                                                         cpu_oracle.lsh_sort(keys))),
+            "O_max_abs": float(np.abs(head0["O"].float().numpy() - O).max()),
+            "lse_max_abs": float(np.abs(head0["lse"].numpy() - lse).max()),
+            "tol": 2e-2 if w.dtype == "bf16" else 2e-3}
+    return res
 
 
 def run_cpu_baseline_threads(w):
@@ -687,9 +883,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(per * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
-                   "n_buckets": w.n_buckets, "n_rounds": w.n_rounds, "chunk": w.chunk,
-                   "causal": w.causal},
+        "config": workload_config(w),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1,
                          "kind": "oracle", "sample": sample, **host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -720,9 +914,15 @@ def main():
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return
+        if args.shard == "heads":
+            res = run_sharded(args, world, rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_ours(args, world, rank)
+        head0 = res.pop("_head0")
         if rank == 0 and not args.no_extras and world == 1:
-            res["cpu_baseline"] = run_cpu_baseline(W.WORKLOADS[args.workload])
+            res["cpu_baseline"] = run_cpu_baseline(W.WORKLOADS[args.workload], head0)
             res["cpu_baseline_threads"] = run_cpu_baseline_threads(W.WORKLOADS[args.workload])
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)

@@ -41,6 +41,10 @@
  *     even number 2..32768; n_buckets * L < 2^31; B*H*L*n_rounds < 2^31;
  *     n_rounds*B*H <= 65535; chunk >= 1 divides L; chunk <= 64.  B, H or L
  *     equal to 0 is an empty call that returns LSH_OK without launching.
+ *   - On the tensor-core path of the attention (bf16 and chunk == 64) the
+ *     softmax weights and V enter the weights-times-values product in fp16:
+ *     |V| must stay below 65504, and values below 2^-24 in magnitude count
+ *     as zero there.
  *   - Every buffer must be 16-byte aligned.
  */
 #ifndef LSH_ATTENTION_LSH_H_
@@ -114,9 +118,13 @@ LSH_API lsh_status lsh_sort(const lsh_shape* shape, const uint32_t* keys, int32_
  * o_part: [R,B,H,L,d] fp32 or NULL; lse_r: [R,B,H,L] fp32 or NULL.
  * O: [B,H,L,d] in dtype, or NULL to skip the combine (then o_part and lse_r
  * are required and receive every round).  lse: [B,H,L] fp32 or NULL.
- * When O is given, the combine runs in the epilogue of the last round;
- * partials of the earlier rounds go to o_part/lse_r when given, else to ws
- * (then ws_bytes >= lsh_workspace_size()). */
+ * When O is given, the rounds are combined into O and lse (fp32 o_part
+ * and lse_r receive every round when given).  Scratch comes from ws
+ * (ws_bytes >= lsh_workspace_size()): on the tensor-core path (bf16, chunk
+ * 64) the per-token key scales, the values in fp16 and, unless the caller
+ * takes o_part or there is one round, every round's fp16 output and fp32
+ * logsumexp, which a combine kernel then reads; on the CUDA-core path the
+ * partials of rounds 0..R-2, combined in the epilogue of the last round. */
 LSH_API lsh_status lsh_attend_fwd(const lsh_shape* shape, const void* Q, const void* V,
                           const uint32_t* keys, const int32_t* perm, float* o_part,
                           float* lse_r, void* O, float* lse, void* ws, size_t ws_bytes,
@@ -129,7 +137,7 @@ LSH_API lsh_status lsh_combine(const lsh_shape* shape, const float* o_part, cons
                        float* lse, void* stream);
 
 /* Whole forward in one call: lsh_hash -> lsh_sort -> lsh_attend_fwd with the
- * fused combine.  keys and perm are outputs (they are also what the backward
+ * combine.  keys and perm are outputs (they are also what the backward
  * needs); buckets may be NULL; lse [B,H,L] fp32 is required (the backward
  * needs it).  ws_bytes >= lsh_workspace_size(). */
 LSH_API lsh_status lsh_forward(const lsh_shape* shape, const void* Q, const void* V, const void* rot,
@@ -187,11 +195,12 @@ LSH_API lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const v
  *   - Capacity.  With n = B * H * L tokens, and every part below rounded up
  *     to a multiple of 256 bytes, the scratch a call needs is
  *       tensor-core path (dtype LSH_BF16 and chunk == 64):
- *         (n_rounds * B * H + 1) * 4   tile and ticket counters
- *       + n * 4                        per-token key scales
- *       + k * n * 256 + k * n * 16     running (output, max, sum) states,
- *                                      k = 2 if n_rounds > 1, else 1;
- *       so about 276 bytes per token for one round and 548 for more;
+ *         n * 4                        per-token key scales
+ *       + n * 64 * 2                   the values in fp16
+ *       + n_rounds * n * 64 * 2        fp16 outputs of every round
+ *       + n_rounds * n * 4             logsumexps of every round,
+ *       the last two only when n_rounds > 1; so 132 bytes per token for
+ *       one round, 396 for two, 660 for four, 1188 for eight;
  *       CUDA-core path (every other supported case):
  *         (n_rounds - 1) * n * d * 4 + (n_rounds - 1) * n * 4
  *                                      partials of rounds 0 .. n_rounds-2,
@@ -215,6 +224,45 @@ LSH_API lsh_status lsh_attend_bwd(const lsh_shape* shape, const void* Q, const v
 LSH_API lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const void* V,
                                          const uint32_t* keys, const int32_t* perm, void* O,
                                          float* lse, void* stream);
+
+/* Chunked position-wise feed-forward, the companion of LSH attention in a
+ * Reformer layer ("Reformer explainer", its single section: a chunked
+ * feed-forward beside LSH attention and reversible layers; "Reformer Language
+ * Models (Korean)", Reformer overview: feed-forward activations can dominate
+ * memory, so the feed-forward is chunked to cut peak memory).  Per position
+ *   Y[t] = W2 max(0, W1 X[t] + b1) + b2,
+ * taken `chunk` positions at a time, so the hidden activation exists for one
+ * chunk only (in ws).  Chunking does not change the result.
+ *   X, Y: [tokens, d_model] bf16;  W1: [d_ff, d_model] bf16;  b1: [d_ff]
+ *   bf16;  W2: [d_model, d_ff] bf16;  b2: [d_model] bf16 (row-major, device).
+ * Both products run on the tensor cores with fp32 accumulation; the hidden
+ * activation is rounded to bf16 between them.  Supported: d_model and d_ff
+ * multiples of 256, tokens and chunk multiples of 128, tokens * d_model and
+ * chunk * d_ff below 2^31; else LSH_ERR_UNSUPPORTED.  ws: at least
+ * lsh_ffn_ws_size() bytes of device scratch (chunk * d_ff * 2), caller-owned.
+ * Asynchronous on `stream`; nothing is allocated. */
+LSH_API size_t lsh_ffn_ws_size(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk);
+LSH_API lsh_status lsh_ffn_forward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk,
+                                   const void* X, const void* W1, const void* b1, const void* W2,
+                                   const void* b2, void* Y, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Test hook for the failure path of the bounded device waits.  No passage of
+ * the pages corresponds to it.  Every wait in the kernels gives up after a
+ * limit of clock cycles (about 2 s by default), records LSH_ERR_TIMEOUT in
+ * the device status word, stops its thread block cleanly (in-flight copies and
+ * tensor-core operations finish, tensor memory is freed) and returns.
+ *   wait_cycles > 0   the limit of the waits of the tensor-core attention and
+ *                     feed-forward kernels for the calls that follow; 0
+ *                     restores the default;
+ *   hold_tile >= 0    in the calls that follow, the tensor-core attention
+ *                     kernel's producers stop before tile `hold_tile` of each
+ *                     thread block, so the waits for that tile's data run out
+ *                     (their outputs are then undefined); -1 restores normal
+ *                     operation.
+ * The setting is process-wide and not synchronised with calls on other host
+ * threads.  LSH_ERR_INVALID_ARG for wait_cycles < 0. */
+LSH_API lsh_status lsh_set_wait_test(int32_t hold_tile, int64_t wait_cycles);
 
 /* Synchronises `stream`, returns the first error a kernel recorded since the
  * last call (LSH_OK if none) and clears it.  LSH_ERR_CUDA if the

@@ -6,7 +6,7 @@ ctypes binding and :mod:`lsh_attention_long_b200.workloads` draws the seeded
 synthetic inputs.
 """
 
-from .lsh import (LshError, Shape, forward_host_workspace, load_library,  # noqa: F401
-                  lsh_attend_bwd, lsh_attend_fwd, lsh_combine, lsh_device_status, lsh_forward,
-                  lsh_forward_host, lsh_hash, lsh_sort, lsh_workspace_size, make_shape,
-                  workspace)
+from .lsh import (LshError, Shape, ffn_workspace, forward_host_workspace,  # noqa: F401
+                  load_library, lsh_attend_bwd, lsh_attend_fwd, lsh_combine, lsh_device_status,
+                  lsh_ffn_forward, lsh_forward, lsh_forward_host, lsh_hash, lsh_set_wait_test,
+                  lsh_sort, lsh_workspace_size, make_shape, workspace)

@@ -217,33 +217,6 @@ attend_fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V,
   }
 }
 
-// Step 5 alone: one thread per (token, 8-wide slice of d).
-template <typename T>
-__global__ void combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_r,
-                               int n_rounds, size_t n_tok, T* __restrict__ O,
-                               float* __restrict__ lse) {
-  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= n_tok * 8) return;
-  const size_t tok = g >> 3;
-  const int k = (int)(g & 7) * 8;
-  float mx = -INFINITY;
-  for (int r = 0; r < n_rounds; ++r) mx = fmaxf(mx, lse_r[(size_t)r * n_tok + tok]);
-  float z = 0.f;
-  for (int r = 0; r < n_rounds; ++r) z += expf(lse_r[(size_t)r * n_tok + tok] - mx);
-  const float rz = 1.f / z;
-  const float tot = mx + logf(z);
-  float o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int r = 0; r < n_rounds; ++r) {
-    const float w = expf(lse_r[(size_t)r * n_tok + tok] - mx) * rz;
-    float t8[8];
-    load8(o_part + ((size_t)r * n_tok + tok) * kHeadDim + k, t8);
-#pragma unroll
-    for (int x = 0; x < 8; ++x) o[x] = fmaf(w, t8[x], o[x]);
-  }
-  store8(O + tok * kHeadDim + k, o);
-  if (lse && k == 0) lse[tok] = tot;
-}
-
 // ---------------------------------------------------------------------------
 // Backward (buckets and permutations constant).
 //

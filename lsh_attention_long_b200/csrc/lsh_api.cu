@@ -12,6 +12,7 @@
 #include "attend_simt.cuh"
 #include "attend_tc.cuh"
 #include "common.cuh"
+#include "ffn_tc.cuh"
 #include "hash_simt.cuh"
 #include "hash_tc.cuh"
 #include "sort.cuh"
@@ -78,24 +79,20 @@ lsh_status allow_smem(K kernel, size_t bytes) {
 // Tensor-core attention: bf16, d = 64, chunk = 64.
 bool attend_tc_supported(const Dims& D) { return D.dtype == LSH_BF16 && D.c == 64; }
 
-size_t counters_bytes(const Dims& D) {
-  return align_up(((size_t)D.B * D.H * D.R + 1) * sizeof(unsigned));
-}
-
 // Workspace of one lsh_attend_fwd call, given which optional outputs the
 // caller supplies.
 size_t attend_fwd_ws_bytes(const Dims& D, bool has_o_part, bool has_lse_r, bool has_O) {
   if (attend_tc_supported(D)) {
-    // counters, per-token key scale, then the running state or the partials
-    const size_t base = counters_bytes(D) + align_up(D.n_tok * sizeof(float));
-    if (has_O && !has_o_part && !has_lse_r) {  // online combine: running states per token
-      const size_t nbuf = D.R > 1 ? 2 : 1;     // even and odd rounds
-      return base + align_up(nbuf * D.n_tok * kHeadDim * sizeof(float)) +
-             align_up(nbuf * D.n_tok * sizeof(float4));
-    }
-    const size_t all = (size_t)D.R * D.n_tok;  // every round's partials
-    return base + (has_o_part ? 0 : align_up(all * kHeadDim * sizeof(float))) +
-           (has_lse_r ? 0 : align_up(all * sizeof(float)));
+    // per-token key scales and fp16 values, then per-round partials the
+    // caller does not take: fp16 outputs and fp32 logsumexps when the rounds
+    // are combined here, none for a single combined round (written as O
+    // directly)
+    size_t b = align_up(D.n_tok * sizeof(float)) + align_up(D.n_tok * kHeadDim * sizeof(__half));
+    if (has_O && !has_o_part && D.R == 1) return b;
+    const size_t all = (size_t)D.R * D.n_tok;
+    if (has_O && !has_o_part) b += align_up(all * kHeadDim * sizeof(__half));
+    if (!has_lse_r) b += align_up(all * sizeof(float));
+    return b;
   }
   if (!has_O) return 0;
   const size_t prev = (size_t)(D.R - 1) * D.n_tok;
@@ -201,7 +198,11 @@ lsh_status sort_launch(const Dims& D, const uint32_t* keys, int32_t* perm, cudaS
   const int by_len = (D.L / P + 127) / 128;  // at least 4 steps of 32 per warp
   nwarps = nwarps > by_len ? by_len : nwarps;
   if (nwarps < 1) nwarps = 1;
-  const size_t smem = (size_t)(nwarps + (P > 1 ? 1 : 0)) * hist;
+  size_t smem = (size_t)(nwarps + (P > 1 ? 1 : 0)) * hist;
+  // this CTA's bucket ids (u16), so that pass 2 reads no keys, when they fit
+  const size_t part = ((((size_t)D.L + P - 1) / P) + 31) & ~(size_t)31;
+  const int cache_ids = smem + part * 2 <= 220 * 1024 ? 1 : 0;
+  if (cache_ids) smem += part * 2;
   lsh_status st0 = allow_smem(lsh::sort_rows_kernel, smem);
   if (st0 != LSH_OK) return st0;
   cudaLaunchConfig_t cfg = {};
@@ -216,15 +217,20 @@ lsh_status sort_launch(const Dims& D, const uint32_t* keys, int32_t* perm, cudaS
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lsh::sort_rows_kernel, keys, perm, D.L, D.nb) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, lsh::sort_rows_kernel, keys, perm, D.L, D.nb,
+                         lsh::make_divl((uint32_t)D.L), cache_ids) != cudaSuccess)
     return LSH_ERR_CUDA;
   return last_launch();
 }
 
+// Test hook state (lsh_set_wait_test): the wait limit of the tensor-core
+// attention kernel and the tile its producers withhold.
+long long g_wait_limit = lsh::tc::kSpinCycles;
+int g_hold_tile = -1;
+
 lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const uint32_t* keys,
                             const int32_t* perm, float* o_part, float* lse_r, void* O,
                             float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
-  const bool online = O && !o_part && !lse_r;
   if (ws_bytes < attend_fwd_ws_bytes(D, o_part != nullptr, lse_r != nullptr, O != nullptr) ||
       !ws)
     return LSH_ERR_WORKSPACE;
@@ -241,43 +247,41 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   a.n_tiles = (a.n_chunks + 1) / 2;
   a.tpi = a.n_tiles < 4 ? a.n_tiles : 4;
   a.ipr = (a.n_tiles + a.tpi - 1) / a.tpi;
-  // heads whose running states and q, v rows share L2 while their rounds
-  // run: enough items between dependent rounds to cover one wave of CTAs
-  const size_t nbuf = D.R > 1 ? 2 : 1;
-  const size_t per_head = (size_t)D.L * (nbuf * (kHeadDim * 4 + 16) + 2 * kHeadDim * 2);
+  // items head by head, every round of a head before the next head: tiles
+  // do not depend on one another, so the CTAs in flight share one or a few
+  // heads' q and v rows, which stay in L2 across the rounds
   const int sms = num_sms();
-  long long hpb = (long long)((112ull << 20) / per_head);
-  const long long want = (2LL * sms + a.ipr - 1) / a.ipr;
-  if (hpb > want) hpb = want;
-  if (hpb < 1) hpb = 1;
-  if (hpb > a.BH) hpb = a.BH;
-  a.heads_per_block = (int)hpb;
+  a.heads_per_block = 1;
   a.n_items = (long long)a.R * a.BH * a.ipr;
-  a.online = online ? 1 : 0;
+  a.wait_limit = g_wait_limit;
+  a.hold_tile = g_hold_tile;
   char* w = static_cast<char*>(ws);
-  a.counters = reinterpret_cast<unsigned*>(w);
-  w += counters_bytes(D);
   float* rn = reinterpret_cast<float*>(w);
   a.rn = rn;
   w += align_up(D.n_tok * sizeof(float));
-  a.acc_o = nullptr;
-  a.acc_ml = nullptr;
-  a.o_part = o_part;
+  __half* v16 = reinterpret_cast<__half*>(w);
+  a.V16 = v16;
+  w += align_up(D.n_tok * kHeadDim * sizeof(__half));
+  a.o16 = nullptr;
+  a.o32 = o_part;
   a.lse_r = lse_r;
-  if (online) {
-    a.acc_o = reinterpret_cast<float*>(w);
-    w += align_up(nbuf * D.n_tok * kHeadDim * sizeof(float));
-    a.acc_ml = reinterpret_cast<float4*>(w);
+  a.O = nullptr;
+  a.lse = nullptr;
+  const size_t all = (size_t)D.R * D.n_tok;
+  if (O && !o_part && D.R == 1) {  // one round: O and lse directly
+    a.mode = lsh::kAtDirect;
+    a.O = static_cast<__nv_bfloat16*>(O);
+    a.lse = lse;
   } else {
-    const size_t all = (size_t)D.R * D.n_tok;
-    if (!a.o_part) {
-      a.o_part = reinterpret_cast<float*>(w);
-      w += align_up(all * kHeadDim * sizeof(float));
+    a.mode = o_part ? lsh::kAtPartial32 : lsh::kAtPartial16;
+    if (!o_part) {
+      a.o16 = reinterpret_cast<__half*>(w);
+      w += align_up(all * kHeadDim * sizeof(__half));
     }
     if (!a.lse_r) a.lse_r = reinterpret_cast<float*>(w);
   }
-  if (cudaMemsetAsync(a.counters, 0, counters_bytes(D), st) != cudaSuccess) return LSH_ERR_CUDA;
-  lsh::key_scale_kernel<<<(unsigned)((D.n_tok + 255) / 256), 256, 0, st>>>(a.Q, D.n_tok, rn);
+  lsh::fwd_prep_kernel<<<(unsigned)((D.n_tok * 8 + 255) / 256), 256, 0, st>>>(
+      a.Q, a.V, D.n_tok, rn, v16);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
   const size_t smem = lsh::attend_tc_smem_bytes();
   lsh_status s0 = allow_smem(lsh::attend_tc_kernel, smem);
@@ -285,15 +289,14 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   const long long grid = a.n_items < sms ? a.n_items : sms;
   lsh::attend_tc_kernel<<<(unsigned)grid, lsh::kAtThreads, smem, st>>>(a);
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  const size_t n8 = D.n_tok * 8;
-  if (online) {
-    lsh::online_merge_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
-        a.acc_o, a.acc_ml, (int)nbuf, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
-    return last_launch();
-  }
-  if (O) {
-    lsh::combine_kernel<__nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
-        a.o_part, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
+  if (O && a.mode != lsh::kAtDirect) {
+    const size_t n8 = D.n_tok * 8;
+    if (a.mode == lsh::kAtPartial16)
+      lsh::combine_kernel<__half, __nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
+          a.o16, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
+    else
+      lsh::combine_kernel<float, __nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
+          a.o32, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
     return last_launch();
   }
   return LSH_OK;
@@ -345,8 +348,8 @@ lsh_status combine_launch(const Dims& D, const float* o_part, const float* lse_r
                           float* lse, cudaStream_t st) {
   const size_t n = D.n_tok * 8;
   const unsigned blocks = (unsigned)((n + 255) / 256);
-  lsh::combine_kernel<T><<<blocks, 256, 0, st>>>(o_part, lse_r, D.R, D.n_tok,
-                                                 static_cast<T*>(O), lse);
+  lsh::combine_kernel<float, T><<<blocks, 256, 0, st>>>(o_part, lse_r, D.R, D.n_tok,
+                                                        static_cast<T*>(O), lse);
   return last_launch();
 }
 
@@ -742,6 +745,124 @@ lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const vo
                                                 scratch, LSH_STATIC_SCRATCH_BYTES, st)
              : attend_fwd_launch<float>(D, Q, V, keys, perm, nullptr, nullptr, O, lse, scratch,
                                         LSH_STATIC_SCRATCH_BYTES, st);
+}
+
+// ---------------------------------------------------------------------------
+// Chunked feed-forward
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// cuTensorMapEncodeTiled, reached through the runtime so that the library
+// does not link the driver library itself.
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiled fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x box_rows
+// rows, 128-byte swizzled (the K-major operand layout of the MMA).
+bool bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  const EncodeTiled f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t elem[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+lsh_status ffn_check(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk) {
+  if (tokens < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return LSH_ERR_INVALID_ARG;
+  if (d_model % lsh::kGmBN || d_ff % lsh::kGmBN || tokens % lsh::kGmBM || chunk % lsh::kGmBM)
+    return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)tokens * d_model >= (int64_t(1) << 31) ||
+      (int64_t)chunk * d_ff >= (int64_t(1) << 31))
+    return LSH_ERR_UNSUPPORTED;
+  return LSH_OK;
+}
+
+lsh_status gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const lsh::GemmArgs& g,
+                       cudaStream_t st) {
+  const size_t smem = lsh::gemm_tc_smem_bytes();
+  lsh_status s0 = allow_smem(lsh::gemm_tc_kernel, smem);
+  if (s0 != LSH_OK) return s0;
+  const int tiles = (g.M / lsh::kGmBM) * (g.N / lsh::kGmBN);
+  const int sms = num_sms();
+  lsh::gemm_tc_kernel<<<(unsigned)(tiles < sms ? tiles : sms), lsh::kGmThreads, smem, st>>>(ma, mb,
+                                                                                          g);
+  return last_launch();
+}
+
+}  // namespace
+
+size_t lsh_ffn_ws_size(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk) {
+  if (ffn_check(tokens, d_model, d_ff, chunk) != LSH_OK || tokens == 0) return 0;
+  return align_up((size_t)chunk * d_ff * sizeof(__nv_bfloat16));
+}
+
+lsh_status lsh_ffn_forward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk,
+                           const void* X, const void* W1, const void* b1, const void* W2,
+                           const void* b2, void* Y, void* ws, size_t ws_bytes, void* stream) {
+  lsh_status s = ffn_check(tokens, d_model, d_ff, chunk);
+  if (s != LSH_OK) return s;
+  if (tokens == 0) return LSH_OK;
+  if (!X || !W1 || !b1 || !W2 || !b2 || !Y || !ws) return LSH_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(W1) || misaligned(b1) || misaligned(W2) || misaligned(b2) ||
+      misaligned(Y) || misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  if (ws_bytes < (size_t)chunk * d_ff * sizeof(__nv_bfloat16)) return LSH_ERR_WORKSPACE;
+  CUtensorMap mx, mw1, mh, mw2;
+  if (!bf16_map(&mx, X, (uint64_t)tokens, (uint64_t)d_model, lsh::kGmBM) ||
+      !bf16_map(&mw1, W1, (uint64_t)d_ff, (uint64_t)d_model, lsh::kGmBN) ||
+      !bf16_map(&mh, ws, (uint64_t)chunk, (uint64_t)d_ff, lsh::kGmBM) ||
+      !bf16_map(&mw2, W2, (uint64_t)d_model, (uint64_t)d_ff, lsh::kGmBN))
+    return LSH_ERR_CUDA;
+  cudaStream_t st = as_stream(stream);
+  __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
+  for (int c0 = 0; c0 < tokens; c0 += chunk) {
+    const int n = tokens - c0 < chunk ? tokens - c0 : chunk;
+    // H = max(0, X[c0 : c0+n] W1^T + b1): the chunk's hidden activation
+    lsh::GemmArgs g1;
+    g1.M = n; g1.N = d_ff; g1.K = d_model; g1.a_row0 = c0;
+    g1.bias = static_cast<const __nv_bfloat16*>(b1);
+    g1.C = H; g1.ldc = d_ff; g1.relu = 1; g1.wait_limit = g_wait_limit;
+    s = gemm_launch(mx, mw1, g1, st);
+    if (s != LSH_OK) return s;
+    // Y[c0 : c0+n] = H W2^T + b2
+    lsh::GemmArgs g2;
+    g2.M = n; g2.N = d_model; g2.K = d_ff; g2.a_row0 = 0;
+    g2.bias = static_cast<const __nv_bfloat16*>(b2);
+    g2.C = static_cast<__nv_bfloat16*>(Y) + (size_t)c0 * d_model; g2.ldc = d_model; g2.relu = 0;
+    g2.wait_limit = g_wait_limit;
+    s = gemm_launch(mh, mw2, g2, st);
+    if (s != LSH_OK) return s;
+  }
+  return LSH_OK;
+}
+
+lsh_status lsh_set_wait_test(int32_t hold_tile, int64_t wait_cycles) {
+  if (wait_cycles < 0) return LSH_ERR_INVALID_ARG;
+  g_wait_limit = wait_cycles > 0 ? (long long)wait_cycles : lsh::tc::kSpinCycles;
+  g_hold_tile = hold_tile >= 0 ? hold_tile : -1;
+  return LSH_OK;
 }
 
 lsh_status lsh_device_status(void* stream) {

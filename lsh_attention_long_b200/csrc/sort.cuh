@@ -7,15 +7,18 @@
 //
 // A row is sorted by one thread-block cluster of P CTAs (P = 1 or 2), CTA c
 // taking the c-th part of the row.  Each warp owns a contiguous segment and a
-// private histogram in shared memory, so counting needs no atomics:
-//   pass 1  per 32-token step, __match_any_sync groups equal buckets and the
-//           group leader adds the group size to the warp's histogram;
+// private histogram in shared memory:
+//   pass 1  every key's bucket (key / L by a multiply-high with a
+//           precomputed constant) is counted into the warp's histogram with a
+//           shared-memory atomic (counts do not depend on order) and, when
+//           the CTA's part fits, kept in shared memory as 16 bits;
 //   scan    per-bucket totals of every CTA of the cluster meet through
 //           distributed shared memory; bucket-major, CTA-minor, warp-minor
 //           exclusive prefix sums give each warp's first output slot per
 //           bucket;
-//   pass 2  the same walk again; a token's slot is its warp's offset for the
-//           bucket plus its rank among equal-bucket lanes of lower index.
+//   pass 2  the same walk again over the kept bucket ids (or the keys); a
+//           token's slot is its warp's offset for the bucket plus its rank
+//           among equal-bucket lanes of lower index (__match_any_sync).
 // CTAs, warps, steps and lanes visit positions in increasing order, so equal
 // buckets keep position order: the sort is stable.
 #pragma once
@@ -28,10 +31,31 @@ namespace lsh {
 
 constexpr uint32_t kNoBucket = 0xffffffffu;
 
+// floor(key / L) for key < 2^31 as umulhi(key, m) >> sh, with
+// m = ceil(2^(31 + l) / L), l = ceil(log2 L), sh = l - 1 (the round-up
+// method of division by an invariant integer); L == 1 is the identity.
+struct DivL {
+  uint32_t m;
+  int sh;  // -1: L == 1
+};
+__host__ inline DivL make_divl(uint32_t L) {
+  DivL d;
+  int l = 0;
+  while ((1ull << l) < L) ++l;
+  if (l == 0) { d.m = 0; d.sh = -1; return d; }
+  const unsigned __int128 num = (unsigned __int128)1 << (31 + l);
+  d.m = (uint32_t)((num + L - 1) / L);
+  d.sh = l - 1;
+  return d;
+}
+__device__ __forceinline__ uint32_t div_l(uint32_t key, DivL d) {
+  return d.sh < 0 ? key : __umulhi(key, d.m) >> d.sh;
+}
+
 __device__ __forceinline__ uint32_t checked_bucket(const uint32_t* k, int t, int L, int nb,
-                                                   bool& bad) {
+                                                   DivL dl, bool& bad) {
   const uint32_t key = k[t];
-  const uint32_t b = key / (uint32_t)L;
+  const uint32_t b = div_l(key, dl);
   if (b >= (uint32_t)nb || key - b * (uint32_t)L != (uint32_t)t) {
     bad = true;
     return kNoBucket;
@@ -40,9 +64,10 @@ __device__ __forceinline__ uint32_t checked_bucket(const uint32_t* k, int t, int
 }
 
 __global__ void __launch_bounds__(1024)
-sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, int L, int nb) {
+sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, int L, int nb,
+                 DivL dl, int cache_ids) {
   namespace cg = cooperative_groups;
-  extern __shared__ uint32_t cnt[];  // [nwarps][nb], then (P > 1) this CTA's totals [nb]
+  extern __shared__ uint32_t cnt[];  // [nwarps][nb], (P > 1) this CTA's totals [nb], ids
   __shared__ uint32_t warp_sums[32];
   cg::cluster_group cluster = cg::this_cluster();
   const int P = (int)cluster.num_blocks(), crank = (int)cluster.block_rank();
@@ -52,6 +77,7 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   const uint32_t* k = keys + row * L;
   int32_t* out = perm + row * L;
   uint32_t* tot = cnt + (size_t)nwarps * nb;
+  uint16_t* ids = reinterpret_cast<uint16_t*>(tot + (P > 1 ? nb : 0));  // this CTA's bucket ids
 
   for (int e = threadIdx.x; e < nwarps * nb; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -64,12 +90,15 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   uint32_t* my = cnt + (size_t)w * nb;
   bool bad = false;
 
-  // pass 1: per-warp histograms
+  // pass 1: per-warp histograms (counts do not depend on order: shared-
+  // memory atomics), bucket ids kept for pass 2 when they fit
   for (int base = begin; base < end; base += 32) {
     const int t = base + lane;
-    const uint32_t b = (t < end) ? checked_bucket(k, t, L, nb, bad) : kNoBucket;
-    const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    if (b != kNoBucket && lane == __ffs(peers) - 1) my[b] += __popc(peers);
+    if (t < end) {
+      const uint32_t b = checked_bucket(k, t, L, nb, dl, bad);
+      if (b != kNoBucket) atomicAdd(&my[b], 1u);
+      if (cache_ids) ids[t - cbeg] = b != kNoBucket ? (uint16_t)b : (uint16_t)0xffffu;
+    }
   }
   if (bad) record_status(kErrBadKeys);
   __syncthreads();
@@ -140,7 +169,15 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   for (int base = begin; base < end; base += 32) {
     const int t = base + lane;
     bool dummy = false;
-    const uint32_t b = (t < end) ? checked_bucket(k, t, L, nb, dummy) : kNoBucket;
+    uint32_t b = kNoBucket;
+    if (t < end) {
+      if (cache_ids) {
+        const uint32_t c = ids[t - cbeg];
+        b = c == 0xffffu ? kNoBucket : c;
+      } else {
+        b = checked_bucket(k, t, L, nb, dl, dummy);
+      }
+    }
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     if (b != kNoBucket) {
       const uint32_t rank = __popc(peers & ((1u << lane) - 1u));

@@ -209,6 +209,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | ((uint32_t)(M >> 4) << 24);     // M / 16
 }
 
+// Instruction descriptor of kind::f16 with fp16 A and B, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                         // D format: f32 (A, B format 0: f16)
+         | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)      // N / 8
+         | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle.
 //   K-major tile: rows of 128 B (64 bf16 along K), 8-row groups `sbo` apart.
 //   MN-major tile: rows of 128 B along MN indexed by K, 8-row groups `sbo`

@@ -25,7 +25,8 @@ STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "L
 
 EXPORTS = ("lsh_workspace_size", "lsh_hash", "lsh_sort", "lsh_attend_fwd", "lsh_combine",
            "lsh_forward", "lsh_forward_host", "lsh_forward_host_ws_size", "lsh_attend_bwd",
-           "lsh_device_status", "lsh_status_string")
+           "lsh_device_status", "lsh_status_string", "lsh_attend_fwd_static", "lsh_set_wait_test",
+           "lsh_ffn_ws_size", "lsh_ffn_forward")
 
 
 class LshError(RuntimeError):
@@ -64,6 +65,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsh_forward_host": ([S, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "lsh_attend_bwd": ([S, P, P, P, P, P, P, P, P, P, P, sz, P], ctypes.c_int),
         "lsh_device_status": ([P], ctypes.c_int),
+        "lsh_attend_fwd_static": ([S, P, P, P, P, P, P, P], ctypes.c_int),
+        "lsh_set_wait_test": ([ctypes.c_int32, ctypes.c_int64], ctypes.c_int),
+        "lsh_ffn_ws_size": ([ctypes.c_int32] * 4, sz),
+        "lsh_ffn_forward": ([ctypes.c_int32] * 4 + [P] * 7 + [sz, P], ctypes.c_int),
         "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -329,6 +334,41 @@ def lsh_attend_bwd(Q, V, O, dO, keys, perm, lse, n_buckets: int, chunk: int, cau
           _ptr(keys), _ptr(perm), _ptr(lse), _ptr(dQ), _ptr(dV), _ptr(ws), ws.numel(),
           _stream(stream))
     return dQ, dV
+
+
+def ffn_workspace(tokens: int, d_model: int, d_ff: int, chunk: int, device) -> torch.Tensor:
+    """Device scratch for lsh_ffn_forward: one chunk's hidden activation."""
+    n = load_library().lsh_ffn_ws_size(tokens, d_model, d_ff, chunk)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def lsh_ffn_forward(X, W1, b1, W2, b2, chunk: int, *, Y=None, ws=None, stream=None):
+    """Chunked feed-forward: Y = W2 max(0, W1 x + b1) + b2 per position of X
+    [..., d_model] (bf16), `chunk` positions at a time."""
+    if not isinstance(X, torch.Tensor) or X.dim() < 2:
+        raise ValueError("X must be a [..., d_model] tensor")
+    d_model = X.shape[-1]
+    tokens = X.numel() // d_model if d_model else 0
+    d_ff = W1.shape[0] if isinstance(W1, torch.Tensor) and W1.dim() == 2 else -1
+    bf = torch.bfloat16
+    _validate([("X", X, None, bf, True), ("W1", W1, (d_ff, d_model), bf, True),
+               ("b1", b1, (d_ff,), bf, True), ("W2", W2, (d_model, d_ff), bf, True),
+               ("b2", b2, (d_model,), bf, True), ("Y", Y, X.shape, bf, True),
+               ("ws", ws, None, None, True)])
+    if Y is None:
+        Y = torch.empty_like(X)
+    if ws is None:
+        ws = ffn_workspace(tokens, d_model, d_ff, chunk, X.device)
+    _call("lsh_ffn_forward", tokens, d_model, d_ff, chunk, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2),
+          _ptr(b2), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream))
+    return Y
+
+
+def lsh_set_wait_test(hold_tile: int = -1, wait_cycles: int = 0) -> None:
+    """Test hook of the bounded device waits (see include/lsh.h): a clock-cycle
+    limit for the tensor-core attention kernel's waits (0 = default) and a tile
+    its producers withhold (-1 = none).  Process-wide."""
+    _call("lsh_set_wait_test", int(hold_tile), int(wait_cycles))
 
 
 def lsh_device_status(stream=None) -> int:

@@ -129,3 +129,47 @@ def make_random(B: int, H: int, L: int, d: int, n_buckets: int, n_rounds: int,
     if backward:
         out["dO"] = gaussian(shape, 0, dtype, generator=g)
     return out
+
+
+# ---------------------------------------------------------------------------
+# chunked feed-forward (the companion op of LSH attention in a Reformer layer)
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class FfnWorkload:
+    name: str
+    tokens: int   # B * L positions
+    d_model: int  # H * d: 8 heads of 64
+    d_ff: int     # 4 * d_model
+    chunk: int    # positions per chunk
+
+    def describe(self) -> dict:
+        return dataclasses.asdict(self)
+
+
+# ``ffn_bf16_L65536``: the L=65536 sequence of one batch element through the
+# feed-forward of width 512 (8 heads of 64) and hidden width 2048, 8192
+# positions per chunk.
+FFN_WORKLOADS: Dict[str, FfnWorkload] = {
+    w.name: w for w in [FfnWorkload("ffn_bf16_L65536", 65536, 512, 2048, 8192)]
+}
+
+
+def ffn_inputs(tokens: int, d_model: int, d_ff: int, seed: int = 20,
+               dtype: torch.dtype = torch.bfloat16, backward: bool = False):
+    """Seeded feed-forward inputs: X ~ N(0, 1) [tokens, d_model] (seed),
+    W1 ~ N(0, 1/d_model) [d_ff, d_model] (seed + 1), b1 ~ N(0, 0.1^2) (seed + 2),
+    W2 ~ N(0, 1/d_ff) [d_model, d_ff] (seed + 3), b2 ~ N(0, 0.1^2) (seed + 4),
+    drawn in fp32 and rounded once to dtype; with backward, dY ~ N(0, 1)
+    (seed + 5).  The weight scales keep every pre-activation and output near
+    unit variance."""
+    def draw(shape, s, scale):
+        return (torch.randn(*shape, generator=_gen(s), dtype=torch.float32) * scale).to(dtype)
+    out = {"X": draw((tokens, d_model), seed, 1.0),
+           "W1": draw((d_ff, d_model), seed + 1, d_model ** -0.5),
+           "b1": draw((d_ff,), seed + 2, 0.1),
+           "W2": draw((d_model, d_ff), seed + 3, d_ff ** -0.5),
+           "b2": draw((d_model,), seed + 4, 0.1)}
+    if backward:
+        out["dY"] = draw((tokens, d_model), seed + 5, 1.0)
+    return out

@@ -1,0 +1,87 @@
+"""GPU parity of the chunked feed-forward (lsh_ffn_forward) against the fp64 oracle.
+
+Y = W2 max(0, W1 x + b1) + b2 per position, `chunk` positions at a time
+("Reformer explainer", single section; "Reformer Language Models (Korean)",
+Reformer overview).  bf16 inputs with fp32 accumulation: max-abs 2e-2.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import lsh_attention_long_b200 as L
+from lsh_attention_long_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from lsh_attention_long_b200 import build
+    build.build()
+    L.load_library()
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def _run(inp, chunk):
+    t = {k: v.cuda() for k, v in inp.items()}
+    Y = L.lsh_ffn_forward(t["X"], t["W1"], t["b1"], t["W2"], t["b2"], chunk)
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
+    return Y
+
+
+@pytest.mark.parametrize("tokens,d_model,d_ff,chunk", [
+    (128, 256, 256, 128),     # one tile, one chunk
+    (512, 256, 512, 128),     # four chunks
+    (1024, 512, 2048, 384),   # chunks of 384, 384, 256 (a ragged last chunk)
+    (640, 768, 1024, 640),    # five token tiles, three output tiles
+])
+def test_ffn_matches_the_oracle(oracle, tokens, d_model, d_ff, chunk):
+    inp = W.ffn_inputs(tokens, d_model, d_ff, seed=tokens + d_ff)
+    Y = _run(inp, chunk)
+    ref = oracle.ffn_forward(*(_np(inp[k]) for k in ("X", "W1", "b1", "W2", "b2")), chunk)
+    np.testing.assert_allclose(_np(Y), ref, rtol=0, atol=TOL)
+
+
+def test_chunking_does_not_change_the_device_result():
+    """Every output row is computed by the same tiles whatever the chunk, so
+    the result is bit-identical across chunk sizes."""
+    inp = W.ffn_inputs(1024, 512, 2048, seed=3)
+    Y1 = _run(inp, 128)
+    Y2 = _run(inp, 1024)
+    assert torch.equal(Y1, Y2)
+
+
+def test_ffn_workload_at_full_size(oracle, parity_record):
+    """The benchmarked workload (65 536 positions, 512 -> 2048 -> 512, chunks
+    of 8192): 512 sampled positions, spread over every chunk, against the
+    oracle."""
+    w = W.FFN_WORKLOADS["ffn_bf16_L65536"]
+    inp = W.ffn_inputs(w.tokens, w.d_model, w.d_ff)
+    Y = _run(inp, w.chunk)
+    rows = np.random.default_rng(0).choice(w.tokens, 512, replace=False)
+    ref = oracle.ffn_forward(_np(inp["X"])[rows], *(_np(inp[k]) for k in ("W1", "b1", "W2", "b2")),
+                             128)
+    err = float(np.abs(_np(Y)[rows] - ref).max())
+    parity_record.append({"workload": w.name, "positions_checked": len(rows), "max_abs": {"Y": err},
+                          "tol": TOL})
+    assert err <= TOL
+
+
+def test_ffn_rejects_unsupported_shapes_and_empty_input_is_a_no_op():
+    inp = W.ffn_inputs(128, 256, 256, seed=1)
+    t = {k: v.cuda() for k, v in inp.items()}
+    with pytest.raises(L.LshError):  # chunk not a multiple of 128
+        L.lsh_ffn_forward(t["X"], t["W1"], t["b1"], t["W2"], t["b2"], 100)
+    empty = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    Y = L.lsh_ffn_forward(empty, t["W1"], t["b1"], t["W2"], t["b2"], 128)
+    assert Y.numel() == 0
+    assert L.lsh_device_status() == 0

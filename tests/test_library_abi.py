@@ -118,10 +118,16 @@ def test_empty_shapes_are_no_ops(lib):
 
 
 def test_workspace_size_covers_partials_and_gradients(lib):
-    s = _shape(B=2, H=8, L=16384, n_buckets=256, n_rounds=4)
     n_tok = 2 * 8 * 16384
-    fwd = 3 * n_tok * 65 * 4
     bwd = n_tok * 4 + 3 * n_tok * 64 * 4
+    # tensor-core path (bf16, chunk 64): key scales, fp16 values and every
+    # round's fp16 output and fp32 logsumexp
+    s = _shape(B=2, H=8, L=16384, n_buckets=256, n_rounds=4)
+    fwd = n_tok * 4 + n_tok * 128 + 4 * n_tok * (64 * 2 + 4)
+    assert lib.lsh_workspace_size(ctypes.byref(s)) >= max(fwd, bwd)
+    # CUDA-core path (f32): fp32 partials of the first R-1 rounds
+    s = _shape(B=2, H=8, L=16384, n_buckets=256, n_rounds=4, dtype=0)
+    fwd = 3 * n_tok * 65 * 4
     assert lib.lsh_workspace_size(ctypes.byref(s)) >= max(fwd, bwd)
 
 
@@ -140,18 +146,27 @@ def _align(x):
     return (x + 255) // 256 * 256
 
 
+def _tc_need(n, R):
+    """Tensor-core path: key scales and fp16 values, then (R > 1) every
+    round's fp16 output and fp32 logsumexp."""
+    base = _align(n * 4) + _align(n * 128)
+    return base if R == 1 else base + _align(R * n * 128) + _align(R * n * 4)
+
+
 @pytest.mark.parametrize("Lx,R,chunk,dtype,need", [
-    # tensor-core path (bf16, chunk 64), one round: counters, key scales, one
-    # running state of 256 + 16 B per token
-    (243136, 1, 64, 1, _align(8) + _align(243136 * 4) + _align(243136 * 272)),
-    (243200, 1, 64, 1, _align(8) + _align(243200 * 4) + _align(243200 * 272)),
+    # tensor-core path (bf16, chunk 64), two rounds, either side of 64 MiB
+    (169408, 2, 64, 1, _tc_need(169408, 2)),
+    (169472, 2, 64, 1, _tc_need(169472, 2)),
+    # one round: only the key scales and fp16 values
+    (508352, 1, 64, 1, _tc_need(508352, 1)),
+    (508416, 1, 64, 1, _tc_need(508416, 1)),
     # CUDA-core path (f32), two rounds: one round of fp32 partials (256 + 4 B)
     (258048, 2, 64, 0, _align(258048 * 256) + _align(258048 * 4)),
     (258112, 2, 64, 0, _align(258112 * 256) + _align(258112 * 4)),
-    # the same L=16384 x 8 heads, R=2 problem on each path: 71 MB on the
-    # tensor-core path, 34 MB on the CUDA-core path (chunk 32)
-    (8 * 16384, 2, 64, 1, _align(3 * 4) + _align(131072 * 4) + _align(2 * 131072 * 272)),
-    (8 * 16384, 2, 32, 1, _align(131072 * 256) + _align(131072 * 4)),
+    # one problem (L=98304, R=4) on each path: 64.9 MB on the tensor-core
+    # path, 76.7 MB on the CUDA-core path (chunk 32)
+    (98304, 4, 64, 1, _tc_need(98304, 4)),
+    (98304, 4, 32, 1, _align(3 * 98304 * 256) + _align(3 * 98304 * 4)),
 ])
 def test_static_scratch_limit_follows_the_path(lib, Lx, R, chunk, dtype, need):
     """lsh_attend_fwd_static refuses exactly the problems whose need, on the
@@ -173,3 +188,19 @@ def test_static_scratch_limit_follows_the_path(lib, Lx, R, chunk, dtype, need):
         pytest.skip("an accepted problem would launch on these placeholder pointers")
     assert lib.lsh_attend_fwd_static(ctypes.byref(s), fake, fake, fake, fake, fake, None,
                                      None) == 3
+
+
+def test_ffn_checks_arguments_before_any_launch(lib):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every call below fails its checks first
+    args = [fake] * 6
+    assert lib.lsh_ffn_forward(128, 200, 512, 128, *args, fake, 1 << 20, None) == 2   # d_model % 256
+    assert lib.lsh_ffn_forward(100, 256, 512, 128, *args, fake, 1 << 20, None) == 2   # tokens % 128
+    assert lib.lsh_ffn_forward(128, 256, 512, 0, *args, fake, 1 << 20, None) == 1     # chunk
+    assert lib.lsh_ffn_forward(128, 256, 512, 128, None, *args[1:], fake, 1 << 20, None) == 1
+    assert lib.lsh_ffn_forward(128, 256, 512, 128, ctypes.c_void_p(264), *args[1:], fake,
+                               1 << 20, None) == 1                                    # misaligned
+    need = lib.lsh_ffn_ws_size(256, 256, 512, 128)
+    assert need >= 128 * 512 * 2
+    assert lib.lsh_ffn_forward(256, 256, 512, 128, *args, fake, need - 1, None) == 4  # workspace
+    assert lib.lsh_ffn_forward(0, 256, 512, 128, None, None, None, None, None, None, None, 0,
+                               None) == 0                                             # empty

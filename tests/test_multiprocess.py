@@ -77,3 +77,72 @@ def test_reference_arm_under_torchrun_prints_once(tmp_path):
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+# ---------------------------------------------------------------------------
+# one problem's heads split over the ranks (lsh_attention_long_b200.shard)
+# ---------------------------------------------------------------------------
+
+def test_head_ranges_cover_every_head_once():
+    from lsh_attention_long_b200.shard import head_range
+    for n in (0, 1, 7, 8, 16, 64, 65, 1000):
+        for world in (1, 2, 3, 4, 8, 13):
+            seen = []
+            sizes = []
+            for r in range(world):
+                h0, h1 = head_range(n, world, r)
+                assert 0 <= h0 <= h1 <= n
+                seen += list(range(h0, h1))
+                sizes.append(h1 - h0)
+            assert seen == list(range(n))           # contiguous, in order, once each
+            assert max(sizes) - min(sizes) <= 1      # balanced
+    with pytest.raises(ValueError):
+        head_range(8, 2, 2)
+
+
+def _oracle_forward(q, v, rot, nb, chunk, causal):
+    """The single-device forward for the CPU ranks: the fp64 oracle."""
+    import torch
+    from oracle import oracle as o
+    f = o.lsh_forward(q.double().numpy(), v.double().numpy(), rot.double().numpy(), nb, chunk,
+                      causal)
+    return {"O": torch.from_numpy(f["O"]), "lse": torch.from_numpy(f["lse"]),
+            "keys": torch.from_numpy(f["keys"].astype("int64")),
+            "perm": torch.from_numpy(f["perm"].astype("int64"))}
+
+
+def _shard_rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from lsh_attention_long_b200 import workloads as W
+    from lsh_attention_long_b200.shard import forward_sharded
+    dist.init_process_group("gloo")
+    inp = W.make_random(2, 3, 256, 64, 16, 2, torch.float32, seed=17)
+    out = forward_sharded(inp["Q"], inp["V"], inp["rot"], 16, 64, True, world, rank,
+                          forward=_oracle_forward, gather=True)
+    torch.save({"O_full": out["O_full"], "lse_full": out["lse_full"], "O": out["O"]},
+               os.path.join(out_dir, f"shard{rank}.pt"))
+    dist.destroy_process_group()
+
+
+def test_two_rank_head_shards_reassemble_the_one_rank_result(tmp_path, oracle):
+    """B*H = 6 heads over two gloo ranks (3 each): every rank's slice is its
+    heads' forward, and the all-gathered O and lse equal the one-rank result
+    on all heads, bit for bit (the oracle is deterministic per head)."""
+    import torch
+    from lsh_attention_long_b200 import workloads as W
+    world, port = 2, _free_port()
+    mp.start_processes(_shard_rank_main, args=(world, port, str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    inp = W.make_random(2, 3, 256, 64, 16, 2, torch.float32, seed=17)
+    ref = _oracle_forward(inp["Q"], inp["V"], inp["rot"], 16, 64, True)
+    got = [torch.load(tmp_path / f"shard{r}.pt") for r in range(world)]
+    for g in got:
+        assert torch.equal(g["O_full"], ref["O"])
+        assert torch.equal(g["lse_full"], ref["lse"])
+    flat = ref["O"].reshape(1, 6, 256, 64)
+    assert torch.equal(got[0]["O"], flat[:, 0:3])
+    assert torch.equal(got[1]["O"], flat[:, 3:6])

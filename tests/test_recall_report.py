@@ -107,3 +107,44 @@ def test_recall_is_a_share_of_the_mass(oracle):
                                       torch.arange(L), 0, 0).numpy()
     assert np.all(rec >= 0.0) and np.all(rec <= 1.0 + 1e-12)
     assert 0.0 < rec.mean() < 1.0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True])
+def test_attended_sets_on_the_device_match_brute_force(causal):
+    """The recall report as the bench runs it: keys and permutations from the
+    CUDA path (clustered queries, several chunks and rounds), the attended
+    sets computed from device tensors, against a brute-force enumeration of
+    the same keys and permutations on the host."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import lsh_attention_long_b200 as L
+    from lsh_attention_long_b200 import build
+    from lsh_attention_long_b200 import workloads as W
+    build.build()
+    L.load_library()
+    Lx, chunk, nb, R = 1024, 64, 16, 3
+    inp = W.make_random(1, 2, Lx, 64, nb, R, torch.bfloat16, seed=29)
+    Q, V, rot = (inp[k].cuda() for k in ("Q", "V", "rot"))
+    out = L.lsh_forward(Q, V, rot, nb, chunk, causal)
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
+    rows = torch.arange(0, Lx, 7, device="cuda")
+    got = bench.attended_mask(out["keys"].to(torch.int64), out["perm"].to(torch.int64), Lx,
+                              chunk, causal, rows, 0, 1).cpu().numpy()
+    keys = out["keys"].cpu().numpy().view(np.uint32)
+    perm = out["perm"].cpu().numpy()
+    nch = Lx // chunk
+    want = np.zeros_like(got)
+    for qi, i in enumerate(rows.tolist()):
+        for r in range(R):
+            k, p = keys[r, 0, 1], perm[r, 0, 1]
+            c = int(np.nonzero(p == i)[0][0]) // chunk
+            for cc in ([c] if nch == 1 else [(c - 1) % nch, c]):
+                for j in p[cc * chunk:(cc + 1) * chunk]:
+                    if j != i and k[j] // Lx == k[i] // Lx and not (causal and j > i):
+                        want[qi, j] = True
+    assert np.array_equal(got, want)
+    rec = bench.full_attention_recall(Q.float(), out["keys"].to(torch.int64),
+                                      out["perm"].to(torch.int64), chunk, causal, rows, 0, 1)
+    assert torch.all((rec >= 0) & (rec <= 1 + 1e-9))

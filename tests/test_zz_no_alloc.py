@@ -35,9 +35,10 @@ def static_need(B, H, Lx, R, chunk, dtype):
     """Scratch bytes the header documents for lsh_attend_fwd_static."""
     n = B * H * Lx
     if dtype == torch.bfloat16 and chunk == 64:  # tensor-core path
-        k = 2 if R > 1 else 1
-        return (_align((R * B * H + 1) * 4) + _align(n * 4) + _align(k * n * 256)
-                + _align(k * n * 16))
+        base = _align(n * 4) + _align(n * 64 * 2)  # key scales, fp16 values
+        if R == 1:
+            return base
+        return base + _align(R * n * 64 * 2) + _align(R * n * 4)
     if R == 1:  # CUDA-core path
         return 0
     return _align((R - 1) * n * 64 * 4) + _align((R - 1) * n * 4)
@@ -88,20 +89,22 @@ def _same_as_workspace_call(lib, B, H, Lx, nb, R, chunk, causal, dtype, seed):
 
 @pytest.mark.parametrize("dtype,chunk2", [(torch.bfloat16, 64), (torch.float32, 32)])
 def test_static_scratch_matches_workspace_entry_point(lib, dtype, chunk2):
-    """Two calls in a row on one path: a larger problem leaves its running
-    states (tensor-core path) or partials (CUDA-core path) in the shared
-    array, then a smaller one must not read any of them."""
+    """Two calls in a row on one path: a larger problem leaves its per-round
+    partials in the shared array, then a smaller one must not read any of
+    them."""
     _same_as_workspace_call(lib, 2, 4, 2048, 64, 4, 64, True, dtype, seed=11)
     _same_as_workspace_call(lib, 1, 3, 320, 16, 3, chunk2, False, dtype, seed=12)
 
 
 def test_static_scratch_capacity_follows_the_path(lib):
-    """B=1 H=8 L=16384 R=2: the tensor-core path (bf16, chunk 64) needs about
-    71 MB and is refused; the CUDA-core path (f32, or bf16 with chunk 32)
-    needs 34 MB and runs.  One round in bf16 needs 36 MB and runs; one round
-    at L=65536 needs 145 MB and is refused."""
+    """Problems that fit one path's formula but not the other's.  B=1 H=2
+    L=49152 R=4: the tensor-core path (bf16, chunk 64) needs 64.9 MB and runs,
+    the CUDA-core path (f32, or bf16 with chunk 32) needs 76.7 MB and is
+    refused.  B=1 H=1 L=254976 R=2: the CUDA-core path needs 66.3 MB and runs,
+    the tensor-core path needs 101 MB and is refused."""
     fake = ctypes.c_void_p(256)  # never dereferenced: the size check fails first
-    refused = [(1, 8, 16384, 2, 64, torch.bfloat16), (1, 8, 65536, 1, 64, torch.bfloat16)]
+    refused = [(1, 2, 49152, 4, 64, torch.float32), (1, 2, 49152, 4, 32, torch.bfloat16),
+               (1, 1, 254976, 2, 64, torch.bfloat16)]
     for B, H, Lx, R, chunk, dtype in refused:
         assert static_need(B, H, Lx, R, chunk, dtype) > STATIC_BYTES
         shape = L.make_shape(B, H, Lx, 64, 64, R, chunk, True, dtype)
@@ -109,6 +112,6 @@ def test_static_scratch_capacity_follows_the_path(lib):
                                        None)
         assert rc == 7
     assert lib.lsh_status_string(7).startswith(b"problem exceeds")
-    _same_as_workspace_call(lib, 1, 8, 16384, 64, 2, 64, True, torch.float32, seed=21)
-    _same_as_workspace_call(lib, 1, 8, 16384, 64, 2, 32, True, torch.bfloat16, seed=22)
-    _same_as_workspace_call(lib, 1, 8, 16384, 64, 1, 64, True, torch.bfloat16, seed=23)
+    _same_as_workspace_call(lib, 1, 2, 49152, 64, 4, 64, True, torch.bfloat16, seed=21)
+    _same_as_workspace_call(lib, 1, 1, 254976, 64, 2, 64, True, torch.float32, seed=22)
+    _same_as_workspace_call(lib, 1, 4, 65536, 64, 1, 64, True, torch.bfloat16, seed=23)
