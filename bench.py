@@ -10,7 +10,8 @@ workload and an L=65536 variant), the same forward end to end from pinned
 host buffers, per-stage times, the roofline of the dominant kernel, every
 other workload's forward with its roofline, recall against full attention
 over rounds and bucket counts, the chunked feed-forward's positions/s with
-its tensor roofline, clocks, and the CPU oracle timed on the host cores
+its tensor roofline, the reversible block's forward and backward tokens/s,
+clocks, and the CPU oracle timed on the host cores
 (with a parity record of the head it recomputes).
 
 ``--impl reference`` times the CPU oracle (the reference arm) on a bounded
@@ -381,6 +382,7 @@ def run_ours(args, world, rank):
         result["workloads"] = run_other_workloads(args, w, world, peaks, peak_kind)
         result["recall"] = run_recall(args)
         result["ffn"] = run_ffn(args, world)
+        result["reversible"] = run_rev(args, world)
     # the head the CPU baseline recomputes, for its parity record
     result["_head0"] = {k: v[:, :1, :1].cpu() if k in ("keys", "perm") else v[:1, :1].cpu()
                         for k, v in outs.items()}
@@ -472,6 +474,54 @@ def run_ffn(args, world):
                          "achieved": round(tfs, 1), "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(tfs / peaks["bf16_tflops"], 4),
                          "traffic": TRAFFIC.get(("ffn", w.name)), "peak_source": peak_kind}}
+
+
+def run_rev(args, world):
+    """The reversible residual block (F = LSH attention, G = chunked
+    feed-forward) on one batch element of L=16384 with 8 heads of 64 (d_model
+    512), 256 buckets, 4 rounds, chunk 64, causal, d_ff 2048, feed-forward
+    chunks of 8192: forward and backward (inputs recomputed from the outputs)
+    tokens per second, device-resident, L2 flushed between steps."""
+    import lsh_attention_long_b200 as L
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, Lx, H, nb, R, chunk, causal, d_ff, fchunk = 1, 16384, 8, 256, 4, 64, True, 2048, 8192
+    D = H * 64
+    g = torch.Generator().manual_seed(30)
+    X1 = torch.randn(B, Lx, D, generator=g).to(dev)
+    X2 = torch.randn(B, Lx, D, generator=g).to(dev)
+    dY1 = torch.randn(B, Lx, D, generator=g).to(dev)
+    dY2 = torch.randn(B, Lx, D, generator=g).to(dev)
+    rot = W.rotations(R, 64, nb, 1, torch.bfloat16).to(dev)
+    w = tuple(v.to(dev) for k, v in W.ffn_inputs(B * Lx, D, d_ff).items()
+              if k in ("W1", "b1", "W2", "b2"))
+    shape = L.make_shape(B, H, Lx, 64, nb, R, chunk, causal, torch.bfloat16)
+    ws = L.rev_workspace(shape, d_ff, fchunk, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    steps = max(3, args.steps // 4)
+    fwd = bwd = 0.0
+    for i in range(max(3, args.warmup) + steps):
+        flush.zero_()
+        e[0].record(stream)
+        Y1, Y2, keys, perm = L.lsh_rev_forward(X1, X2, rot, *w, H, nb, chunk, causal, fchunk,
+                                               ws=ws)
+        e[1].record(stream)
+        L.lsh_rev_backward(Y1, Y2, dY1, dY2, keys, perm, *w, H, nb, chunk, causal, fchunk, ws=ws)
+        e[2].record(stream)
+        e[2].synchronize()
+        if i >= max(3, args.warmup):
+            fwd += e[0].elapsed_time(e[1])
+            bwd += e[1].elapsed_time(e[2])
+    if L.lsh_device_status() != 0:
+        raise RuntimeError("device status error in the reversible block")
+    fwd, bwd = max_over_ranks(fwd, world) / steps, max_over_ranks(bwd, world) / steps
+    del flush, ws
+    return {"value": round(world * B * Lx / ((fwd + bwd) / 1e3), 1), "unit": "tokens/s",
+            "ms_fwd": round(fwd, 4), "ms_bwd": round(bwd, 4), "steps": steps,
+            "fwd_tokens_per_s": round(world * B * Lx / (fwd / 1e3), 1),
+            "config": {"B": B, "L": Lx, "H": H, "d_model": D, "n_buckets": nb, "n_rounds": R,
+                       "chunk": chunk, "causal": causal, "d_ff": d_ff, "ffn_chunk": fchunk}}
 
 
 def run_other_workloads(args, headline, world, peaks, peak_kind):
@@ -706,12 +756,14 @@ def run_recall(args):
 
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-# for the kernel as it stands, keyed by (stage, workload); absent until taken.
-# From one ncu capture of the timed step of `bench.py --steps 1 --warmup 1
-# --no-extras`; to be cleared whenever the kernel changes.
+# for the kernel as it stands, keyed by (stage, workload); absent until taken,
+# and to be cleared whenever the kernel changes.  The attention kernel's figure
+# is from one capture of the L=16384 workload's forward (profiles/
+# attend_tc_kernel_fwd_bf16_L16384.md), the hash kernel's from one capture of
+# the timed step at L=65536.
 TRAFFIC = {
     ("hash", "fwd_bf16_L65536"): 67665000 + 4091648,
-    ("sort", "fwd_bf16_L65536"): 19975000 + 3175936,
+    ("attend", "fwdbwd_bf16_L16384"): 77895168 + 90932992,
 }
 
 

@@ -247,6 +247,64 @@ LSH_API lsh_status lsh_ffn_forward(int32_t tokens, int32_t d_model, int32_t d_ff
                                    const void* b2, void* Y, void* ws, size_t ws_bytes,
                                    void* stream);
 
+/* Backward of the chunked feed-forward (gradients of sum(dY * Y)):
+ *   dA[t] = (W2^T dY[t]) where W1 X[t] + b1 > 0 (max(0, .)' = 0 at 0),
+ *   dX[t] = R[t] + W1^T dA[t]            (R: fp32 [tokens, d_model] or NULL),
+ *   dW1 = sum_t dA[t] X[t]^T,  db1 = sum_t dA[t],
+ *   dW2 = sum_t dY[t] H[t]^T,  db2 = sum_t dY[t],  H[t] = max(0, W1 X[t] + b1),
+ * the hidden activation recomputed chunk by chunk (ws holds one chunk's H
+ * and dA, lsh_ffn_bwd_ws_size() bytes).  X, W1, b1, W2, dY bf16 as in
+ * lsh_ffn_forward; dX [tokens, d_model], dW1 [d_ff, d_model], db1 [d_ff],
+ * dW2 [d_model, d_ff], db2 [d_model] fp32 (the four parameter gradients are
+ * overwritten).  The products run on the tensor cores: the transposed
+ * operands are read in place (MN-major), the parameter gradients accumulate
+ * with fp32 atomics over positions split across thread blocks, so their
+ * summation order varies from call to call. */
+LSH_API size_t lsh_ffn_bwd_ws_size(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk);
+LSH_API lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk,
+                                    const void* X, const void* W1, const void* b1, const void* W2,
+                                    const void* dY, const float* R, float* dX, float* dW1,
+                                    float* db1, float* dW2, float* db2, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* Reversible residual block around LSH attention.  The Reformer abstract
+ * (codewithpapers.app listing) and the explainer (its single section) use
+ * reversible residual layers (RevNet) so that a layer's inputs are
+ * recomputed from its outputs in the backward pass instead of being stored:
+ *   Y1 = X1 + F(X2),   Y2 = X2 + G(Y1),
+ * with F = LSH attention of X2 (each token's features, split into H heads of
+ * d = 64, are its query = key and its value; shape's B, H, L, n_buckets,
+ * n_rounds, chunk, causal; dtype must be LSH_BF16) and G = the chunked
+ * feed-forward (d_model = H * 64, d_ff, ffn_chunk; see lsh_ffn_forward).
+ *   X1, X2, Y1, Y2, dY1, dY2, dX1, dX2: fp32 [B, L, H * 64] (the residual
+ *   stream); the sublayers take bf16 copies of their inputs.
+ *   rot [n_rounds, 64, n_buckets / 2] bf16; W1, b1, W2, b2 bf16 as in
+ *   lsh_ffn_forward; dW1, db1, dW2, db2 fp32 (overwritten).
+ * lsh_rev_forward writes Y1, Y2 and the keys and permutations of X2's hash
+ * ([n_rounds, B, H, L]), which the backward holds constant.
+ * lsh_rev_backward takes only the outputs: it recomputes X2 = Y2 - G(Y1) and
+ * X1 = Y1 - F(X2) (written to X1, X2), and writes
+ *   dX1 = dY1 + G'(Y1)^T dY2,   dX2 = dY2 + F'(X2)^T dX1,
+ * (F'(X2)^T g is the sum of the attention's query and value gradients for
+ * the upstream gradient g) and G's parameter gradients.  ws: at least
+ * lsh_rev_ws_size() bytes of device scratch, caller-owned.  Every step runs
+ * in this library's kernels; nothing is allocated.  Supported: H a multiple
+ * of 4, B * L a multiple of 128, and the limits of lsh_forward and
+ * lsh_ffn_forward. */
+LSH_API size_t lsh_rev_ws_size(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk);
+LSH_API lsh_status lsh_rev_forward(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk,
+                                   const float* X1, const float* X2, const void* rot,
+                                   const void* W1, const void* b1, const void* W2, const void* b2,
+                                   float* Y1, float* Y2, uint32_t* keys, int32_t* perm, void* ws,
+                                   size_t ws_bytes, void* stream);
+LSH_API lsh_status lsh_rev_backward(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk,
+                                    const float* Y1, const float* Y2, const float* dY1,
+                                    const float* dY2, const uint32_t* keys, const int32_t* perm,
+                                    const void* W1, const void* b1, const void* W2,
+                                    const void* b2, float* X1, float* X2, float* dX1, float* dX2,
+                                    float* dW1, float* db1, float* dW2, float* db2, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /* Test hook for the failure path of the bounded device waits.  No passage of
  * the pages corresponds to it.  Every wait in the kernels gives up after a
  * limit of clock cycles (about 2 s by default), records LSH_ERR_TIMEOUT in

@@ -8,5 +8,6 @@ synthetic inputs.
 
 from .lsh import (LshError, Shape, ffn_workspace, forward_host_workspace,  # noqa: F401
                   load_library, lsh_attend_bwd, lsh_attend_fwd, lsh_combine, lsh_device_status,
-                  lsh_ffn_forward, lsh_forward, lsh_forward_host, lsh_hash, lsh_set_wait_test,
-                  lsh_sort, lsh_workspace_size, make_shape, workspace)
+                  lsh_ffn_backward, lsh_ffn_forward, lsh_forward, lsh_forward_host, lsh_hash, lsh_rev_backward, lsh_rev_forward,
+                  lsh_set_wait_test,
+                  lsh_sort, lsh_workspace_size, make_shape, rev_workspace, workspace)

@@ -12,18 +12,24 @@
 // two products).
 //
 // Each product is one launch of gemm_tc_kernel:
-//   C[M, N] = act(A[M, K] . B[N, K]^T + bias[N])
-// with A and B row-major bf16 (both K-major), C row-major bf16.  Tiles of
-// 128 x 256 outputs, K in steps of 64.  Warp roles (192 threads):
+//   C[M, N] = epilogue(A[M, K] . B[N, K]^T)
+// with A and B bf16, each stored either K-major (row-major [M or N][K]) or
+// MN-major (row-major [K][M or N]: a transposed operand read in place, as the
+// backward's products need).  Epilogues: bias and optional max(0, .) to bf16;
+// a zero mask from a bf16 matrix (the derivative of max(0, .)) to bf16; fp32
+// addition of a residual matrix; fp32 atomic accumulation (weight
+// gradients, with K split over CTAs).  Tiles of 128 x 256 outputs, K in
+// steps of 64.  Warp roles (192 threads):
 //   warp 0     one thread loads A and B tiles with TMA (tensor maps, 128-byte
 //              swizzle) into a ring of four stages (full/empty mbarriers with
 //              transaction counts);
 //   warp 1     one thread issues tcgen05.mma (M = 128, N = 256, K = 16) into
 //              one of two 256-column TMEM accumulators;
 //   warps 2-5  epilogue: each thread reads its output row from TMEM (lane =
-//              row), adds the bias, applies max(0, .) when asked, and stores
-//              bf16; it frees the accumulator for the tile after next.
-// CTAs are persistent and take tiles round-robin.
+//              row) and writes it through the epilogue; it frees the
+//              accumulator for the work unit after next.
+// CTAs are persistent and take work units (an output tile and a range of K)
+// round-robin.
 #pragma once
 
 #include <cuda.h>
@@ -37,13 +43,24 @@ constexpr int kGmThreads = 192;
 constexpr int kGmABytes = kGmBM * kGmBK * 2;  // 16 KB
 constexpr int kGmBBytes = kGmBN * kGmBK * 2;  // 32 KB
 
+enum GemmEpi { kEpiBiasAct = 0, kEpiMask = 1, kEpiAddF32 = 2, kEpiAtomicF32 = 3 };
+
 struct GemmArgs {
   int M, N, K;       // M % 128 == 0, N % 256 == 0, K % 64 == 0
-  int a_row0;        // first row of A inside its tensor map
-  const __nv_bfloat16* bias;  // [N]
-  __nv_bfloat16* C;  // row-major, ldc elements per row
+  int a_mn, b_mn;    // operand stored MN-major ([K][M], [K][N]) rather than K-major
+  int a_row0, b_row0;  // offset added to each operand's row (outer) coordinate
+  int k_splits;      // K ranges per output tile (kEpiAtomicF32 only; else 1)
+  int epi;           // GemmEpi
+  const __nv_bfloat16* bias;  // kEpiBiasAct: [N]
+  int relu;                   // kEpiBiasAct: max(0, .)
+  const __nv_bfloat16* mask;  // kEpiMask: output zero where mask <= 0; [M][ldm]
+  int ldm;
+  __nv_bfloat16* C;  // bf16 output, ldc elements per row
   int ldc;
-  int relu;
+  float* C32;        // kEpiAddF32 (C32 = R + acc) and kEpiAtomicF32 (C32 += acc)
+  int ldc32;
+  const float* R;    // kEpiAddF32: [M][ldr], or NULL (C32 = acc)
+  int ldr;
   long long wait_limit;
 };
 
@@ -124,7 +141,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = S.tmem_base;
   const int n_n = g.N / kGmBN;
-  const int n_tiles = (g.M / kGmBM) * n_n;
+  const int n_units = (g.M / kGmBM) * n_n * g.k_splits;
   const int n_k = g.K / kGmBK;
 
   if (warp == 0) {
@@ -133,15 +150,28 @@ __global__ void __launch_bounds__(kGmThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
       uint32_t q = 0;  // k-steps issued
-      for (int t = blockIdx.x; t < n_tiles && !*(volatile int*)&S.abort; t += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units && !*(volatile int*)&S.abort; u += gridDim.x) {
+        const int t = u / g.k_splits, sp = u % g.k_splits;
         const int m0 = (t / n_n) * kGmBM, n0 = (t % n_n) * kGmBN;
-        for (int ks = 0; ks < n_k; ++ks, ++q) {
+        const int k_lo = sp * n_k / g.k_splits, k_hi = (sp + 1) * n_k / g.k_splits;
+        for (int ks = k_lo; ks < k_hi; ++ks, ++q) {
           const int s = q % kGmStages;
           if (!gm_wait(&S.empty[s], ((q / kGmStages) & 1u) ^ 1u, &S.abort, limit)) break;
           mbar_expect_tx(&S.full[s], kGmABytes + kGmBBytes);
-          tma_load_2d(tc::smem_u32(stage_a + s * kGmABytes), &map_a, ks * kGmBK, g.a_row0 + m0,
-                      &S.full[s]);
-          tma_load_2d(tc::smem_u32(stage_b + s * kGmBBytes), &map_b, ks * kGmBK, n0, &S.full[s]);
+          const uint32_t sa = tc::smem_u32(stage_a + s * kGmABytes);
+          const uint32_t sb = tc::smem_u32(stage_b + s * kGmBBytes);
+          if (!g.a_mn) {  // one box: 64 K x 128 rows
+            tma_load_2d(sa, &map_a, ks * kGmBK, g.a_row0 + m0, &S.full[s]);
+          } else {        // two boxes: 64 M x 64 K rows each
+            for (int h = 0; h < kGmBM / 64; ++h)
+              tma_load_2d(sa + h * 8192, &map_a, m0 + 64 * h, g.a_row0 + ks * kGmBK, &S.full[s]);
+          }
+          if (!g.b_mn) {
+            tma_load_2d(sb, &map_b, ks * kGmBK, g.b_row0 + n0, &S.full[s]);
+          } else {
+            for (int h = 0; h < kGmBN / 64; ++h)
+              tma_load_2d(sb + h * 8192, &map_b, n0 + 64 * h, g.b_row0 + ks * kGmBK, &S.full[s]);
+          }
         }
       }
       // every load issued has landed before the CTA leaves
@@ -160,24 +190,32 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_bf16(kGmBM, kGmBN, 0, 0);
+      const uint32_t idesc = tc::idesc_bf16(kGmBM, kGmBN, g.a_mn, g.b_mn);
       uint32_t q = 0, i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++i) {
+        const int sp = u % g.k_splits;
+        const int k_lo = sp * n_k / g.k_splits, k_hi = (sp + 1) * n_k / g.k_splits;
         const int b = i & 1;
         if (!gm_wait(&S.acc_empty[b], ((i >> 1) & 1u) ^ 1u, &S.abort, limit)) break;
         tc::fence_after_sync();
         const uint32_t d = tmem + b * 256;
-        for (int ks = 0; ks < n_k; ++ks, ++q) {
+        for (int ks = k_lo; ks < k_hi; ++ks, ++q) {
           const int s = q % kGmStages;
           if (!gm_wait(&S.full[s], (q / kGmStages) & 1u, &S.abort, limit)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t sa = tc::smem_u32(stage_a + s * kGmABytes);
           const uint32_t sb = tc::smem_u32(stage_b + s * kGmBBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(d, tc::sdesc_sw128(sa + kk * 32, 16, 1024),
-                         tc::sdesc_sw128(sb + kk * 32, 16, 1024), idesc, (ks | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            // K-major: 16 K = 32 bytes along the row; MN-major: 16 K rows of
+            // 128 bytes, 64-element MN blocks 8 KB apart
+            const uint64_t da = g.a_mn ? tc::sdesc_sw128(sa + kk * 2048, 8192, 1024)
+                                       : tc::sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t db = g.b_mn ? tc::sdesc_sw128(sb + kk * 2048, 8192, 1024)
+                                       : tc::sdesc_sw128(sb + kk * 32, 16, 1024);
+            tc::mma_bf16(d, da, db, idesc, (ks > k_lo || kk > 0) ? 1u : 0u);
+          }
           tc::mma_commit(&S.empty[s]);  // the stage is free once these MMAs are done
         }
         if (ok) tc::mma_commit(&S.acc_full[b]);
@@ -198,14 +236,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     const int sub = warp & 3;  // TMEM lanes 32*sub .. 32*sub+31
     const int row_in_tile = sub * 32 + lane;
     uint32_t i = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
+      const int t = u / g.k_splits;
       const int b = i & 1;
       const int m0 = (t / n_n) * kGmBM, n0 = (t % n_n) * kGmBN;
       const bool okw = gm_wait(&S.acc_full[b], (i >> 1) & 1u, &S.abort, limit);
       if (!__all_sync(0xffffffffu, okw)) break;
       tc::fence_after_sync();
       const uint32_t taddr = tmem + b * 256 + ((uint32_t)(sub * 32) << 16);
-      __nv_bfloat16* crow = g.C + (size_t)(m0 + row_in_tile) * g.ldc + n0;
+      const size_t row = (size_t)(m0 + row_in_tile);
 #pragma unroll 1
       for (int c = 0; c < kGmBN / 32; ++c) {
         float v[32];
@@ -216,16 +255,39 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           tc::fence_before_sync();
           tc::mbar_arrive(&S.acc_empty[b]);
         }
+        const int col = n0 + 32 * c;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float bias[8], o[8];
-          load8(g.bias + n0 + 32 * c + 8 * q, bias);
+          float* x = v + 8 * q;
+          if (g.epi == kEpiBiasAct) {
+            float bias[8];
+            load8(g.bias + col + 8 * q, bias);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = v[8 * q + e] + bias[e];
-            o[e] = g.relu ? fmaxf(x, 0.f) : x;
+            for (int e = 0; e < 8; ++e) x[e] = g.relu ? fmaxf(x[e] + bias[e], 0.f) : x[e] + bias[e];
+            store8(g.C + row * g.ldc + col + 8 * q, x);
+          } else if (g.epi == kEpiMask) {
+            float mk[8];
+            load8(g.mask + row * g.ldm + col + 8 * q, mk);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = mk[e] > 0.f ? x[e] : 0.f;
+            store8(g.C + row * g.ldc + col + 8 * q, x);
+          } else if (g.epi == kEpiAddF32) {
+            if (g.R) {
+              float r[8];
+              load8(g.R + row * g.ldr + col + 8 * q, r);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) x[e] += r[e];
+            }
+            store8(g.C32 + row * g.ldc32 + col + 8 * q, x);
+          } else {
+            float* dst = g.C32 + row * g.ldc32 + col + 8 * q;
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(x[0]),
+                         "f"(x[1]), "f"(x[2]), "f"(x[3])
+                         : "memory");
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4), "f"(x[4]),
+                         "f"(x[5]), "f"(x[6]), "f"(x[7])
+                         : "memory");
           }
-          store8(crow + 32 * c + 8 * q, o);
         }
       }
     }
@@ -236,6 +298,19 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
+}
+
+// Column sums of a bf16 matrix [rows][cols] added into fp32 out[cols] (bias
+// gradients): thread x of block (y) sums its column over a slab of rows.
+__global__ void colsum_add_kernel(const __nv_bfloat16* __restrict__ a, int rows, int cols,
+                                  int rows_per_block, float* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const int r0 = blockIdx.y * rows_per_block;
+  const int r1 = min(rows, r0 + rows_per_block);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) s += __bfloat162float(a[(size_t)r * cols + c]);
+  atomicAdd(out + c, s);
 }
 
 }  // namespace lsh

@@ -15,6 +15,7 @@
 #include "ffn_tc.cuh"
 #include "hash_simt.cuh"
 #include "hash_tc.cuh"
+#include "rev.cuh"
 #include "sort.cuh"
 
 // Scratch of lsh_attend_fwd_static: the per-round partials of rounds
@@ -799,16 +800,33 @@ lsh_status ffn_check(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chun
   return LSH_OK;
 }
 
+lsh::GemmArgs gemm_args(int M, int N, int K, int epi) {
+  lsh::GemmArgs g = {};
+  g.M = M; g.N = N; g.K = K; g.epi = epi; g.k_splits = 1;
+  g.wait_limit = g_wait_limit;
+  return g;
+}
+
 lsh_status gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const lsh::GemmArgs& g,
                        cudaStream_t st) {
   const size_t smem = lsh::gemm_tc_smem_bytes();
   lsh_status s0 = allow_smem(lsh::gemm_tc_kernel, smem);
   if (s0 != LSH_OK) return s0;
-  const int tiles = (g.M / lsh::kGmBM) * (g.N / lsh::kGmBN);
+  const int units = (g.M / lsh::kGmBM) * (g.N / lsh::kGmBN) * g.k_splits;
   const int sms = num_sms();
-  lsh::gemm_tc_kernel<<<(unsigned)(tiles < sms ? tiles : sms), lsh::kGmThreads, smem, st>>>(ma, mb,
+  lsh::gemm_tc_kernel<<<(unsigned)(units < sms ? units : sms), lsh::kGmThreads, smem, st>>>(ma, mb,
                                                                                           g);
   return last_launch();
+}
+
+// K ranges per output tile for a weight-gradient product: enough work units
+// to fill the SMs, each at least four K steps long.
+int k_splits_for(int tiles, int K) {
+  const int sms = num_sms();
+  int ks = (sms + tiles - 1) / tiles;
+  const int max_ks = (K / lsh::kGmBK) / 4;
+  if (ks > max_ks) ks = max_ks;
+  return ks < 1 ? 1 : ks;
 }
 
 }  // namespace
@@ -840,22 +858,250 @@ lsh_status lsh_ffn_forward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_
   for (int c0 = 0; c0 < tokens; c0 += chunk) {
     const int n = tokens - c0 < chunk ? tokens - c0 : chunk;
     // H = max(0, X[c0 : c0+n] W1^T + b1): the chunk's hidden activation
-    lsh::GemmArgs g1;
-    g1.M = n; g1.N = d_ff; g1.K = d_model; g1.a_row0 = c0;
+    lsh::GemmArgs g1 = gemm_args(n, d_ff, d_model, lsh::kEpiBiasAct);
+    g1.a_row0 = c0;
     g1.bias = static_cast<const __nv_bfloat16*>(b1);
-    g1.C = H; g1.ldc = d_ff; g1.relu = 1; g1.wait_limit = g_wait_limit;
+    g1.relu = 1;
+    g1.C = H; g1.ldc = d_ff;
     s = gemm_launch(mx, mw1, g1, st);
     if (s != LSH_OK) return s;
     // Y[c0 : c0+n] = H W2^T + b2
-    lsh::GemmArgs g2;
-    g2.M = n; g2.N = d_model; g2.K = d_ff; g2.a_row0 = 0;
+    lsh::GemmArgs g2 = gemm_args(n, d_model, d_ff, lsh::kEpiBiasAct);
     g2.bias = static_cast<const __nv_bfloat16*>(b2);
-    g2.C = static_cast<__nv_bfloat16*>(Y) + (size_t)c0 * d_model; g2.ldc = d_model; g2.relu = 0;
-    g2.wait_limit = g_wait_limit;
+    g2.C = static_cast<__nv_bfloat16*>(Y) + (size_t)c0 * d_model; g2.ldc = d_model;
     s = gemm_launch(mh, mw2, g2, st);
     if (s != LSH_OK) return s;
   }
   return LSH_OK;
+}
+
+size_t lsh_ffn_bwd_ws_size(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk) {
+  if (ffn_check(tokens, d_model, d_ff, chunk) != LSH_OK || tokens == 0) return 0;
+  return 2 * align_up((size_t)chunk * d_ff * sizeof(__nv_bfloat16));
+}
+
+lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk,
+                            const void* X, const void* W1, const void* b1, const void* W2,
+                            const void* dY, const float* R, float* dX, float* dW1, float* db1,
+                            float* dW2, float* db2, void* ws, size_t ws_bytes, void* stream) {
+  lsh_status s = ffn_check(tokens, d_model, d_ff, chunk);
+  if (s != LSH_OK) return s;
+  if (!X || !W1 || !b1 || !W2 || !dY || !dX || !dW1 || !db1 || !dW2 || !db2 || !ws)
+    return LSH_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(W1) || misaligned(b1) || misaligned(W2) || misaligned(dY) ||
+      misaligned(R) || misaligned(dX) || misaligned(dW1) || misaligned(db1) || misaligned(dW2) ||
+      misaligned(db2) || misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  // the weight and bias gradients are sums over every position
+  if (cudaMemsetAsync(dW1, 0, (size_t)d_ff * d_model * sizeof(float), st) != cudaSuccess ||
+      cudaMemsetAsync(db1, 0, (size_t)d_ff * sizeof(float), st) != cudaSuccess ||
+      cudaMemsetAsync(dW2, 0, (size_t)d_model * d_ff * sizeof(float), st) != cudaSuccess ||
+      cudaMemsetAsync(db2, 0, (size_t)d_model * sizeof(float), st) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  if (tokens == 0) return LSH_OK;
+  const size_t hbytes = align_up((size_t)chunk * d_ff * sizeof(__nv_bfloat16));
+  if (ws_bytes < 2 * hbytes) return LSH_ERR_WORKSPACE;
+  __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + hbytes);
+  // K-major operands read rows of K in 128-row (A) or 256-row (B) boxes;
+  // MN-major operands read 64 x 64 boxes of [K][MN] storage
+  CUtensorMap mx, mw1, mdy, mda, mw2_mn, mw1_mn, mdy_mn, mh_mn, mda_mn, mx_mn;
+  const uint64_t T = (uint64_t)tokens, C = (uint64_t)chunk, D = (uint64_t)d_model,
+                 F = (uint64_t)d_ff;
+  if (!bf16_map(&mx, X, T, D, lsh::kGmBM) || !bf16_map(&mw1, W1, F, D, lsh::kGmBN) ||
+      !bf16_map(&mdy, dY, T, D, lsh::kGmBM) || !bf16_map(&mda, dA, C, F, lsh::kGmBM) ||
+      !bf16_map(&mw2_mn, W2, D, F, 64) || !bf16_map(&mw1_mn, W1, F, D, 64) ||
+      !bf16_map(&mdy_mn, dY, T, D, 64) || !bf16_map(&mh_mn, H, C, F, 64) ||
+      !bf16_map(&mda_mn, dA, C, F, 64) || !bf16_map(&mx_mn, X, T, D, 64))
+    return LSH_ERR_CUDA;
+  for (int c0 = 0; c0 < tokens; c0 += chunk) {
+    const int n = tokens - c0 < chunk ? tokens - c0 : chunk;
+    // H = max(0, X W1^T + b1), recomputed for the chunk
+    lsh::GemmArgs g1 = gemm_args(n, d_ff, d_model, lsh::kEpiBiasAct);
+    g1.a_row0 = c0;
+    g1.bias = static_cast<const __nv_bfloat16*>(b1);
+    g1.relu = 1;
+    g1.C = H; g1.ldc = d_ff;
+    if ((s = gemm_launch(mx, mw1, g1, st)) != LSH_OK) return s;
+    // dA = (dY W2) where H > 0: the gradient at the pre-activation
+    lsh::GemmArgs g2 = gemm_args(n, d_ff, d_model, lsh::kEpiMask);
+    g2.a_row0 = c0;
+    g2.b_mn = 1;  // W2 [d_model][d_ff] is [K][N]
+    g2.mask = H; g2.ldm = d_ff;
+    g2.C = dA; g2.ldc = d_ff;
+    if ((s = gemm_launch(mdy, mw2_mn, g2, st)) != LSH_OK) return s;
+    // dX = R + dA W1
+    lsh::GemmArgs g3 = gemm_args(n, d_model, d_ff, lsh::kEpiAddF32);
+    g3.b_mn = 1;  // W1 [d_ff][d_model] is [K][N]
+    g3.C32 = dX + (size_t)c0 * d_model; g3.ldc32 = d_model;
+    g3.R = R ? R + (size_t)c0 * d_model : nullptr; g3.ldr = d_model;
+    if ((s = gemm_launch(mda, mw1_mn, g3, st)) != LSH_OK) return s;
+    // dW2 += dY^T H, dW1 += dA^T X (positions are K, split over CTAs)
+    lsh::GemmArgs g4 = gemm_args(d_model, d_ff, n, lsh::kEpiAtomicF32);
+    g4.a_mn = 1; g4.b_mn = 1; g4.a_row0 = c0;
+    g4.k_splits = k_splits_for((d_model / lsh::kGmBM) * (d_ff / lsh::kGmBN), n);
+    g4.C32 = dW2; g4.ldc32 = d_ff;
+    if ((s = gemm_launch(mdy_mn, mh_mn, g4, st)) != LSH_OK) return s;
+    lsh::GemmArgs g5 = gemm_args(d_ff, d_model, n, lsh::kEpiAtomicF32);
+    g5.a_mn = 1; g5.b_mn = 1; g5.b_row0 = c0;
+    g5.k_splits = k_splits_for((d_ff / lsh::kGmBM) * (d_model / lsh::kGmBN), n);
+    g5.C32 = dW1; g5.ldc32 = d_model;
+    if ((s = gemm_launch(mda_mn, mx_mn, g5, st)) != LSH_OK) return s;
+    // db2 += column sums of dY, db1 += column sums of dA
+    const int rpb = 256;
+    const dim3 gb2((unsigned)((d_model + 255) / 256), (unsigned)((n + rpb - 1) / rpb));
+    lsh::colsum_add_kernel<<<gb2, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dY) + (size_t)c0 * d_model, n, d_model, rpb, db2);
+    const dim3 gb1((unsigned)((d_ff + 255) / 256), (unsigned)((n + rpb - 1) / rpb));
+    lsh::colsum_add_kernel<<<gb1, 256, 0, st>>>(dA, n, d_ff, rpb, db1);
+    if ((s = last_launch()) != LSH_OK) return s;
+  }
+  return LSH_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Reversible residual block around LSH attention
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct RevLayout {
+  size_t x2h, o, lse, y1b, g, dyb, dO, dq, dv, attn, ffn, total;
+  size_t attn_bytes, ffn_bytes;
+};
+
+lsh_status rev_check(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk, Dims* D) {
+  lsh_status s = check_shape(shape, D);
+  if (s != LSH_OK) return s;
+  if (D->dtype != LSH_BF16) return LSH_ERR_UNSUPPORTED;
+  return ffn_check(D->B * D->L, D->H * kHeadDim, d_ff, ffn_chunk);
+}
+
+RevLayout rev_layout(const lsh_shape* shape, const Dims& D, int32_t d_ff, int32_t ffn_chunk) {
+  RevLayout l;
+  const size_t n = D.n_tok * kHeadDim;  // elements of one activation
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off += align_up(bytes); return at; };
+  l.x2h = take(n * 2);
+  l.o = take(n * 2);
+  l.lse = take(D.n_tok * sizeof(float));
+  l.y1b = take(n * 2);
+  l.g = take(n * 2);
+  l.dyb = take(n * 2);
+  l.dO = take(n * 2);
+  l.dq = take(n * 2);
+  l.dv = take(n * 2);
+  l.attn_bytes = lsh_workspace_size(shape);
+  l.attn = take(l.attn_bytes);
+  const int T = D.B * D.L, Dm = D.H * kHeadDim;
+  const size_t f = lsh_ffn_ws_size(T, Dm, d_ff, ffn_chunk),
+               b = lsh_ffn_bwd_ws_size(T, Dm, d_ff, ffn_chunk);
+  l.ffn_bytes = f > b ? f : b;
+  l.ffn = take(l.ffn_bytes);
+  l.total = off;
+  return l;
+}
+
+inline unsigned blocks8(size_t n8) { return (unsigned)((n8 + 255) / 256); }
+
+}  // namespace
+
+size_t lsh_rev_ws_size(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk) {
+  Dims D;
+  if (rev_check(shape, d_ff, ffn_chunk, &D) != LSH_OK || D.empty) return 0;
+  return rev_layout(shape, D, d_ff, ffn_chunk).total;
+}
+
+lsh_status lsh_rev_forward(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk,
+                           const float* X1, const float* X2, const void* rot, const void* W1,
+                           const void* b1, const void* W2, const void* b2, float* Y1, float* Y2,
+                           uint32_t* keys, int32_t* perm, void* ws, size_t ws_bytes,
+                           void* stream) {
+  Dims D;
+  lsh_status s = rev_check(shape, d_ff, ffn_chunk, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!X1 || !X2 || !Y1 || !Y2 || !keys || !perm || !ws || (D.nb > 1 && !rot))
+    return LSH_ERR_INVALID_ARG;
+  if (misaligned(X1) || misaligned(X2) || misaligned(Y1) || misaligned(Y2) || misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  const RevLayout l = rev_layout(shape, D, d_ff, ffn_chunk);
+  if (ws_bytes < l.total) return LSH_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  char* w = static_cast<char*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w + off); };
+  const lsh::RevDims r{D.B, D.H, D.L};
+  const size_t n8 = D.n_tok * 8;
+  const int T = D.B * D.L, Dm = D.H * kHeadDim;
+  // F: LSH attention of X2 (its own query, key and value), head-major bf16
+  lsh::rev_to_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, X2, bf(l.x2h));
+  if ((s = last_launch()) != LSH_OK) return s;
+  s = lsh_forward(shape, bf(l.x2h), bf(l.x2h), rot, keys, nullptr, perm, bf(l.o),
+                  reinterpret_cast<float*>(w + l.lse), w + l.attn, l.attn_bytes, stream);
+  if (s != LSH_OK) return s;
+  // Y1 = X1 + F(X2), and Y1 in bf16 for G
+  lsh::rev_residual_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, X1, bf(l.o), 1.f, Y1, bf(l.y1b));
+  if ((s = last_launch()) != LSH_OK) return s;
+  // G: the chunked feed-forward of Y1; Y2 = X2 + G(Y1)
+  s = lsh_ffn_forward(T, Dm, d_ff, ffn_chunk, bf(l.y1b), W1, b1, W2, b2, bf(l.g), w + l.ffn,
+                      l.ffn_bytes, stream);
+  if (s != LSH_OK) return s;
+  lsh::rev_residual_kernel<<<blocks8(n8), 256, 0, st>>>(n8, X2, bf(l.g), 1.f, Y2, nullptr);
+  return last_launch();
+}
+
+lsh_status lsh_rev_backward(const lsh_shape* shape, int32_t d_ff, int32_t ffn_chunk,
+                            const float* Y1, const float* Y2, const float* dY1, const float* dY2,
+                            const uint32_t* keys, const int32_t* perm, const void* W1,
+                            const void* b1, const void* W2, const void* b2, float* X1, float* X2,
+                            float* dX1, float* dX2, float* dW1, float* db1, float* dW2, float* db2,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  lsh_status s = rev_check(shape, d_ff, ffn_chunk, &D);
+  if (s != LSH_OK) return s;
+  if (D.empty) return LSH_OK;
+  if (!Y1 || !Y2 || !dY1 || !dY2 || !keys || !perm || !X1 || !X2 || !dX1 || !dX2 || !ws)
+    return LSH_ERR_INVALID_ARG;
+  if (misaligned(Y1) || misaligned(Y2) || misaligned(dY1) || misaligned(dY2) || misaligned(X1) ||
+      misaligned(X2) || misaligned(dX1) || misaligned(dX2) || misaligned(ws))
+    return LSH_ERR_INVALID_ARG;
+  const RevLayout l = rev_layout(shape, D, d_ff, ffn_chunk);
+  if (ws_bytes < l.total) return LSH_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  char* w = static_cast<char*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w + off); };
+  float* lse = reinterpret_cast<float*>(w + l.lse);
+  const lsh::RevDims r{D.B, D.H, D.L};
+  const size_t n8 = D.n_tok * 8;
+  const int T = D.B * D.L, Dm = D.H * kHeadDim;
+  // X2 = Y2 - G(Y1), G recomputed from Y1
+  lsh::rev_residual_kernel<<<blocks8(n8), 256, 0, st>>>(n8, Y1, nullptr, 0.f, nullptr, bf(l.y1b));
+  if ((s = last_launch()) != LSH_OK) return s;
+  s = lsh_ffn_forward(T, Dm, d_ff, ffn_chunk, bf(l.y1b), W1, b1, W2, b2, bf(l.g), w + l.ffn,
+                      l.ffn_bytes, stream);
+  if (s != LSH_OK) return s;
+  lsh::rev_residual_kernel<<<blocks8(n8), 256, 0, st>>>(n8, Y2, bf(l.g), -1.f, X2, nullptr);
+  lsh::rev_to_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, X2, bf(l.x2h));
+  // dX1 = dY1 + G'(Y1)^T dY2, with G's parameter gradients
+  lsh::rev_residual_kernel<<<blocks8(n8), 256, 0, st>>>(n8, dY2, nullptr, 0.f, nullptr, bf(l.dyb));
+  if ((s = last_launch()) != LSH_OK) return s;
+  s = lsh_ffn_backward(T, Dm, d_ff, ffn_chunk, bf(l.y1b), W1, b1, W2, bf(l.dyb), dY1, dX1, dW1,
+                       db1, dW2, db2, w + l.ffn, l.ffn_bytes, stream);
+  if (s != LSH_OK) return s;
+  // X1 = Y1 - F(X2), F recomputed with the forward's buckets
+  s = lsh_attend_fwd(shape, bf(l.x2h), bf(l.x2h), keys, perm, nullptr, nullptr, bf(l.o), lse,
+                     w + l.attn, l.attn_bytes, stream);
+  if (s != LSH_OK) return s;
+  lsh::rev_residual_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, Y1, bf(l.o), -1.f, X1, nullptr);
+  // dX2 = dY2 + F'(X2)^T dX1: the attention's query and value gradients
+  lsh::rev_to_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, dX1, bf(l.dO));
+  if ((s = last_launch()) != LSH_OK) return s;
+  s = lsh_attend_bwd(shape, bf(l.x2h), bf(l.x2h), bf(l.o), bf(l.dO), keys, perm, lse, bf(l.dq),
+                     bf(l.dv), w + l.attn, l.attn_bytes, stream);
+  if (s != LSH_OK) return s;
+  lsh::rev_grad_x2_kernel<<<blocks8(n8), 256, 0, st>>>(r, dY2, bf(l.dq), bf(l.dv), dX2);
+  return last_launch();
 }
 
 lsh_status lsh_set_wait_test(int32_t hold_tile, int64_t wait_cycles) {

@@ -26,7 +26,8 @@ STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "L
 EXPORTS = ("lsh_workspace_size", "lsh_hash", "lsh_sort", "lsh_attend_fwd", "lsh_combine",
            "lsh_forward", "lsh_forward_host", "lsh_forward_host_ws_size", "lsh_attend_bwd",
            "lsh_device_status", "lsh_status_string", "lsh_attend_fwd_static", "lsh_set_wait_test",
-           "lsh_ffn_ws_size", "lsh_ffn_forward")
+           "lsh_ffn_ws_size", "lsh_ffn_forward", "lsh_ffn_bwd_ws_size", "lsh_ffn_backward",
+           "lsh_rev_ws_size", "lsh_rev_forward", "lsh_rev_backward")
 
 
 class LshError(RuntimeError):
@@ -69,6 +70,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lsh_set_wait_test": ([ctypes.c_int32, ctypes.c_int64], ctypes.c_int),
         "lsh_ffn_ws_size": ([ctypes.c_int32] * 4, sz),
         "lsh_ffn_forward": ([ctypes.c_int32] * 4 + [P] * 7 + [sz, P], ctypes.c_int),
+        "lsh_ffn_bwd_ws_size": ([ctypes.c_int32] * 4, sz),
+        "lsh_ffn_backward": ([ctypes.c_int32] * 4 + [P] * 12 + [sz, P], ctypes.c_int),
+        "lsh_rev_ws_size": ([S, ctypes.c_int32, ctypes.c_int32], sz),
+        "lsh_rev_forward": ([S, ctypes.c_int32, ctypes.c_int32] + [P] * 12 + [sz, P],
+                            ctypes.c_int),
+        "lsh_rev_backward": ([S, ctypes.c_int32, ctypes.c_int32] + [P] * 19 + [sz, P],
+                             ctypes.c_int),
         "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -362,6 +370,110 @@ def lsh_ffn_forward(X, W1, b1, W2, b2, chunk: int, *, Y=None, ws=None, stream=No
     _call("lsh_ffn_forward", tokens, d_model, d_ff, chunk, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2),
           _ptr(b2), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream))
     return Y
+
+
+def lsh_ffn_backward(X, W1, b1, W2, dY, chunk: int, *, R=None, dX=None, grads=None, ws=None,
+                     stream=None):
+    """Backward of the chunked feed-forward: returns dX (fp32, plus R when
+    given) and the fp32 gradients dW1, db1, dW2, db2 (in ``grads`` when given)."""
+    if not isinstance(X, torch.Tensor) or X.dim() < 2:
+        raise ValueError("X must be a [..., d_model] tensor")
+    d_model = X.shape[-1]
+    tokens = X.numel() // d_model if d_model else 0
+    d_ff = W1.shape[0] if isinstance(W1, torch.Tensor) and W1.dim() == 2 else -1
+    bf, f32 = torch.bfloat16, torch.float32
+    g = dict(grads or {})
+    _validate([("X", X, None, bf, True), ("W1", W1, (d_ff, d_model), bf, True),
+               ("b1", b1, (d_ff,), bf, True), ("W2", W2, (d_model, d_ff), bf, True),
+               ("dY", dY, X.shape, bf, True), ("R", R, X.shape, f32, True),
+               ("dX", dX, X.shape, f32, True), ("dW1", g.get("dW1"), (d_ff, d_model), f32, True),
+               ("db1", g.get("db1"), (d_ff,), f32, True),
+               ("dW2", g.get("dW2"), (d_model, d_ff), f32, True),
+               ("db2", g.get("db2"), (d_model,), f32, True), ("ws", ws, None, None, True)])
+    dev = X.device
+    if dX is None:
+        dX = torch.empty(X.shape, dtype=f32, device=dev)
+    g.setdefault("dW1", torch.empty((d_ff, d_model), dtype=f32, device=dev))
+    g.setdefault("db1", torch.empty((d_ff,), dtype=f32, device=dev))
+    g.setdefault("dW2", torch.empty((d_model, d_ff), dtype=f32, device=dev))
+    g.setdefault("db2", torch.empty((d_model,), dtype=f32, device=dev))
+    if ws is None:
+        n = load_library().lsh_ffn_bwd_ws_size(tokens, d_model, d_ff, chunk)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+    _call("lsh_ffn_backward", tokens, d_model, d_ff, chunk, _ptr(X), _ptr(W1), _ptr(b1), _ptr(W2),
+          _ptr(dY), _ptr(R), _ptr(dX), _ptr(g["dW1"]), _ptr(g["db1"]), _ptr(g["dW2"]),
+          _ptr(g["db2"]), _ptr(ws), ws.numel(), _stream(stream))
+    return dX, g
+
+
+def _rev_shape(X, H, n_buckets, n_rounds, chunk, causal):
+    if not isinstance(X, torch.Tensor) or X.dim() != 3 or X.shape[2] % H:
+        raise ValueError("X must be a [B, L, H * 64] tensor")
+    B, Lx, D = X.shape
+    return make_shape(B, H, Lx, D // H, n_buckets, n_rounds, chunk, causal, torch.bfloat16)
+
+
+def rev_workspace(shape: Shape, d_ff: int, ffn_chunk: int, device) -> torch.Tensor:
+    n = load_library().lsh_rev_ws_size(ctypes.byref(shape), d_ff, ffn_chunk)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def lsh_rev_forward(X1, X2, rot, W1, b1, W2, b2, H: int, n_buckets: int, chunk: int,
+                    causal: bool, ffn_chunk: int, *, ws=None, stream=None):
+    """Reversible block: Y1 = X1 + F(X2), Y2 = X2 + G(Y1) (F: LSH attention,
+    G: chunked feed-forward).  X1, X2 fp32 [B, L, H*64].  Returns Y1, Y2 and
+    the keys and permutations of X2's hash."""
+    R = rot.shape[0]
+    shape = _rev_shape(X2, H, n_buckets, R, chunk, causal)
+    B, Lx, D = X2.shape
+    d_ff = W1.shape[0] if isinstance(W1, torch.Tensor) and W1.dim() == 2 else -1
+    f32, bf = torch.float32, torch.bfloat16
+    _validate([("X1", X1, X2.shape, f32, True), ("X2", X2, None, f32, True),
+               _rot_spec(rot, R, 64, n_buckets, bf), ("W1", W1, (d_ff, D), bf, True),
+               ("b1", b1, (d_ff,), bf, True), ("W2", W2, (D, d_ff), bf, True),
+               ("b2", b2, (D,), bf, True), ("ws", ws, None, None, True)])
+    dev = X2.device
+    Y1, Y2 = torch.empty_like(X2), torch.empty_like(X2)
+    keys = torch.empty((R, B, H, Lx), dtype=torch.int32, device=dev)
+    perm = torch.empty_like(keys)
+    if ws is None:
+        ws = rev_workspace(shape, d_ff, ffn_chunk, dev)
+    _call("lsh_rev_forward", ctypes.byref(shape), d_ff, ffn_chunk, _ptr(X1), _ptr(X2),
+          _ptr(rot) if n_buckets > 1 else None, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(Y1),
+          _ptr(Y2), _ptr(keys), _ptr(perm), _ptr(ws), ws.numel(), _stream(stream))
+    return Y1, Y2, keys, perm
+
+
+def lsh_rev_backward(Y1, Y2, dY1, dY2, keys, perm, W1, b1, W2, b2, H: int, n_buckets: int,
+                     chunk: int, causal: bool, ffn_chunk: int, *, ws=None, stream=None):
+    """Backward of the reversible block from its outputs: returns the
+    recomputed X1, X2, the input gradients dX1, dX2 (fp32) and G's parameter
+    gradients {dW1, db1, dW2, db2} (fp32)."""
+    R = keys.shape[0]
+    shape = _rev_shape(Y2, H, n_buckets, R, chunk, causal)
+    B, Lx, D = Y2.shape
+    d_ff = W1.shape[0] if isinstance(W1, torch.Tensor) and W1.dim() == 2 else -1
+    f32, bf = torch.float32, torch.bfloat16
+    rows = (R, B, H, Lx)
+    _validate([("Y1", Y1, Y2.shape, f32, True), ("Y2", Y2, None, f32, True),
+               ("dY1", dY1, Y2.shape, f32, True), ("dY2", dY2, Y2.shape, f32, True),
+               ("keys", keys, rows, torch.int32, True), ("perm", perm, rows, torch.int32, True),
+               ("W1", W1, (d_ff, D), bf, True), ("b1", b1, (d_ff,), bf, True),
+               ("W2", W2, (D, d_ff), bf, True), ("b2", b2, (D,), bf, True),
+               ("ws", ws, None, None, True)])
+    dev = Y2.device
+    X1, X2, dX1, dX2 = (torch.empty_like(Y2) for _ in range(4))
+    g = {"dW1": torch.empty((d_ff, D), dtype=f32, device=dev),
+         "db1": torch.empty((d_ff,), dtype=f32, device=dev),
+         "dW2": torch.empty((D, d_ff), dtype=f32, device=dev),
+         "db2": torch.empty((D,), dtype=f32, device=dev)}
+    if ws is None:
+        ws = rev_workspace(shape, d_ff, ffn_chunk, dev)
+    _call("lsh_rev_backward", ctypes.byref(shape), d_ff, ffn_chunk, _ptr(Y1), _ptr(Y2), _ptr(dY1),
+          _ptr(dY2), _ptr(keys), _ptr(perm), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(X1),
+          _ptr(X2), _ptr(dX1), _ptr(dX2), _ptr(g["dW1"]), _ptr(g["db1"]), _ptr(g["dW2"]),
+          _ptr(g["db2"]), _ptr(ws), ws.numel(), _stream(stream))
+    return X1, X2, dX1, dX2, g
 
 
 def lsh_set_wait_test(hold_tile: int = -1, wait_cycles: int = 0) -> None:

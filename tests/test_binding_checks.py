@@ -70,3 +70,22 @@ def test_host_buffer_forward_wants_host_inputs_and_a_device_workspace():
                                                                    dtype=Q.dtype))
     with pytest.raises(ValueError, match="ws must be a CUDA tensor"):
         L.lsh_forward_host(Q, V, rot, NB, 64, True, ws=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every entry point's ctypes signature has as many arguments as its
+    declaration in include/lsh.h (the C functions take plain pointers, so a
+    miscounted signature would pass the wrong value to the library)."""
+    import os
+    import re
+    from lsh_attention_long_b200 import lsh as M
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    text = open(os.path.join(root, "include", "lsh.h")).read()
+    decls = {m.group(1): m.group(2) for m in
+             re.finditer(r"LSH_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)", text)}
+    lib = M.load_library() if os.path.exists(M.LIB_PATH) else None
+    if lib is None:
+        pytest.skip("library not built")
+    for name, params in decls.items():
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        assert len(getattr(lib, name).argtypes or []) == n, name

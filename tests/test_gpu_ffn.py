@@ -85,3 +85,54 @@ def test_ffn_rejects_unsupported_shapes_and_empty_input_is_a_no_op():
     Y = L.lsh_ffn_forward(empty, t["W1"], t["b1"], t["W2"], t["b2"], 128)
     assert Y.numel() == 0
     assert L.lsh_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def _run_bwd(inp, chunk, with_residual):
+    t = {k: v.cuda() for k, v in inp.items()}
+    R = torch.randn(t["X"].shape, generator=torch.Generator().manual_seed(9)).cuda() \
+        if with_residual else None
+    dX, g = L.lsh_ffn_backward(t["X"], t["W1"], t["b1"], t["W2"], t["dY"], chunk, R=R)
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
+    return dX, g, R
+
+
+@pytest.mark.parametrize("tokens,d_model,d_ff,chunk,with_residual", [
+    (128, 256, 256, 128, False),
+    (512, 256, 512, 128, True),
+    (1024, 512, 2048, 384, True),   # a ragged last chunk
+])
+def test_ffn_backward_matches_the_oracle(oracle, tokens, d_model, d_ff, chunk, with_residual):
+    inp = W.ffn_inputs(tokens, d_model, d_ff, seed=7 * tokens + d_ff, backward=True)
+    dX, g, R = _run_bwd(inp, chunk, with_residual)
+    ref = oracle.ffn_backward(*(_np(inp[k]) for k in ("X", "W1", "b1", "W2", "dY")), chunk)
+    rdX = ref[0] + (_np(R) if R is not None else 0.0)
+    np.testing.assert_allclose(_np(dX), rdX, rtol=0, atol=TOL)
+    # parameter gradients sum over every position: compare relative to their
+    # scale (bf16 operands, fp32 accumulation)
+    for name, r in zip(("dW1", "db1", "dW2", "db2"), ref[1:]):
+        scale = max(1.0, float(np.abs(r).max()))
+        np.testing.assert_allclose(_np(g[name]), r, rtol=0, atol=TOL * scale, err_msg=name)
+
+
+def test_ffn_backward_at_full_size(oracle, parity_record):
+    """The workload's backward: dX on 256 sampled positions and the bias
+    gradients in full (they sum every position) against the oracle."""
+    w = W.FFN_WORKLOADS["ffn_bf16_L65536"]
+    inp = W.ffn_inputs(w.tokens, w.d_model, w.d_ff, backward=True)
+    dX, g, _ = _run_bwd(inp, w.chunk, False)
+    rows = np.random.default_rng(1).choice(w.tokens, 256, replace=False)
+    ref = oracle.ffn_backward(_np(inp["X"])[rows], *(_np(inp[k]) for k in ("W1", "b1", "W2")),
+                              _np(inp["dY"])[rows], 128)
+    err = float(np.abs(_np(dX)[rows] - ref[0]).max())
+    db2 = _np(inp["dY"]).astype(np.float64).sum(0)
+    scale = max(1.0, float(np.abs(db2).max()))
+    err_db2 = float(np.abs(_np(g["db2"]) - db2).max())
+    parity_record.append({"workload": w.name + " (backward)", "positions_checked": len(rows),
+                          "max_abs": {"dX": err, "db2": err_db2}, "tol": TOL})
+    assert err <= TOL
+    assert err_db2 <= TOL * scale
