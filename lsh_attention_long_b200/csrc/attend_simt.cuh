@@ -367,11 +367,11 @@ attend_bwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ V, const T
 
 // dQ = dq + (dkhat - khat (khat . dkhat)) / |q|,  dV = dv, cast to T.  With
 // dk_acc null the projection is already inside dq (dQ = dq).
-template <typename T>
+template <typename T, typename OutT = T>
 __global__ void bwd_finalize_kernel(const T* __restrict__ Q, const float* __restrict__ dq_acc,
                                     const float* __restrict__ dk_acc,
                                     const float* __restrict__ dv_acc, size_t n_tok,
-                                    T* __restrict__ dQ, T* __restrict__ dV) {
+                                    OutT* __restrict__ dQ, OutT* __restrict__ dV) {
   const size_t tok = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tok >= n_tok) return;
   if (!dk_acc) {

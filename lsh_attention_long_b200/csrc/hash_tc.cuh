@@ -342,4 +342,174 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
   }
 }
 
+// ---------------------------------------------------------------------------
+// Four epilogue warpgroups, for nb/2 = 128 and an even number of rounds per
+// group.  Every job (128 tokens x two rounds = 256 columns in one of two TMEM
+// buffers) is read by the pair of warpgroups of its buffer, one round each,
+// so four epilogue warps share each SM sub-partition instead of two and every
+// warpgroup finishes the exact argmax of a whole round on its own.  Measured
+// against the two-warpgroup kernel (same keys): 10% faster at nb = 256, but
+// slower at nb = 1024, where a round's 512 columns would be split over four
+// warpgroups and their partial maxima merged.
+// ---------------------------------------------------------------------------
+
+constexpr int kHash4Threads = 576;  // four epilogue warpgroups, MMA warp, Q loader
+constexpr int kHash4Batch = 32;     // TMEM columns read per wait
+
+__host__ __device__ inline size_t hash_tc4_smem_bytes(int rounds_per_group) {
+  // alignment slack, rotation columns (128 per round), two Q tiles, 64 bytes
+  // of parking per epilogue thread
+  return 1024 + (size_t)rounds_per_group * 128 * 128 + 2 * 16384 + 512 * 64;
+}
+
+__global__ void __launch_bounds__(kHash4Threads, 1) hash_tc4_kernel(HashTcArgs a) {
+  constexpr int CW = 16;
+  constexpr int kHalf = 128;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t buf_full[2], buf_empty[2], q_full[2], q_empty[2];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int g = blockIdx.x % a.n_groups;
+  const int c = blockIdx.x / a.n_groups;
+  const int r0 = g * a.rounds_per_group;
+  const int nr = min(a.rounds_per_group, a.R - r0);
+  const int cols = nr * kHalf;
+  const int T = cols / 256;  // N-tiles (round pairs) per token tile
+  uint8_t* rot_s = sm;
+  uint8_t* q_s = sm + (size_t)a.rounds_per_group * kHalf * 128;
+  uint8_t* park = q_s + 2 * 16384;
+
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&buf_full[b], 1);
+      tc::mbar_init(&buf_empty[b], 256);  // both warpgroups of the buffer's pair
+      tc::mbar_init(&q_full[b], 32);
+      tc::mbar_init(&q_empty[b], 1);
+    }
+    tc::mbar_init_fence();
+    abort_s = 0;
+  }
+  if (warp == 16) {
+    tc::tmem_alloc(&tmem_base_s, 512);
+    tc::tmem_relinquish();
+  }
+  // rotation columns of this group, transposed: smem row j holds column j
+  for (int row = tid; row < cols; row += blockDim.x) {
+    const __nv_bfloat16* src = a.rot + (size_t)(r0 + row / a.half) * 64 * a.half + row % a.half;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = __bfloat16_as_ushort(src[(size_t)(ch * 8 + 2 * e) * a.half]);
+        const uint32_t hi = __bfloat16_as_ushort(src[(size_t)(ch * 8 + 2 * e + 1) * a.half]);
+        w[e] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(rot_s + tc::sw128_offset(row, ch)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  tc::fence_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base_s;
+  const int n_items =
+      (c < a.n_mtiles) ? (a.n_mtiles - c + a.ctas_per_group - 1) / a.ctas_per_group : 0;
+  const int n_jobs = n_items * T;
+
+  if (warp == 17) {
+    // ------------------------------------------------------- Q tile loads
+    for (int k = 0; k < n_items; ++k) {
+      const int b = k & 1;
+      if (!__all_sync(0xffffffffu, hash_wait(&q_empty[b], ((k >> 1) & 1) ^ 1, &abort_s))) break;
+      const int tok0 = (c + k * a.ctas_per_group) * 128;
+      uint8_t* dst = q_s + b * 16384;
+      for (int e = lane; e < 128 * 8; e += 32) {
+        const int row = e >> 3, ch = e & 7;
+        const int tok = tok0 + row;
+        if (tok < a.n_tok)
+          tc::cp_async16(tc::smem_u32(dst + tc::sw128_offset(row, ch)),
+                         a.Q + (size_t)tok * 64 + ch * 8);
+        else
+          *reinterpret_cast<uint4*>(dst + tc::sw128_offset(row, ch)) = make_uint4(0, 0, 0, 0);
+      }
+      tc::cp_async_commit();
+      tc::cp_async_wait<0>();
+      tc::fence_async_smem();
+      tc::mbar_arrive(&q_full[b]);
+    }
+  } else if (warp == 16) {
+    // ------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, 256, 0, 0);
+      for (int n = 0; n < n_jobs; ++n) {
+        const int k = n / T, t = n % T, b = n & 1;
+        if (t == 0 && !hash_wait(&q_full[k & 1], (k >> 1) & 1, &abort_s)) break;
+        if (!hash_wait(&buf_empty[b], ((n >> 1) & 1) ^ 1, &abort_s)) break;
+        tc::fence_after_sync();
+        const uint32_t qa = tc::smem_u32(q_s + (k & 1) * 16384);
+        const uint32_t ra = tc::smem_u32(rot_s + (size_t)t * 256 * 128);
+        const uint32_t d = tmem + b * 256;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16(d, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                       tc::sdesc_sw128(ra + kk * 32, 16, 1024), idesc, kk > 0);
+        tc::mma_commit(&buf_full[b]);
+        if (t == T - 1) tc::mma_commit(&q_empty[k & 1]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------- epilogue
+    const int w = warp >> 2, row = tid & 127;
+    const int pb = w >> 1, h = w & 1;  // buffer of the pair, round of each job
+    uint8_t* slot = park + tid * 64;
+    const int sw = tid & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    uint32_t phase = 0;
+    for (int n = pb; n < n_jobs; n += 2, phase ^= 1u) {
+      const int k = n / T, t = n % T;
+      if (!__all_sync(0xffffffffu, hash_wait(&buf_full[pb], phase, &abort_s))) break;
+      tc::fence_after_sync();
+      const int tok = (c + k * a.ctas_per_group) * 128 + row;
+      const uint32_t pos = (uint32_t)(tok % a.L);
+      const int rl = 2 * t + h;  // round of this warpgroup's 128 columns
+      const uint32_t ta = lane_base + pb * 256 + h * kHalf;
+      ArgmaxState st;
+      st.reset();
+#pragma unroll 1
+      for (int i = 0; i < kHalf / kHash4Batch; ++i) {
+        float va[kHash4Batch];
+        tc::tmem_ld32(ta + i * kHash4Batch, va);
+        tc::tmem_ld_wait();
+        tc::tmem_pin<kHash4Batch>(va);
+        if (i == kHalf / kHash4Batch - 1) {  // the round is read: free the buffer half
+          tc::fence_before_sync();
+          tc::mbar_arrive(&buf_empty[pb]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < kHash4Batch / CW; ++ch)
+          argmax_update<CW>(st, va + ch * CW, i * kHash4Batch + ch * CW, kHalf, slot, sw);
+      }
+      const int bkt = argmax_finish<CW>(st, kHalf, slot, sw);
+      if (tok < a.n_tok) {
+        const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
+        a.keys[o] = (uint32_t)bkt * (uint32_t)a.L + pos;
+        if (a.buckets) a.buckets[o] = bkt;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 16) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace lsh

@@ -161,8 +161,17 @@ lsh_status hash_tc_launch(const Dims& D, const void* Q, const void* rot, uint32_
   if (per < 1) per = 1;
   if (per > a.n_mtiles) per = a.n_mtiles;
   a.ctas_per_group = per;
-  const size_t smem = lsh::hash_tc_smem_bytes(rg, a.half);
   const unsigned grid = (unsigned)(a.n_groups * per);
+  // four epilogue warpgroups when a round is 128 columns and every group
+  // holds an even number of rounds (R even makes rg and the last group even)
+  if (a.half == 128 && D.R % 2 == 0 && rg % 2 == 0) {
+    const size_t smem4 = lsh::hash_tc4_smem_bytes(rg);
+    lsh_status s0 = allow_smem(lsh::hash_tc4_kernel, smem4);
+    if (s0 != LSH_OK) return s0;
+    lsh::hash_tc4_kernel<<<grid, lsh::kHash4Threads, smem4, st>>>(a);
+    return last_launch();
+  }
+  const size_t smem = lsh::hash_tc_smem_bytes(rg, a.half);
   if (a.half >= 32) {
     lsh_status s0 = allow_smem(lsh::hash_tc_kernel<32>, smem);
     if (s0 != LSH_OK) return s0;
@@ -354,11 +363,13 @@ lsh_status combine_launch(const Dims& D, const float* o_part, const float* lse_r
   return last_launch();
 }
 
+// f32_out: dQ and dV are written as fp32 (for callers inside the library
+// that add them up before any rounding), else in the shape's dtype.
 template <typename T>
 lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const void* O,
                              const void* dO, const uint32_t* keys, const int32_t* perm,
                              const float* lse, void* dQ, void* dV, void* ws, size_t ws_bytes,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool f32_out = false) {
   if (!ws || ws_bytes < bwd_ws_bytes(D)) return LSH_ERR_WORKSPACE;
   const lsh::AttnDims a = attn_dims(D);
   char* w = static_cast<char*>(ws);
@@ -416,8 +427,13 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
         1.f / (float)D.R, dq, dk, dv);
   }
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv, D.n_tok,
-                                                  static_cast<T*>(dQ), static_cast<T*>(dV));
+  if (f32_out)
+    lsh::bwd_finalize_kernel<T, float><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv,
+                                                           D.n_tok, static_cast<float*>(dQ),
+                                                           static_cast<float*>(dV));
+  else
+    lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv, D.n_tok,
+                                                    static_cast<T*>(dQ), static_cast<T*>(dV));
   return last_launch();
 }
 
@@ -990,8 +1006,8 @@ RevLayout rev_layout(const lsh_shape* shape, const Dims& D, int32_t d_ff, int32_
   l.g = take(n * 2);
   l.dyb = take(n * 2);
   l.dO = take(n * 2);
-  l.dq = take(n * 2);
-  l.dv = take(n * 2);
+  l.dq = take(n * 4);  // the attention's input gradients in fp32
+  l.dv = take(n * 4);
   l.attn_bytes = lsh_workspace_size(shape);
   l.attn = take(l.attn_bytes);
   const int T = D.B * D.L, Dm = D.H * kHeadDim;
@@ -1097,10 +1113,12 @@ lsh_status lsh_rev_backward(const lsh_shape* shape, int32_t d_ff, int32_t ffn_ch
   // dX2 = dY2 + F'(X2)^T dX1: the attention's query and value gradients
   lsh::rev_to_heads_kernel<<<blocks8(n8), 256, 0, st>>>(r, dX1, bf(l.dO));
   if ((s = last_launch()) != LSH_OK) return s;
-  s = lsh_attend_bwd(shape, bf(l.x2h), bf(l.x2h), bf(l.o), bf(l.dO), keys, perm, lse, bf(l.dq),
-                     bf(l.dv), w + l.attn, l.attn_bytes, stream);
+  s = attend_bwd_launch<__nv_bfloat16>(D, bf(l.x2h), bf(l.x2h), bf(l.o), bf(l.dO), keys, perm,
+                                       lse, w + l.dq, w + l.dv, w + l.attn, l.attn_bytes, st,
+                                       true);
   if (s != LSH_OK) return s;
-  lsh::rev_grad_x2_kernel<<<blocks8(n8), 256, 0, st>>>(r, dY2, bf(l.dq), bf(l.dv), dX2);
+  lsh::rev_grad_x2_kernel<<<blocks8(n8), 256, 0, st>>>(r, dY2, reinterpret_cast<float*>(w + l.dq),
+                                                       reinterpret_cast<float*>(w + l.dv), dX2);
   return last_launch();
 }
 

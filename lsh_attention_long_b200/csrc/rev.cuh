@@ -81,8 +81,7 @@ __global__ void rev_residual_kernel(size_t n8, const float* __restrict__ a,
 // dx2[b, l, h, :] = dy2[b, l, h, :] + dq[b, h, l, :] + dv[b, h, l, :]: the
 // attention's input is both its query and its value
 __global__ void rev_grad_x2_kernel(RevDims r, const float* __restrict__ dy2,
-                                   const __nv_bfloat16* __restrict__ dq,
-                                   const __nv_bfloat16* __restrict__ dv,
+                                   const float* __restrict__ dq, const float* __restrict__ dv,
                                    float* __restrict__ dx2) {
   const size_t g8 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g8 >= (size_t)r.B * r.H * r.L * 8) return;

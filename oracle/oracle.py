@@ -237,23 +237,29 @@ def rev_forward(X1, X2, rot, n_buckets, H, chunk, causal, W1, b1, W2, b2, ffn_ch
     return Y1, Y2, keys, perm
 
 
-def rev_backward(Y1, Y2, dY1, dY2, keys, perm, H, chunk, causal, W1, b1, W2, b2, ffn_chunk):
+def rev_backward(Y1, Y2, dY1, dY2, keys, perm, H, chunk, causal, W1, b1, W2, b2, ffn_chunk,
+                 g_input=None, f_upstream=None):
     """Backward of the reversible block from its outputs alone: the inputs
     are recomputed (X2 = Y2 - G(Y1), X1 = Y1 - F(X2)), not stored.  With the
     buckets held constant:
       dY1' = dY1 + G'(Y1)^T dY2,   dX2 = dY2 + F'(X2)^T dY1',   dX1 = dY1',
     and the feed-forward's weight and bias gradients.  F'(x)^T g is the sum
-    of the attention's query and value gradients (both are x).
+    of the attention's query and value gradients (both are x).  `g_input`
+    (default Y1) is the input G is evaluated at, for a comparison with an
+    implementation that feeds G a rounded copy of Y1: G's max(0, .) then
+    takes the same decisions on both sides; `f_upstream` (default dY1') is the
+    upstream gradient F's backward is given, likewise.
     Returns X1, X2, dX1, dX2, dW1, db1, dW2, db2."""
     Y1, Y2, dY1, dY2 = (_f64(a) for a in (Y1, Y2, dY1, dY2))
     B, L, D = Y1.shape
     T = B * L
-    X2 = Y2 - ffn_forward(Y1.reshape(T, D), W1, b1, W2, b2, ffn_chunk).reshape(B, L, D)
-    gY1, dW1, db1, dW2, db2 = ffn_backward(Y1.reshape(T, D), W1, b1, W2, dY2.reshape(T, D),
-                                           ffn_chunk)
+    gin = (Y1 if g_input is None else _f64(g_input)).reshape(T, D)
+    X2 = Y2 - ffn_forward(gin, W1, b1, W2, b2, ffn_chunk).reshape(B, L, D)
+    gY1, dW1, db1, dW2, db2 = ffn_backward(gin, W1, b1, W2, dY2.reshape(T, D), ffn_chunk)
     dY1p = dY1 + gY1.reshape(B, L, D)
     X1 = Y1 - rev_attention(X2, keys, perm, H, chunk, causal)
     q = _heads(X2, H)
-    dQ, dV = lsh_attend_bwd(q, q, _heads(dY1p, H), keys, perm, chunk, causal)
+    up = dY1p if f_upstream is None else _f64(f_upstream)
+    dQ, dV = lsh_attend_bwd(q, q, _heads(up, H), keys, perm, chunk, causal)
     dX2 = dY2 + _tokens(dQ + dV)
     return X1, X2, dY1p, dX2, dW1, db1, dW2, db2

@@ -414,6 +414,11 @@ def test_empty_batch_is_a_no_op():
     (1, 2, 512, 256, 3),    # 3 * 128 columns: groups of two rounds, then one
     (1, 1, 384, 512, 9),    # 9 * 256: one round per N-tile, two groups
     (1, 1, 256, 2048, 2),   # nb/2 = 1024: four N-tiles per round
+    (2, 2, 256, 256, 4),    # nb/2 = 128, even rounds: four epilogue warpgroups, a round each
+    (1, 3, 320, 256, 2),    # the same kernel, one round pair, ragged token tiles
+    (1, 1, 256, 256, 10),   # the same kernel, groups of eight rounds and of two
+    (1, 3, 320, 512, 5),    # nb/2 = 256, odd rounds, ragged token tiles
+    (1, 3, 320, 1024, 2),   # nb/2 = 512: two N-tiles per round, ragged token tiles
 ])
 def test_tensor_core_hash_shapes(oracle, B, H, Lx, nb, R):
     inp = W.make_random(B, H, Lx, 64, nb, R, torch.bfloat16, seed=nb + R)

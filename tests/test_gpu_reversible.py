@@ -10,7 +10,10 @@ buckets of X2's hash are held constant in the backward.
 Each sublayer is compared with the fp64 oracle fed the input the GPU used
 (the GPU's buckets for F, the bf16 copy of Y1 for G), so that a near-tie
 bucket flip or a bf16 rounding upstream cannot masquerade as an error of the
-sublayer.  bf16 sublayers with fp32 accumulation: max-abs 2e-2; parameter
+sublayer: G's max(0, .) is a decision floating point takes, and a
+pre-activation within a bf16 rounding of zero would otherwise switch a
+hidden unit's whole gradient on one side only.  F's backward likewise gets
+the bf16 copy of dX1 that the GPU's attention backward consumes.  bf16 sublayers with fp32 accumulation: max-abs 2e-2; parameter
 gradients (sums over every position) relative to their largest entry.
 """
 
@@ -79,9 +82,12 @@ def _check(oracle, c, H, nb, chunk, causal, fchunk, parity_record=None, name=Non
     y1b = _np(Y1.to(torch.bfloat16)).reshape(B * Lx, D)
     Y2_ref = X2 + oracle.ffn_forward(y1b, W1, b1, W2, b2, fchunk).reshape(B, Lx, D)
     err["Y2"] = float(np.abs(_np(Y2) - Y2_ref).max())
-    # backward from the GPU's outputs, the oracle in fp64
+    # backward from the GPU's outputs, the oracle in fp64, G evaluated at the
+    # bf16 copy of Y1 the GPU fed it (its max(0, .) mask is decided there)
     ref = oracle.rev_backward(_np(Y1), _np(Y2), _np(c["dY1"]), _np(c["dY2"]), keys_np, perm_np,
-                              H, chunk, causal, W1, b1, W2, b2, fchunk)
+                              H, chunk, causal, W1, b1, W2, b2, fchunk,
+                              g_input=y1b.reshape(B, Lx, D),
+                              f_upstream=_np(dX1.to(torch.bfloat16)))
     err["X1"] = float(np.abs(_np(X1r) - X1).max())
     err["X2"] = float(np.abs(_np(X2r) - X2).max())
     err["dX1"] = float(np.abs(_np(dX1) - ref[2]).max())
