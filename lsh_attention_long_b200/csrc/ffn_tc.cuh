@@ -76,22 +76,6 @@ __host__ __device__ inline size_t gemm_tc_smem_bytes() {
   return 1024 + (size_t)kGmStages * (kGmABytes + kGmBBytes) + sizeof(GemmSmem);
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc::smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-// 2-D tiled TMA load of the box at (x = inner coordinate, y = row) into
-// shared memory, completing on `bar` with its byte count.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(tc::smem_u32(bar))
-      : "memory");
-}
-
 // Waits for a phase unless the CTA aborted; false on abort or timeout.
 __device__ __forceinline__ bool gm_wait(uint64_t* bar, uint32_t parity, int* abort,
                                         long long limit) {
@@ -157,20 +141,20 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         for (int ks = k_lo; ks < k_hi; ++ks, ++q) {
           const int s = q % kGmStages;
           if (!gm_wait(&S.empty[s], ((q / kGmStages) & 1u) ^ 1u, &S.abort, limit)) break;
-          mbar_expect_tx(&S.full[s], kGmABytes + kGmBBytes);
+          tc::mbar_expect_tx(&S.full[s], kGmABytes + kGmBBytes);
           const uint32_t sa = tc::smem_u32(stage_a + s * kGmABytes);
           const uint32_t sb = tc::smem_u32(stage_b + s * kGmBBytes);
           if (!g.a_mn) {  // one box: 64 K x 128 rows
-            tma_load_2d(sa, &map_a, ks * kGmBK, g.a_row0 + m0, &S.full[s]);
+            tc::tma_load_2d(sa, &map_a, ks * kGmBK, g.a_row0 + m0, &S.full[s]);
           } else {        // two boxes: 64 M x 64 K rows each
             for (int h = 0; h < kGmBM / 64; ++h)
-              tma_load_2d(sa + h * 8192, &map_a, m0 + 64 * h, g.a_row0 + ks * kGmBK, &S.full[s]);
+              tc::tma_load_2d(sa + h * 8192, &map_a, m0 + 64 * h, g.a_row0 + ks * kGmBK, &S.full[s]);
           }
           if (!g.b_mn) {
-            tma_load_2d(sb, &map_b, ks * kGmBK, g.b_row0 + n0, &S.full[s]);
+            tc::tma_load_2d(sb, &map_b, ks * kGmBK, g.b_row0 + n0, &S.full[s]);
           } else {
             for (int h = 0; h < kGmBN / 64; ++h)
-              tma_load_2d(sb + h * 8192, &map_b, n0 + 64 * h, g.b_row0 + ks * kGmBK, &S.full[s]);
+              tc::tma_load_2d(sb + h * 8192, &map_b, n0 + 64 * h, g.b_row0 + ks * kGmBK, &S.full[s]);
           }
         }
       }

@@ -25,7 +25,7 @@
 // columns resident in shared memory (transposed to K-major, 128B-swizzled,
 // <= 128 KB) and streams 128-token Q tiles.  Warp roles, synchronised only
 // by mbarriers (no block-wide barrier in the steady state):
-//   warp 9      loads Q tiles (cp.async) into two buffers;
+//   warp 9      loads Q tiles (one TMA copy each) into two buffers;
 //   warp 8      one thread issues the MMAs of each N-tile (<= 256 columns)
 //               into one of two 256-column TMEM buffers;
 //   warps 0-7   two epilogue warpgroups; a whole round goes to one of them
@@ -159,7 +159,8 @@ __device__ __forceinline__ bool hash_wait(uint64_t* bar, uint32_t parity, int* a
 }
 
 template <int CW>
-__global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a) {
+__global__ void __launch_bounds__(kHashTcThreads, 1)
+    hash_tc_kernel(const __grid_constant__ CUtensorMap map_q, HashTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // buf_full[w][b]: a job for warpgroup w landed in TMEM buffer b.  Each
   // warpgroup has its own pair, so it waits on every phase of the barriers
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
       tc::mbar_init(&buf_full[0][b], 1);
       tc::mbar_init(&buf_full[1][b], 1);
       tc::mbar_init(&buf_empty[b], 128);
-      tc::mbar_init(&q_full[b], 32);
+      tc::mbar_init(&q_full[b], 1);  // the TMA issuer's arrive
       tc::mbar_init(&q_empty[b], 1);
     }
     tc::mbar_init_fence();
@@ -232,27 +233,18 @@ __global__ void __launch_bounds__(kHashTcThreads, 1) hash_tc_kernel(HashTcArgs a
 
   if (warp == 9) {
     // ------------------------------------------------------- Q tile loads
-    for (int k = 0; k < n_items; ++k) {
-      const int b = k & 1;
-      if (!__all_sync(0xffffffffu, hash_wait(&q_empty[b], ((k >> 1) & 1) ^ 1, &abort_s))) break;
-      const int tok0 = (c + k * a.ctas_per_group) * 128;
-      uint8_t* dst = q_s + b * 16384;
-      for (int e = lane; e < 128 * 8; e += 32) {
-        const int row = e >> 3, ch = e & 7;
-        const int tok = tok0 + row;
-        if (tok < a.n_tok)
-          tc::cp_async16(tc::smem_u32(dst + tc::sw128_offset(row, ch)),
-                         a.Q + (size_t)tok * 64 + ch * 8);
-        else
-          *reinterpret_cast<uint4*>(dst + tc::sw128_offset(row, ch)) = make_uint4(0, 0, 0, 0);
+    // one TMA copy per 128-token tile (16 KB, 128B-swizzled: the MMA's
+    // K-major layout); rows past the last token read as zeros
+    if (lane == 0) {
+      for (int k = 0; k < n_items; ++k) {
+        const int b = k & 1;
+        if (!hash_wait(&q_empty[b], ((k >> 1) & 1) ^ 1, &abort_s)) break;
+        tc::mbar_expect_tx(&q_full[b], 16384);
+        tc::tma_load_2d(tc::smem_u32(q_s + b * 16384), &map_q, 0,
+                        (c + k * a.ctas_per_group) * 128, &q_full[b]);
       }
-      // the rows land, then become visible to the tensor cores' (async proxy)
-      // reads, then the tile is published
-      tc::cp_async_commit();
-      tc::cp_async_wait<0>();
-      tc::fence_async_smem();
-      tc::mbar_arrive(&q_full[b]);
     }
+    __syncwarp();
   } else if (warp == 8) {
     // ------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -362,7 +354,8 @@ __host__ __device__ inline size_t hash_tc4_smem_bytes(int rounds_per_group) {
   return 1024 + (size_t)rounds_per_group * 128 * 128 + 2 * 16384 + 512 * 64;
 }
 
-__global__ void __launch_bounds__(kHash4Threads, 1) hash_tc4_kernel(HashTcArgs a) {
+__global__ void __launch_bounds__(kHash4Threads, 1)
+    hash_tc4_kernel(const __grid_constant__ CUtensorMap map_q, HashTcArgs a) {
   constexpr int CW = 16;
   constexpr int kHalf = 128;
   extern __shared__ uint8_t smem_raw[];
@@ -387,7 +380,7 @@ __global__ void __launch_bounds__(kHash4Threads, 1) hash_tc4_kernel(HashTcArgs a
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&buf_full[b], 1);
       tc::mbar_init(&buf_empty[b], 256);  // both warpgroups of the buffer's pair
-      tc::mbar_init(&q_full[b], 32);
+      tc::mbar_init(&q_full[b], 1);  // the TMA issuer's arrive
       tc::mbar_init(&q_empty[b], 1);
     }
     tc::mbar_init_fence();
@@ -424,25 +417,16 @@ __global__ void __launch_bounds__(kHash4Threads, 1) hash_tc4_kernel(HashTcArgs a
 
   if (warp == 17) {
     // ------------------------------------------------------- Q tile loads
-    for (int k = 0; k < n_items; ++k) {
-      const int b = k & 1;
-      if (!__all_sync(0xffffffffu, hash_wait(&q_empty[b], ((k >> 1) & 1) ^ 1, &abort_s))) break;
-      const int tok0 = (c + k * a.ctas_per_group) * 128;
-      uint8_t* dst = q_s + b * 16384;
-      for (int e = lane; e < 128 * 8; e += 32) {
-        const int row = e >> 3, ch = e & 7;
-        const int tok = tok0 + row;
-        if (tok < a.n_tok)
-          tc::cp_async16(tc::smem_u32(dst + tc::sw128_offset(row, ch)),
-                         a.Q + (size_t)tok * 64 + ch * 8);
-        else
-          *reinterpret_cast<uint4*>(dst + tc::sw128_offset(row, ch)) = make_uint4(0, 0, 0, 0);
+    if (lane == 0) {
+      for (int k = 0; k < n_items; ++k) {
+        const int b = k & 1;
+        if (!hash_wait(&q_empty[b], ((k >> 1) & 1) ^ 1, &abort_s)) break;
+        tc::mbar_expect_tx(&q_full[b], 16384);
+        tc::tma_load_2d(tc::smem_u32(q_s + b * 16384), &map_q, 0,
+                        (c + k * a.ctas_per_group) * 128, &q_full[b]);
       }
-      tc::cp_async_commit();
-      tc::cp_async_wait<0>();
-      tc::fence_async_smem();
-      tc::mbar_arrive(&q_full[b]);
     }
+    __syncwarp();
   } else if (warp == 16) {
     // ------------------------------------------------------- MMA issue
     if (lane == 0) {

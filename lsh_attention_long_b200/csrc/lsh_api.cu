@@ -131,6 +131,42 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime so that the library
+// does not link the driver library itself.
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiled fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x box_rows
+// rows, 128-byte swizzled (the K-major operand layout of the MMA).
+bool bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  const EncodeTiled f = encode_tiled();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t elem[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tensor-core hash: bf16, nb/2 a power of two in [16, 1024].
 bool hash_tc_supported(const Dims& D) {
   const int half = D.nb / 2;
@@ -162,24 +198,27 @@ lsh_status hash_tc_launch(const Dims& D, const void* Q, const void* rot, uint32_
   if (per > a.n_mtiles) per = a.n_mtiles;
   a.ctas_per_group = per;
   const unsigned grid = (unsigned)(a.n_groups * per);
+  // Q as [n_tok, 64] rows, read in 128-token boxes
+  CUtensorMap mq;
+  if (!bf16_map(&mq, Q, (uint64_t)D.n_tok, 64, 128)) return LSH_ERR_CUDA;
   // four epilogue warpgroups when a round is 128 columns and every group
   // holds an even number of rounds (R even makes rg and the last group even)
   if (a.half == 128 && D.R % 2 == 0 && rg % 2 == 0) {
     const size_t smem4 = lsh::hash_tc4_smem_bytes(rg);
     lsh_status s0 = allow_smem(lsh::hash_tc4_kernel, smem4);
     if (s0 != LSH_OK) return s0;
-    lsh::hash_tc4_kernel<<<grid, lsh::kHash4Threads, smem4, st>>>(a);
+    lsh::hash_tc4_kernel<<<grid, lsh::kHash4Threads, smem4, st>>>(mq, a);
     return last_launch();
   }
   const size_t smem = lsh::hash_tc_smem_bytes(rg, a.half);
   if (a.half >= 32) {
     lsh_status s0 = allow_smem(lsh::hash_tc_kernel<32>, smem);
     if (s0 != LSH_OK) return s0;
-    lsh::hash_tc_kernel<32><<<grid, lsh::kHashTcThreads, smem, st>>>(a);
+    lsh::hash_tc_kernel<32><<<grid, lsh::kHashTcThreads, smem, st>>>(mq, a);
   } else {
     lsh_status s0 = allow_smem(lsh::hash_tc_kernel<16>, smem);
     if (s0 != LSH_OK) return s0;
-    lsh::hash_tc_kernel<16><<<grid, lsh::kHashTcThreads, smem, st>>>(a);
+    lsh::hash_tc_kernel<16><<<grid, lsh::kHashTcThreads, smem, st>>>(mq, a);
   }
   return last_launch();
 }
@@ -769,42 +808,6 @@ lsh_status lsh_attend_fwd_static(const lsh_shape* shape, const void* Q, const vo
 // ---------------------------------------------------------------------------
 
 namespace {
-
-// cuTensorMapEncodeTiled, reached through the runtime so that the library
-// does not link the driver library itself.
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_tiled() {
-  static std::once_flag once;
-  static EncodeTiled fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  });
-  return fn;
-}
-
-// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x box_rows
-// rows, 128-byte swizzled (the K-major operand layout of the MMA).
-bool bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-              uint32_t box_rows) {
-  const EncodeTiled f = encode_tiled();
-  if (!f) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t elem[2] = {1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 lsh_status ffn_check(int32_t tokens, int32_t d_model, int32_t d_ff, int32_t chunk) {
   if (tokens < 0 || d_model <= 0 || d_ff <= 0 || chunk <= 0) return LSH_ERR_INVALID_ARG;
