@@ -63,6 +63,10 @@ def parse_args():
     p.add_argument("--recall", action="store_true",
                    help="recall of LSH attention against full attention on the clustered "
                         "L=16384 workload, over rounds and bucket counts (a report)")
+    p.add_argument("--ffn", action="store_true",
+                   help="only the chunked feed-forward line (a diagnostic line)")
+    p.add_argument("--rev", action="store_true",
+                   help="only the reversible-block line (a diagnostic line)")
     p.add_argument("--shard", choices=["none", "heads"], default="none",
                    help="heads: split one problem's B*H heads over the ranks (strong "
                         "scaling) instead of a replica per rank")
@@ -756,13 +760,17 @@ def run_recall(args):
 
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-# for the kernel as it stands, keyed by (stage, workload); absent until taken,
-# and to be cleared whenever the kernel changes.  The attention kernel's figure
-# is from one capture of the L=16384 workload's forward (profiles/
-# attend_tc_kernel_fwd_bf16_L16384.md), the hash kernel's from one capture of
-# the timed step at L=65536.
+# for the kernels as they stand, keyed by (stage, workload); absent until
+# taken, and to be cleared whenever a kernel changes.  A stage's figure covers
+# the launches its time covers: the attention call is fwd_prep_kernel +
+# attend_tc_kernel + combine_kernel.  The L=65536 figures are from one
+# capture of the timed step (profiles/launches_fwd_bf16_L65536.md); the
+# L=16384 attention figure is the attention kernel alone, from one capture of
+# that workload's forward (profiles/attend_tc_kernel_fwd_bf16_L16384.md).
 TRAFFIC = {
-    ("hash", "fwd_bf16_L65536"): 67665000 + 4091648,
+    ("hash", "fwd_bf16_L65536"): 67664896 + 2832384,
+    ("attend", "fwd_bf16_L65536"): (134223360 + 32006144) + (180196352 + 497440256)
+                                   + (553665792 + 58548736),
     ("attend", "fwdbwd_bf16_L16384"): 77895168 + 90932992,
 }
 
@@ -963,6 +971,15 @@ def main():
         if args.fwd_bwd:
             res = {"workload": args.workload,
                    "fwd_bwd": run_fwd_bwd(args, W.WORKLOADS[args.workload], world)}
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
+        if args.ffn or args.rev:
+            res = {}
+            if args.ffn:
+                res["ffn"] = run_ffn(args, world)
+            if args.rev:
+                res["reversible"] = run_rev(args, world)
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return

@@ -64,7 +64,10 @@ struct GemmArgs {
   long long wait_limit;
 };
 
+constexpr int kGmStageOutBytes = 4 * 32 * 128;  // per epilogue warp: 32 rows of 128 B
+
 struct GemmSmem {
+  float bias[kGmBN];  // the output tile's bias columns (kEpiBiasAct)
   uint64_t full[kGmStages], empty[kGmStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
@@ -73,7 +76,26 @@ struct GemmSmem {
 };
 
 __host__ __device__ inline size_t gemm_tc_smem_bytes() {
-  return 1024 + (size_t)kGmStages * (kGmABytes + kGmBBytes) + sizeof(GemmSmem);
+  return 1024 + (size_t)kGmStages * (kGmABytes + kGmBBytes) + kGmStageOutBytes +
+         sizeof(GemmSmem);
+}
+
+// OR of pred over the 128 epilogue threads (named barrier 2).
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Waits for a phase unless the CTA aborted; false on abort or timeout.
@@ -99,7 +121,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* stage_a = sm;
   uint8_t* stage_b = sm + kGmStages * kGmABytes;
-  GemmSmem& S = *reinterpret_cast<GemmSmem*>(stage_b + kGmStages * kGmBBytes);
+  uint8_t* stage_out = stage_b + kGmStages * kGmBBytes;
+  GemmSmem& S = *reinterpret_cast<GemmSmem*>(stage_out + kGmStageOutBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long limit = g.wait_limit;
 
@@ -217,20 +240,48 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each thread owns one output row (its TMEM lane) and works 32 columns
+    // at a time.  Per-row operands (mask, residual) are loaded before the
+    // TMEM load they are combined with; the bias of the tile sits in shared
+    // memory.  Results go through this warp's staging rows (16-byte pieces
+    // rotated by row) and leave eight lanes per 128-byte row: bf16 rows
+    // every 64 columns, fp32 rows (stores or reductions) every 32.
     const int sub = warp & 3;  // TMEM lanes 32*sub .. 32*sub+31
     const int row_in_tile = sub * 32 + lane;
+    const int et = tid - 64;   // 0..127 over the epilogue warps
+    uint8_t* stg = stage_out + sub * (32 * 128);
+    uint8_t* my_row = stg + lane * 128;
+    const bool f32_out = g.epi == kEpiAddF32 || g.epi == kEpiAtomicF32;
     uint32_t i = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++i) {
       const int t = u / g.k_splits;
       const int b = i & 1;
       const int m0 = (t / n_n) * kGmBM, n0 = (t % n_n) * kGmBN;
+      if (g.epi == kEpiBiasAct) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the last tile's bias is read
+        for (int c = et; c < kGmBN; c += 128) S.bias[c] = __bfloat162float(g.bias[n0 + c]);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
       const bool okw = gm_wait(&S.acc_full[b], (i >> 1) & 1u, &S.abort, limit);
-      if (!__all_sync(0xffffffffu, okw)) break;
+      // all four epilogue warps leave together (they share named barriers)
+      if (epi_any(!okw)) break;
       tc::fence_after_sync();
       const uint32_t taddr = tmem + b * 256 + ((uint32_t)(sub * 32) << 16);
       const size_t row = (size_t)(m0 + row_in_tile);
 #pragma unroll 1
       for (int c = 0; c < kGmBN / 32; ++c) {
+        const int col = n0 + 32 * c;
+        uint4 mk[4];
+        float4 rr[8];
+        if (g.epi == kEpiMask) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mk[q] = *reinterpret_cast<const uint4*>(g.mask + row * g.ldm + col + 8 * q);
+        } else if (g.epi == kEpiAddF32 && g.R) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            rr[q] = *reinterpret_cast<const float4*>(g.R + row * g.ldr + col + 4 * q);
+        }
         float v[32];
         tc::tmem_ld32(taddr + 32 * c, v);
         tc::tmem_ld_wait();
@@ -239,39 +290,64 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           tc::fence_before_sync();
           tc::mbar_arrive(&S.acc_empty[b]);
         }
-        const int col = n0 + 32 * c;
+        if (g.epi == kEpiBiasAct) {
+          const float* bs = S.bias + 32 * c;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float* x = v + 8 * q;
-          if (g.epi == kEpiBiasAct) {
-            float bias[8];
-            load8(g.bias + col + 8 * q, bias);
+          for (int e = 0; e < 32; ++e) v[e] = g.relu ? fmaxf(v[e] + bs[e], 0.f) : v[e] + bs[e];
+        } else if (g.epi == kEpiMask) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = g.relu ? fmaxf(x[e] + bias[e], 0.f) : x[e] + bias[e];
-            store8(g.C + row * g.ldc + col + 8 * q, x);
-          } else if (g.epi == kEpiMask) {
-            float mk[8];
-            load8(g.mask + row * g.ldm + col + 8 * q, mk);
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat16* m8 = reinterpret_cast<const __nv_bfloat16*>(&mk[q]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = mk[e] > 0.f ? x[e] : 0.f;
-            store8(g.C + row * g.ldc + col + 8 * q, x);
-          } else if (g.epi == kEpiAddF32) {
-            if (g.R) {
-              float r[8];
-              load8(g.R + row * g.ldr + col + 8 * q, r);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] += r[e];
-            }
-            store8(g.C32 + row * g.ldc32 + col + 8 * q, x);
-          } else {
-            float* dst = g.C32 + row * g.ldc32 + col + 8 * q;
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(x[0]),
-                         "f"(x[1]), "f"(x[2]), "f"(x[3])
-                         : "memory");
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4), "f"(x[4]),
-                         "f"(x[5]), "f"(x[6]), "f"(x[7])
-                         : "memory");
+            for (int e = 0; e < 8; ++e)
+              v[8 * q + e] = __bfloat162float(m8[e]) > 0.f ? v[8 * q + e] : 0.f;
           }
+        } else if (g.epi == kEpiAddF32 && g.R) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            v[4 * q] += rr[q].x; v[4 * q + 1] += rr[q].y;
+            v[4 * q + 2] += rr[q].z; v[4 * q + 3] += rr[q].w;
+          }
+        }
+        if (!f32_out) {
+          // 32 bf16 = 64 B: pieces 4(c&1) .. 4(c&1)+3 of the staging row
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int p = 4 * (c & 1) + q;
+            *reinterpret_cast<uint4*>(my_row + ((p ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          }
+          if ((c & 1) == 0) continue;
+          __syncwarp();
+          const int col0 = n0 + 64 * (c >> 1);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rl = 4 * k + (lane >> 3), p = lane & 7;
+            const uint4 w = *reinterpret_cast<const uint4*>(stg + rl * 128 + ((p ^ (rl & 7)) << 4));
+            *reinterpret_cast<uint4*>(g.C + (size_t)(m0 + sub * 32 + rl) * g.ldc + col0 + 8 * p) = w;
+          }
+          __syncwarp();
+        } else {
+          // 32 fp32 = 128 B: the whole staging row
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(my_row + ((q ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rl = 4 * k + (lane >> 3), p = lane & 7;
+            const float4 w = *reinterpret_cast<const float4*>(stg + rl * 128 + ((p ^ (rl & 7)) << 4));
+            float* dst = g.C32 + (size_t)(m0 + sub * 32 + rl) * g.ldc32 + col + 4 * p;
+            if (g.epi == kEpiAddF32)
+              *reinterpret_cast<float4*>(dst) = w;
+            else
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(w.x),
+                           "f"(w.y), "f"(w.z), "f"(w.w)
+                           : "memory");
+          }
+          __syncwarp();
         }
       }
     }

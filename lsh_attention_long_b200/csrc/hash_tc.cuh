@@ -452,8 +452,11 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
     // ------------------------------------------------------- epilogue
     const int w = warp >> 2, row = tid & 127;
     const int pb = w >> 1, h = w & 1;  // buffer of the pair, round of each job
+    // 64-byte slots: the eight lanes of a quarter-warp take two slot bases
+    // (tid & 1) and four piece rotations ((tid >> 1) & 3), so a 16-byte
+    // store of piece q lands on eight distinct bank groups
     uint8_t* slot = park + tid * 64;
-    const int sw = tid & 3;
+    const int sw = (tid >> 1) & 3;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t phase = 0;
     for (int n = pb; n < n_jobs; n += 2, phase ^= 1u) {
