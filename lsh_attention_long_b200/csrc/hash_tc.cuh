@@ -144,6 +144,11 @@ __device__ __forceinline__ int argmax_finish(const ArgmaxState& st, int half, co
   return min(chunk_candidate<CW>(v, st.best, st.bc, half), st.tie_cand);
 }
 
+// Named barrier (id 1 + w) over the 128 threads of warpgroup w.
+__device__ __forceinline__ void wg_sync(int w) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+}
+
 // Bounded mbarrier wait that also gives up once the CTA has aborted.
 __device__ __forceinline__ bool hash_wait(uint64_t* bar, uint32_t parity, int* abort) {
   const long long t0 = clock64();
@@ -335,29 +340,40 @@ __global__ void __launch_bounds__(kHashTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Four epilogue warpgroups, for nb/2 = 128 and an even number of rounds per
-// group.  Every job (128 tokens x two rounds = 256 columns in one of two TMEM
-// buffers) is read by the pair of warpgroups of its buffer, one round each,
-// so four epilogue warps share each SM sub-partition instead of two and every
-// warpgroup finishes the exact argmax of a whole round on its own.  Measured
-// against the two-warpgroup kernel (same keys): 10% faster at nb = 256, but
-// slower at nb = 1024, where a round's 512 columns would be split over four
-// warpgroups and their partial maxima merged.
+// Four epilogue warpgroups (nb/2 = 128, 256 or 512; every N-tile 256 columns
+// wide).  Each job (128 tokens x 256 columns in one of two TMEM buffers) is
+// read by the two warpgroups of its buffer's pair, 128 columns each, so four
+// epilogue warps share each SM sub-partition instead of two.  A round's
+// columns then fall to one warpgroup (nb/2 = 128), to a pair (256) or to all
+// four (512); each keeps the exact partial argmax of its columns (largest
+// |p|, then its lowest bucket candidate), and the last warpgroup to finish a
+// round merges the partials through shared memory: the largest |p| wins,
+// equal ones go to the lowest candidate, the same first index of the maximum
+// of [p ; -p] as one scan of the whole round.  Measured against the
+// two-warpgroup kernel (same keys): 0.514 against 0.541 ms at 1024 buckets
+// and 8 rounds, 0.039 against 0.051 ms at 256 buckets and 4 rounds.
 // ---------------------------------------------------------------------------
 
 constexpr int kHash4Threads = 576;  // four epilogue warpgroups, MMA warp, Q loader
 constexpr int kHash4Batch = 32;     // TMEM columns read per wait
+constexpr int kHash4Slots = 4;      // rounds whose partials may be in flight
 
-__host__ __device__ inline size_t hash_tc4_smem_bytes(int rounds_per_group) {
-  // alignment slack, rotation columns (128 per round), two Q tiles, 64 bytes
-  // of parking per epilogue thread
-  return 1024 + (size_t)rounds_per_group * 128 * 128 + 2 * 16384 + 512 * 64;
+struct Hash4Merge {
+  float best[kHash4Slots][4][128];
+  int cand[kHash4Slots][4][128];
+  unsigned cnt[kHash4Slots];
+  int last[4];
+};
+
+__host__ __device__ inline size_t hash_tc4_smem_bytes(int rounds_per_group, int half) {
+  // alignment slack, rotation columns, two Q tiles, 64 bytes of parking per
+  // epilogue thread, the merge slots
+  return 1024 + (size_t)rounds_per_group * half * 128 + 2 * 16384 + 512 * 64 + sizeof(Hash4Merge);
 }
 
 __global__ void __launch_bounds__(kHash4Threads, 1)
     hash_tc4_kernel(const __grid_constant__ CUtensorMap map_q, HashTcArgs a) {
   constexpr int CW = 16;
-  constexpr int kHalf = 128;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t buf_full[2], buf_empty[2], q_full[2], q_empty[2];
   __shared__ uint32_t tmem_base_s;
@@ -370,21 +386,23 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
   const int c = blockIdx.x / a.n_groups;
   const int r0 = g * a.rounds_per_group;
   const int nr = min(a.rounds_per_group, a.R - r0);
-  const int cols = nr * kHalf;
-  const int T = cols / 256;  // N-tiles (round pairs) per token tile
+  const int cols = nr * a.half;
+  const int T = cols / 256;  // N-tiles per token tile, all 256 wide
   uint8_t* rot_s = sm;
-  uint8_t* q_s = sm + (size_t)a.rounds_per_group * kHalf * 128;
+  uint8_t* q_s = sm + (size_t)a.rounds_per_group * a.half * 128;
   uint8_t* park = q_s + 2 * 16384;
+  Hash4Merge& M = *reinterpret_cast<Hash4Merge*>(park + 512 * 64);
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&buf_full[b], 1);
       tc::mbar_init(&buf_empty[b], 256);  // both warpgroups of the buffer's pair
-      tc::mbar_init(&q_full[b], 1);  // the TMA issuer's arrive
+      tc::mbar_init(&q_full[b], 1);
       tc::mbar_init(&q_empty[b], 1);
     }
     tc::mbar_init_fence();
     abort_s = 0;
+    for (int s = 0; s < kHash4Slots; ++s) M.cnt[s] = 0;
   }
   if (warp == 16) {
     tc::tmem_alloc(&tmem_base_s, 512);
@@ -451,13 +469,16 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
   } else {
     // ------------------------------------------------------- epilogue
     const int w = warp >> 2, row = tid & 127;
-    const int pb = w >> 1, h = w & 1;  // buffer of the pair, round of each job
+    const int pb = w >> 1, h = w & 1;  // buffer of the pair, half of each job
     // 64-byte slots: the eight lanes of a quarter-warp take two slot bases
     // (tid & 1) and four piece rotations ((tid >> 1) & 3), so a 16-byte
     // store of piece q lands on eight distinct bank groups
     uint8_t* slot = park + tid * 64;
     const int sw = (tid >> 1) & 3;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int np = a.half / 128;           // 128-column pieces per round
+    const int P = np < 4 ? np : 4;         // warpgroups that share a round
+    const int half_shift = __ffs(a.half) - 1;
     uint32_t phase = 0;
     for (int n = pb; n < n_jobs; n += 2, phase ^= 1u) {
       const int k = n / T, t = n % T;
@@ -465,25 +486,55 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
       tc::fence_after_sync();
       const int tok = (c + k * a.ctas_per_group) * 128 + row;
       const uint32_t pos = (uint32_t)(tok % a.L);
-      const int rl = 2 * t + h;  // round of this warpgroup's 128 columns
-      const uint32_t ta = lane_base + pb * 256 + h * kHalf;
+      const int gc0 = t * 256 + h * 128;  // first column of this piece in the group
+      const int rl = gc0 >> half_shift, jb0 = gc0 & (a.half - 1);
+      const uint32_t ta = lane_base + pb * 256 + h * 128;
       ArgmaxState st;
       st.reset();
 #pragma unroll 1
-      for (int i = 0; i < kHalf / kHash4Batch; ++i) {
+      for (int i = 0; i < 128 / kHash4Batch; ++i) {
         float va[kHash4Batch];
         tc::tmem_ld32(ta + i * kHash4Batch, va);
         tc::tmem_ld_wait();
         tc::tmem_pin<kHash4Batch>(va);
-        if (i == kHalf / kHash4Batch - 1) {  // the round is read: free the buffer half
+        if (i == 128 / kHash4Batch - 1) {  // the piece is read: free the buffer half
           tc::fence_before_sync();
           tc::mbar_arrive(&buf_empty[pb]);
         }
 #pragma unroll
         for (int ch = 0; ch < kHash4Batch / CW; ++ch)
-          argmax_update<CW>(st, va + ch * CW, i * kHash4Batch + ch * CW, kHalf, slot, sw);
+          argmax_update<CW>(st, va + ch * CW, jb0 + i * kHash4Batch + ch * CW, a.half, slot, sw);
       }
-      const int bkt = argmax_finish<CW>(st, kHalf, slot, sw);
+      const int cand = argmax_finish<CW>(st, a.half, slot, sw);
+      int bkt = cand;
+      if (P > 1) {
+        // publish this piece's partial; the last warpgroup of the round merges
+        const int gr = k * nr + rl, ms = gr % kHash4Slots;
+        M.best[ms][w][row] = st.best;
+        M.cand[ms][w][row] = cand;
+        tc::fence_before_sync();
+        wg_sync(w);  // the warpgroup's partials are written
+        if (row == 0) {
+          __threadfence_block();
+          const unsigned old = atomicAdd(&M.cnt[ms], 1u);
+          const int is_last = old == (unsigned)(P - 1);
+          if (is_last) M.cnt[ms] = 0;  // no other contributor of this round is left
+          __threadfence_block();
+          M.last[w] = is_last;
+        }
+        wg_sync(w);
+        if (!M.last[w]) continue;
+        // contributors: the pair (P = 2) or every warpgroup (P = 4)
+        const int w0 = P == 2 ? (w & ~1) : 0;
+        float best = -1.f;
+        bkt = 0x7fffffff;
+        for (int x = w0; x < w0 + P; ++x) {
+          const float b2 = M.best[ms][x][row];
+          const int c2 = M.cand[ms][x][row];
+          if (b2 > best) { best = b2; bkt = c2; }
+          else if (b2 == best) bkt = min(bkt, c2);
+        }
+      }
       if (tok < a.n_tok) {
         const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
         a.keys[o] = (uint32_t)bkt * (uint32_t)a.L + pos;

@@ -201,10 +201,12 @@ lsh_status hash_tc_launch(const Dims& D, const void* Q, const void* rot, uint32_
   // Q as [n_tok, 64] rows, read in 128-token boxes
   CUtensorMap mq;
   if (!bf16_map(&mq, Q, (uint64_t)D.n_tok, 64, 128)) return LSH_ERR_CUDA;
-  // four epilogue warpgroups when a round is 128 columns and every group
-  // holds an even number of rounds (R even makes rg and the last group even)
-  if (a.half == 128 && D.R % 2 == 0 && rg % 2 == 0) {
-    const size_t smem4 = lsh::hash_tc4_smem_bytes(rg);
+  // four epilogue warpgroups when every N-tile is 256 columns wide: rounds
+  // of 256 or 512 columns, or of 128 in groups of an even number of rounds
+  // (R even makes rg and the last group even)
+  if ((a.half == 256 || a.half == 512 || (a.half == 128 && D.R % 2 == 0 && rg % 2 == 0)) &&
+      rg * a.half >= 256) {
+    const size_t smem4 = lsh::hash_tc4_smem_bytes(rg, a.half);
     lsh_status s0 = allow_smem(lsh::hash_tc4_kernel, smem4);
     if (s0 != LSH_OK) return s0;
     lsh::hash_tc4_kernel<<<grid, lsh::kHash4Threads, smem4, st>>>(mq, a);

@@ -417,8 +417,8 @@ def test_empty_batch_is_a_no_op():
     (2, 2, 256, 256, 4),    # nb/2 = 128, even rounds: four epilogue warpgroups, a round each
     (1, 3, 320, 256, 2),    # the same kernel, one round pair, ragged token tiles
     (1, 1, 256, 256, 10),   # the same kernel, groups of eight rounds and of two
-    (1, 3, 320, 512, 5),    # nb/2 = 256, odd rounds, ragged token tiles
-    (1, 3, 320, 1024, 2),   # nb/2 = 512: two N-tiles per round, ragged token tiles
+    (1, 3, 320, 512, 5),    # nb/2 = 256: a round shared by a pair of warpgroups, groups of 4 and 1
+    (1, 3, 320, 1024, 2),   # nb/2 = 512: a round shared by all four warpgroups, ragged token tiles
 ])
 def test_tensor_core_hash_shapes(oracle, B, H, Lx, nb, R):
     inp = W.make_random(B, H, Lx, 64, nb, R, torch.bfloat16, seed=nb + R)
