@@ -23,6 +23,7 @@ max-reduced over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -63,6 +64,10 @@ def parse_args():
     p.add_argument("--recall", action="store_true",
                    help="recall of LSH attention against full attention on the clustered "
                         "L=16384 workload, over rounds and bucket counts (a report)")
+    p.add_argument("--heads", type=int, default=0,
+                   help="run --workload with this many heads instead of its own (a "
+                        "smaller case of the same kernels, e.g. for profiling); the "
+                        "line's workload name gets an _H<heads> suffix")
     p.add_argument("--ffn", action="store_true",
                    help="only the chunked feed-forward line (a diagnostic line)")
     p.add_argument("--rev", action="store_true",
@@ -953,6 +958,11 @@ def run_reference(args, world, rank):
 
 def main():
     args = parse_args()
+    if args.heads > 0:
+        w = W.WORKLOADS[args.workload]
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_H{args.heads}")
+        W.WORKLOADS[w.name] = w
+        args.workload = w.name
     if args.impl == "reference":
         # the CPU oracle runs on rank 0 only; other ranks exit without work
         if int(os.environ.get("RANK", "0")) != 0:

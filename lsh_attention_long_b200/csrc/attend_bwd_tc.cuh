@@ -39,22 +39,26 @@
 // fp32 gradient buffers with vector reductions; they sum over tiles and
 // rounds.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3, 4-7  two compute warpgroups; warpgroup 1 takes the w1 columns
 //                   of every query row, warpgroup 0 the row's other window
 //                   chunk (w0 for q0, w2 for q1); in the drain warpgroup 0
-//                   forms the dq rows and warpgroup 1 the dv rows.
-//   warp 8          producer: gathers the tile's window (q, v rows, packed
-//                   keys, key scales) and its queries' dO rows, lse and G into
-//                   one of two shared-memory slots.
-//   warp 9          one thread issues the MMAs.
+//                   forms the dq rows and warpgroup 1 the dv rows of the
+//                   column-64+m tokens, and the other way round for the w0
+//                   tokens of lanes 0..63.
+//   warps 8, 9      producers: warp 8 + p gathers the CTA's tiles p, p + 2,
+//                   ... (window q, v rows, packed keys, key scales; the
+//                   queries' dO rows, lse and G) into shared-memory slot p.
+//   warp 10         one thread issues the MMAs.
 #pragma once
 
 #include "attend_tc.cuh"
 
 namespace lsh {
 
-constexpr int kBwThreads = 320;
+constexpr int kBwThreads = 352;
+constexpr int kBwProducerWarp = 8;  // warps 8, 9
+constexpr int kBwMmaWarp = 10;
 constexpr int kBwSlots = 2;
 constexpr int kBwChunkBytes = 64 * 128;                 // 64 rows of 128 B
 constexpr int kBwSlotBytes = 8 * kBwChunkBytes;         // q x3, v x3, dO x2
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
     tc::mbar_init_fence();
     S.abort = 0;
   }
-  if (warp == 9) {
+  if (warp == kBwMmaWarp) {
     tc::tmem_alloc(&S.tmem_base, 512);
     tc::tmem_relinquish();
   }
@@ -238,9 +242,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
   tc::fence_after_sync();
   const uint32_t tmem = S.tmem_base;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    for (uint32_t n = 0;; ++n) {
+  if (warp == kBwProducerWarp || warp == kBwProducerWarp + 1) {
+    // ------------------------------------------------------------ producers
+    // producer p fills slot p with the CTA's tiles p, p + 2, ...
+    for (uint32_t n = (uint32_t)(warp - kBwProducerWarp);; n += kBwSlots) {
       const int s = n % kBwSlots;
       const long long tile = (long long)blockIdx.x + (long long)n * gridDim.x;
       if (!__all_sync(0xffffffffu, at_wait(&S.empty[s], ((n / kBwSlots) & 1u) ^ 1u, &S.abort)))
@@ -280,6 +285,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
           record_status(kErrBadKeys);
           p = 0;
         }
+        pe[e] = p;
         S.pos[s][u] = p;
         if (p != kAtNoKey) {
           cp_async4(tc::smem_u32(&S.key[s][u]), a.keys + rowbase + p);
@@ -303,10 +309,11 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       const __nv_bfloat16* Qbh = a.Q + bhL * 64;
       const __nv_bfloat16* Vbh = a.V + bhL * 64;
       const __nv_bfloat16* dObh = a.dO + bhL * 64;
-#pragma unroll 2
+      // window column u's position is pe[u / 32] of lane u % 32
+#pragma unroll
       for (int i = 0; i < 48; ++i) {
         const int u = 4 * i + (lane >> 3), c = lane & 7;
-        const uint32_t p = S.pos[s][u];
+        const uint32_t p = __shfl_sync(0xffffffffu, pe[i >> 3], u & 31);
         uint8_t* qd = slot + tc::sw128_offset(u, c);
         uint8_t* vd = slot + 3 * kBwChunkBytes + tc::sw128_offset(u, c);
         uint8_t* dd = slot + 6 * kBwChunkBytes + tc::sw128_offset(u - 64, c);
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       __syncwarp();
       tc::mbar_arrive(&S.full[s]);
     }
-  } else if (warp == 9) {
+  } else if (warp == kBwMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t id_s = tc::idesc_bf16(128, 192, 0, 0);
@@ -505,7 +512,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
       tc::fence_after_sync();
       // drain, merged per lane: lanes 64..127 hold the w1 token of column
       // 64 + m, lanes 0..63 the w2 token of column 64 + m and the w0 token of
-      // column m; warpgroup 0 adds the dq rows, warpgroup 1 the dv rows
+      // column m
       const size_t bhL = (size_t)inf.bh * a.L;
       const bool two = inf.nq == 2;
       const uint8_t* qrows = slots + (size_t)s * kBwSlotBytes;
@@ -519,8 +526,12 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
         // accumulators holding this token on this lane
         const bool acc1 = rr == 1 || w1row;       // dV1 / dK1
         const bool acc2 = rr == 0 && (!w1row || two);  // dV2 / dK2
-        float* dst = (g == 0 ? a.dq_acc : a.dv_acc) + (bhL + S.pos[s][c]) * 64;
-        if (g == 0) drain_dq(region, rr == 0, acc1, acc2, qrows, c, S.rn[s][c] * inv_scale, dst);
+        // lanes 0..63 drain two tokens: warpgroup 0 takes the dq row of the
+        // first and the dv row of the second, warpgroup 1 the others, so both
+        // do one dq and one dv row there
+        const bool dq_row = (g == 0) == (rr == 0);
+        float* dst = (dq_row ? a.dq_acc : a.dv_acc) + (bhL + S.pos[s][c]) * 64;
+        if (dq_row) drain_dq(region, rr == 0, acc1, acc2, qrows, c, S.rn[s][c] * inv_scale, dst);
         else drain_dv(region, acc1, acc2, dst);
       }
       tc::fence_before_sync();
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kBwMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
