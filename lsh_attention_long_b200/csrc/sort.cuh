@@ -52,9 +52,10 @@ __device__ __forceinline__ uint32_t div_l(uint32_t key, DivL d) {
   return d.sh < 0 ? key : __umulhi(key, d.m) >> d.sh;
 }
 
-__device__ __forceinline__ uint32_t checked_bucket(const uint32_t* k, int t, int L, int nb,
-                                                   DivL dl, bool& bad) {
-  const uint32_t key = k[t];
+// Bucket of the key at position t, or kNoBucket (and bad) when the key is
+// not bucket * L + t with bucket < nb.
+__device__ __forceinline__ uint32_t checked_bucket(uint32_t key, int t, int L, int nb, DivL dl,
+                                                   bool& bad) {
   const uint32_t b = div_l(key, dl);
   if (b >= (uint32_t)nb || key - b * (uint32_t)L != (uint32_t)t) {
     bad = true;
@@ -91,13 +92,23 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
   bool bad = false;
 
   // pass 1: per-warp histograms (counts do not depend on order: shared-
-  // memory atomics), bucket ids kept for pass 2 when they fit
-  for (int base = begin; base < end; base += 32) {
-    const int t = base + lane;
-    if (t < end) {
-      const uint32_t b = checked_bucket(k, t, L, nb, dl, bad);
-      if (b != kNoBucket) atomicAdd(&my[b], 1u);
-      if (cache_ids) ids[t - cbeg] = b != kNoBucket ? (uint16_t)b : (uint16_t)0xffffu;
+  // memory atomics), bucket ids kept for pass 2 when they fit; each lane
+  // has four keys in flight before it counts them
+  for (int base = begin; base < end; base += 128) {
+    uint32_t kv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = base + 32 * j + lane;
+      kv[j] = t < end ? __ldg(k + t) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = base + 32 * j + lane;
+      if (t < end) {
+        const uint32_t b = checked_bucket(kv[j], t, L, nb, dl, bad);
+        if (b != kNoBucket) atomicAdd(&my[b], 1u);
+        if (cache_ids) ids[t - cbeg] = b != kNoBucket ? (uint16_t)b : (uint16_t)0xffffu;
+      }
     }
   }
   if (bad) record_status(kErrBadKeys);
@@ -175,7 +186,7 @@ sort_rows_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ perm, 
         const uint32_t c = ids[t - cbeg];
         b = c == 0xffffu ? kNoBucket : c;
       } else {
-        b = checked_bucket(k, t, L, nb, dl, dummy);
+        b = checked_bucket(k[t], t, L, nb, dl, dummy);
       }
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
