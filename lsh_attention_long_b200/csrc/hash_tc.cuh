@@ -144,11 +144,6 @@ __device__ __forceinline__ int argmax_finish(const ArgmaxState& st, int half, co
   return min(chunk_candidate<CW>(v, st.best, st.bc, half), st.tie_cand);
 }
 
-// Named barrier (id 1 + w) over the 128 threads of warpgroup w.
-__device__ __forceinline__ void wg_sync(int w) {
-  asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
-}
-
 // Bounded mbarrier wait that also gives up once the CTA has aborted.
 __device__ __forceinline__ bool hash_wait(uint64_t* bar, uint32_t parity, int* abort) {
   const long long t0 = clock64();
@@ -358,11 +353,12 @@ constexpr int kHash4Threads = 576;  // four epilogue warpgroups, MMA warp, Q loa
 constexpr int kHash4Batch = 32;     // TMEM columns read per wait
 constexpr int kHash4Slots = 4;      // rounds whose partials may be in flight
 
+// Per round slot and token row: the largest (|p| bits, ~candidate) pair of
+// the pieces merged so far (non-negative floats order as their bits; a
+// larger ~candidate is a smaller candidate), and how many pieces are in.
 struct Hash4Merge {
-  float best[kHash4Slots][4][128];
-  int cand[kHash4Slots][4][128];
-  unsigned cnt[kHash4Slots];
-  int last[4];
+  unsigned long long key[kHash4Slots][128];
+  unsigned cnt[kHash4Slots][128];
 };
 
 __host__ __device__ inline size_t hash_tc4_smem_bytes(int rounds_per_group, int half) {
@@ -402,11 +398,14 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
     }
     tc::mbar_init_fence();
     abort_s = 0;
-    for (int s = 0; s < kHash4Slots; ++s) M.cnt[s] = 0;
   }
   if (warp == 16) {
     tc::tmem_alloc(&tmem_base_s, 512);
     tc::tmem_relinquish();
+  }
+  for (int e = tid; e < kHash4Slots * 128; e += blockDim.x) {
+    M.key[e / 128][e % 128] = 0ull;
+    M.cnt[e / 128][e % 128] = 0u;
   }
   // rotation columns of this group, transposed: smem row j holds column j
   for (int row = tid; row < cols; row += blockDim.x) {
@@ -508,32 +507,18 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
       const int cand = argmax_finish<CW>(st, a.half, slot, sw);
       int bkt = cand;
       if (P > 1) {
-        // publish this piece's partial; the last warpgroup of the round merges
+        // merge this piece into the round's row; the last of its P pieces
+        // takes the result (and clears the slot for a later round)
         const int gr = k * nr + rl, ms = gr % kHash4Slots;
-        M.best[ms][w][row] = st.best;
-        M.cand[ms][w][row] = cand;
-        tc::fence_before_sync();
-        wg_sync(w);  // the warpgroup's partials are written
-        if (row == 0) {
-          __threadfence_block();
-          const unsigned old = atomicAdd(&M.cnt[ms], 1u);
-          const int is_last = old == (unsigned)(P - 1);
-          if (is_last) M.cnt[ms] = 0;  // no other contributor of this round is left
-          __threadfence_block();
-          M.last[w] = is_last;
-        }
-        wg_sync(w);
-        if (!M.last[w]) continue;
-        // contributors: the pair (P = 2) or every warpgroup (P = 4)
-        const int w0 = P == 2 ? (w & ~1) : 0;
-        float best = -1.f;
-        bkt = 0x7fffffff;
-        for (int x = w0; x < w0 + P; ++x) {
-          const float b2 = M.best[ms][x][row];
-          const int c2 = M.cand[ms][x][row];
-          if (b2 > best) { best = b2; bkt = c2; }
-          else if (b2 == best) bkt = min(bkt, c2);
-        }
+        const unsigned long long mine =
+            ((unsigned long long)__float_as_uint(st.best) << 32) | (uint32_t)~(uint32_t)cand;
+        atomicMax(&M.key[ms][row], mine);
+        __threadfence_block();
+        if (atomicAdd(&M.cnt[ms][row], 1u) != (unsigned)(P - 1)) continue;
+        __threadfence_block();
+        const unsigned long long all = atomicExch(&M.key[ms][row], 0ull);
+        M.cnt[ms][row] = 0;
+        bkt = (int)~(uint32_t)(all & 0xffffffffull);
       }
       if (tok < a.n_tok) {
         const size_t o = (size_t)(r0 + rl) * a.n_tok + tok;
