@@ -758,4 +758,44 @@ __global__ void combine_kernel(const P* __restrict__ o_part, const float* __rest
   if (lse && k == 0) lse[tok] = tot;
 }
 
+// The same for the fp16 partials with R a compile-time constant, so that all
+// R partial rows of a token are in flight before they are weighed (same
+// arithmetic, same order, as combine_kernel).
+template <int R, typename T>
+__global__ void combine16_kernel(const __half* __restrict__ o_part, const float* __restrict__ lse_r,
+                                 size_t n_tok, T* __restrict__ O, float* __restrict__ lse) {
+  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= n_tok * 8) return;
+  const size_t tok = g >> 3;
+  const int k = (int)(g & 7) * 8;
+  float l[R];
+  uint4 raw[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    l[r] = lse_r[(size_t)r * n_tok + tok];
+    raw[r] = *reinterpret_cast<const uint4*>(o_part + ((size_t)r * n_tok + tok) * kHeadDim + k);
+  }
+  float mx = l[0];
+#pragma unroll
+  for (int r = 1; r < R; ++r) mx = fmaxf(mx, l[r]);
+  float w[R], z = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) { w[r] = expf(l[r] - mx); z += w[r]; }
+  const float rz = 1.f / z;
+  float o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float wr = w[r] * rz;
+    const __half2* h = reinterpret_cast<const __half2*>(&raw[r]);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float2 v = __half22float2(h[x]);
+      o[2 * x] = fmaf(wr, v.x, o[2 * x]);
+      o[2 * x + 1] = fmaf(wr, v.y, o[2 * x + 1]);
+    }
+  }
+  store8(O + tok * kHeadDim + k, o);
+  if (lse && k == 0) lse[tok] = mx + logf(z);
+}
+
 }  // namespace lsh

@@ -343,8 +343,22 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   if (O && a.mode != lsh::kAtDirect) {
     const size_t n8 = D.n_tok * 8;
     if (a.mode == lsh::kAtPartial16)
-      lsh::combine_kernel<__half, __nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
-          a.o16, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);
+      {
+        const unsigned nb8 = (unsigned)((n8 + 255) / 256);
+        __nv_bfloat16* Ob = static_cast<__nv_bfloat16*>(O);
+        switch (D.R) {
+          case 2: lsh::combine16_kernel<2><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 3: lsh::combine16_kernel<3><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 4: lsh::combine16_kernel<4><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 5: lsh::combine16_kernel<5><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 6: lsh::combine16_kernel<6><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 7: lsh::combine16_kernel<7><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          case 8: lsh::combine16_kernel<8><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.n_tok, Ob, lse); break;
+          default:
+            lsh::combine_kernel<__half, __nv_bfloat16><<<nb8, 256, 0, st>>>(a.o16, a.lse_r, D.R,
+                                                                            D.n_tok, Ob, lse);
+        }
+      }
     else
       lsh::combine_kernel<float, __nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
           a.o32, a.lse_r, D.R, D.n_tok, static_cast<__nv_bfloat16*>(O), lse);

@@ -201,8 +201,12 @@ CASES = [
     (1, 1, 256, 1024, 1, 64, False),  # more buckets than tokens: lone tokens
     (1, 2, 64, 4, 1, 4, True),        # tiny chunks
     (1, 1, 512, 32768, 1, 64, True),  # the largest bucket count
-    (1, 2, 384, 8, 5, 64, True),      # five rounds: three fold into one running state, two into the other
+    (1, 2, 384, 8, 5, 64, True),      # five rounds of fp16 partials, combined
     (2, 1, 256, 4, 8, 64, False),     # eight rounds, non-causal
+    (1, 2, 384, 8, 3, 64, True),      # three rounds (each round count has its own combine)
+    (1, 1, 512, 16, 4, 64, False),    # four rounds
+    (1, 2, 256, 8, 6, 64, True),      # six rounds
+    (1, 1, 320, 16, 7, 64, False),    # seven rounds, ragged last tile
     (1, 1, 256, 96, 2, 64, True),     # nb/2 = 48, not a power of two: CUDA-core hash
 ]
 
