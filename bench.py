@@ -768,15 +768,14 @@ def run_recall(args):
 # for the kernels as they stand, keyed by (stage, workload); absent until
 # taken, and to be cleared whenever a kernel changes.  A stage's figure covers
 # the launches its time covers: the attention call is fwd_prep_kernel +
-# attend_tc_kernel + combine_kernel.  The L=65536 figures are from one
-# capture of the timed step (profiles/launches_fwd_bf16_L65536.md); the
-# L=16384 attention figure is the attention kernel alone, from one capture of
-# that workload's forward (profiles/attend_tc_kernel_fwd_bf16_L16384.md).
+# attend_tc_kernel + combine16_kernel.  Each is from one capture of the
+# workload's timed step (profiles/launches_fwd_bf16_L65536.md).
 TRAFFIC = {
-    ("hash", "fwd_bf16_L65536"): 67664896 + 2832384,
-    ("attend", "fwd_bf16_L65536"): (134223360 + 32006144) + (180196352 + 497440256)
-                                   + (553665792 + 58548736),
-    ("attend", "fwdbwd_bf16_L16384"): 77895168 + 90932992,
+    ("hash", "fwd_bf16_L65536"): 67661568 + 2845952,
+    ("attend", "fwd_bf16_L65536"): (134224128 + 32802304) + (179826944 + 497401088)
+                                   + (553662208 + 57920000),
+    ("attend", "fwdbwd_bf16_L16384"): (67114752 + 6025984) + (77961216 + 87083008)
+                                      + (138421504 + 14498816),
 }
 
 
