@@ -358,16 +358,18 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
         if (!at_wait(&S.tm_free, (n & 1u) ^ 1u, &S.abort)) break;
         tc::fence_after_sync();
         const uint32_t sq = tc::smem_u32(slots + (size_t)s * kBwSlotBytes);
-        const uint32_t sv = sq + 3 * kBwChunkBytes, sdo = sq + 6 * kBwChunkBytes;
+        // descriptors built once; the address field counts 16-byte units, so
+        // the other pieces of an operand are constant offsets (C(x) = x / 16)
+        const uint64_t kq = tc::sdesc_sw128(sq, 16, 1024);        // K-major rows of the slot
+        const uint64_t mq = tc::sdesc_sw128(sq, 8192, 1024);      // MN-major view of the slot
+        constexpr uint32_t CH = kBwChunkBytes >> 4, SV = 3 * CH, SDO = 6 * CH;
         // S = Q(window rows 64..191) . Qw^T,  dP = dO . Vw^T  (K-major, K = 64)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(tmem + kBwColS, tc::sdesc_sw128(sq + kBwChunkBytes + kk * 32, 16, 1024),
-                       tc::sdesc_sw128(sq + kk * 32, 16, 1024), id_s, kk > 0);
+          tc::mma_bf16(tmem + kBwColS, kq + CH + 2 * kk, kq + 2 * kk, id_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(tmem + kBwColDP, tc::sdesc_sw128(sdo + kk * 32, 16, 1024),
-                       tc::sdesc_sw128(sv + kk * 32, 16, 1024), id_s, kk > 0);
+          tc::mma_bf16(tmem + kBwColDP, kq + SDO + 2 * kk, kq + SV + 2 * kk, id_s, kk > 0);
         tc::mma_commit(&S.s_full);
         if (!at_wait(&S.p_full, n & 1u, &S.abort)) break;
         tc::fence_after_sync();
@@ -375,28 +377,23 @@ __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcA
 #pragma unroll
         for (int kk = 0; kk < 12; ++kk)
           tc::mma_bf16_ts(tmem + kBwColDQ, tmem + kBwColDS + kk * 8,
-                          tc::sdesc_sw128(sq + (kk >> 2) * kBwChunkBytes + (kk & 3) * 2048, 8192, 1024),
-                          id_q, kk > 0);
+                          mq + (kk >> 2) * CH + (kk & 3) * 128, id_q, kk > 0);
         // key side: A = P^T / dS^T of one query chunk (two 64-key atoms,
         // MN-major), B = that chunk's dO / q rows (MN-major), K = 64 queries.
         // q0 = columns 128..191 (dO rows 64..127), q1 = columns 64..127.
-        const uint32_t p0 = tc::smem_u32(opP), d0 = tc::smem_u32(opD);
+        const uint64_t mp = tc::sdesc_sw128(tc::smem_u32(opP), kBwChunkBytes, 1024);
+        const uint64_t md = tc::sdesc_sw128(tc::smem_u32(opD), kBwChunkBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          tc::mma_bf16(tmem + kBwColDV1, tc::sdesc_sw128(p0 + kk * 2048, kBwChunkBytes, 1024),
-                       tc::sdesc_sw128(sdo + kBwChunkBytes + kk * 2048, 8192, 1024), id_k, kk > 0);
-          tc::mma_bf16(tmem + kBwColDK1, tc::sdesc_sw128(d0 + kk * 2048, kBwChunkBytes, 1024),
-                       tc::sdesc_sw128(sq + 2 * kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
-                       kk > 0);
+          tc::mma_bf16(tmem + kBwColDV1, mp + 128 * kk, mq + SDO + CH + 128 * kk, id_k, kk > 0);
+          tc::mma_bf16(tmem + kBwColDK1, md + 128 * kk, mq + 2 * CH + 128 * kk, id_k, kk > 0);
         }
         if (nq == 2) {
-          const uint32_t p1 = p0 + 2 * kBwChunkBytes, d1 = d0 + 2 * kBwChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            tc::mma_bf16(tmem + kBwColDV2, tc::sdesc_sw128(p1 + kk * 2048, kBwChunkBytes, 1024),
-                         tc::sdesc_sw128(sdo + kk * 2048, 8192, 1024), id_k, kk > 0);
-            tc::mma_bf16(tmem + kBwColDK2, tc::sdesc_sw128(d1 + kk * 2048, kBwChunkBytes, 1024),
-                         tc::sdesc_sw128(sq + kBwChunkBytes + kk * 2048, 8192, 1024), id_k,
+            tc::mma_bf16(tmem + kBwColDV2, mp + 2 * CH + 128 * kk, mq + SDO + 128 * kk, id_k,
+                         kk > 0);
+            tc::mma_bf16(tmem + kBwColDK2, md + 2 * CH + 128 * kk, mq + CH + 128 * kk, id_k,
                          kk > 0);
           }
         }

@@ -522,15 +522,17 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             tc::fence_after_sync();
             tc::fence_async_smem();  // cp.async rows of this slot -> tensor-core reads
             uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
-            const uint32_t qa = tc::smem_u32(slot + kAtChunkBytes);  // chunks k0, k0+1
+            // descriptors of the slot's first chunk; the address field counts
+            // 16-byte units, so later pieces are constant offsets
+            const uint64_t dk0 = tc::sdesc_sw128(tc::smem_u32(slot), 16, 1024);
+            const uint64_t dq0 = dk0 + (kAtChunkBytes >> 4);  // chunks k0, k0+1
             const uint32_t d = tmem + b * 256;
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
-              const uint32_t kb = tc::smem_u32(slot + c * kAtChunkBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(d + c * 64, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                             tc::sdesc_sw128(kb + kk * 32, 16, 1024), idesc_s, kk > 0);
+                tc::mma_bf16(d + c * 64, dq0 + 2 * kk, dk0 + ((c * kAtChunkBytes) >> 4) + 2 * kk,
+                             idesc_s, kk > 0);
             }
             tc::mma_commit(&S.s_full[b]);
             ++n_s;
@@ -543,13 +545,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             tc::fence_after_sync();
             uint8_t* slot = slots + (size_t)s * kAtSlotBytes;
             const uint32_t pa = tmem + b * 256;  // P over S: key block c at columns 32c
+            const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(slot + 3 * kAtChunkBytes), 8192, 1024);
 #pragma unroll
             for (int c = 0; c < 3; ++c) {
-              const uint32_t vb = tc::smem_u32(slot + (3 + c) * kAtChunkBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16_ts(tmem + b * 256 + 192, pa + c * 32 + kk * 8,
-                                tc::sdesc_sw128(vb + kk * 2048, 8192, 1024), idesc_o,
+                                dv0 + ((c * kAtChunkBytes + kk * 2048) >> 4), idesc_o,
                                 (c | kk) != 0);
             }
             tc::mma_commit(&S.o_full[b]);

@@ -213,16 +213,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
           tc::fence_after_sync();
           const uint32_t sa = tc::smem_u32(stage_a + s * kGmABytes);
           const uint32_t sb = tc::smem_u32(stage_b + s * kGmBBytes);
+          // K-major: 16 K = 32 bytes along the row; MN-major: 16 K rows of
+          // 128 bytes, 64-element MN blocks 8 KB apart.  The address field
+          // counts 16-byte units: a K step adds 2 (K-major) or 128 (MN-major).
+          const uint64_t da0 = g.a_mn ? tc::sdesc_sw128(sa, 8192, 1024) : tc::sdesc_sw128(sa, 16, 1024);
+          const uint64_t db0 = g.b_mn ? tc::sdesc_sw128(sb, 8192, 1024) : tc::sdesc_sw128(sb, 16, 1024);
+          const uint32_t sta = g.a_mn ? 128u : 2u, stb = g.b_mn ? 128u : 2u;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // K-major: 16 K = 32 bytes along the row; MN-major: 16 K rows of
-            // 128 bytes, 64-element MN blocks 8 KB apart
-            const uint64_t da = g.a_mn ? tc::sdesc_sw128(sa + kk * 2048, 8192, 1024)
-                                       : tc::sdesc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t db = g.b_mn ? tc::sdesc_sw128(sb + kk * 2048, 8192, 1024)
-                                       : tc::sdesc_sw128(sb + kk * 32, 16, 1024);
-            tc::mma_bf16(d, da, db, idesc, (ks > k_lo || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(d, da0 + kk * sta, db0 + kk * stb, idesc, (ks > k_lo || kk > 0) ? 1u : 0u);
           tc::mma_commit(&S.empty[s]);  // the stage is free once these MMAs are done
         }
         if (ok) tc::mma_commit(&S.acc_full[b]);

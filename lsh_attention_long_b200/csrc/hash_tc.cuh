@@ -255,13 +255,12 @@ __global__ void __launch_bounds__(kHashTcThreads, 1)
         tc::fence_after_sync();
         const int nt = min(256, cols - t * 256);
         const uint32_t idesc = tc::idesc_bf16(128, nt, 0, 0);
-        const uint32_t qa = tc::smem_u32(q_s + (k & 1) * 16384);
-        const uint32_t ra = tc::smem_u32(rot_s + (size_t)t * 256 * 128);
+        const uint64_t dq = tc::sdesc_sw128(tc::smem_u32(q_s + (k & 1) * 16384), 16, 1024);
+        const uint64_t dr = tc::sdesc_sw128(tc::smem_u32(rot_s + (size_t)t * 256 * 128), 16, 1024);
         const uint32_t d = tmem + b * 256;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(d, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                       tc::sdesc_sw128(ra + kk * 32, 16, 1024), idesc, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)  // K steps of 32 bytes: 2 units of the address field
+          tc::mma_bf16(d, dq + 2 * kk, dr + 2 * kk, idesc, kk > 0);
         tc::mma_commit(&buf_full[job_wg(n)][b]);
         if (t == T - 1) tc::mma_commit(&q_empty[k & 1]);  // the Q buffer frees after these
       }
@@ -453,13 +452,12 @@ __global__ void __launch_bounds__(kHash4Threads, 1)
         if (t == 0 && !hash_wait(&q_full[k & 1], (k >> 1) & 1, &abort_s)) break;
         if (!hash_wait(&buf_empty[b], ((n >> 1) & 1) ^ 1, &abort_s)) break;
         tc::fence_after_sync();
-        const uint32_t qa = tc::smem_u32(q_s + (k & 1) * 16384);
-        const uint32_t ra = tc::smem_u32(rot_s + (size_t)t * 256 * 128);
+        const uint64_t dq = tc::sdesc_sw128(tc::smem_u32(q_s + (k & 1) * 16384), 16, 1024);
+        const uint64_t dr = tc::sdesc_sw128(tc::smem_u32(rot_s + (size_t)t * 256 * 128), 16, 1024);
         const uint32_t d = tmem + b * 256;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16(d, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                       tc::sdesc_sw128(ra + kk * 32, 16, 1024), idesc, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)  // K steps of 32 bytes: 2 units of the address field
+          tc::mma_bf16(d, dq + 2 * kk, dr + 2 * kk, idesc, kk > 0);
         tc::mma_commit(&buf_full[b]);
         if (t == T - 1) tc::mma_commit(&q_empty[k & 1]);
       }
