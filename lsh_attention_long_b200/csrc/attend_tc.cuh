@@ -12,7 +12,8 @@
 // Tile = two consecutive chunks (128 query rows, one TMEM lane each); its
 // window is three chunks (k-1, k, k+1), 192 keys, of which each query chunk
 // uses two.  Per tile:
-//   S  = Q[128 x 64] . K[192 x 64]^T   tcgen05.mma (three N=64 MMAs) -> TMEM
+//   S  = Q[128 x 64] . K[192 x 64]^T   tcgen05.mma (N=192, the window's three
+//                                       chunks contiguous in the slot) -> TMEM
 //   P  = masked softmax numerators      CUDA cores, fp16, written over S in TMEM
 //   O  = P[128 x 192] . V[192 x 64]     tcgen05.mma with A = P from TMEM
 // The raw queries serve as keys in the MMA; 1/|q_j| (precomputed per token)
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
   } else if (warp == kAtMmaWarp) {
     // ------------------------------------------------------ tensor-core issue
     if (lane == 0) {
-      const uint32_t idesc_s = tc::idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc_s = tc::idesc_bf16(128, 192, 0, 0);
       const uint32_t idesc_o = tc::idesc_f16(128, 64, 0, 1);
       uint32_t n_s = 0, n_p = 0;  // next S to issue, next P.V to issue
       long long idle_since = clock64();
@@ -528,12 +529,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_tc_kernel(AttnTcArgs a) 
             const uint64_t dq0 = dk0 + (kAtChunkBytes >> 4);  // chunks k0, k0+1
             const uint32_t d = tmem + b * 256;
 #pragma unroll
-            for (int c = 0; c < 3; ++c) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(d + c * 64, dq0 + 2 * kk, dk0 + ((c * kAtChunkBytes) >> 4) + 2 * kk,
-                             idesc_s, kk > 0);
-            }
+            for (int kk = 0; kk < 4; ++kk)  // N = 192: the window's three chunks at once
+              tc::mma_bf16(d, dq0 + 2 * kk, dk0 + 2 * kk, idesc_s, kk > 0);
             tc::mma_commit(&S.s_full[b]);
             ++n_s;
             progress = true;
