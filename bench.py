@@ -771,11 +771,11 @@ def run_recall(args):
 # attend_tc_kernel + combine16_kernel.  Each is from one capture of the
 # workload's timed step (profiles/launches_fwd_bf16_L65536.md).
 TRAFFIC = {
-    ("hash", "fwd_bf16_L65536"): 67661568 + 2845952,
-    ("attend", "fwd_bf16_L65536"): (134224128 + 32802304) + (179826944 + 497401088)
-                                   + (553662208 + 57920000),
-    ("attend", "fwdbwd_bf16_L16384"): (67114752 + 6025984) + (77961216 + 87083008)
-                                      + (138421504 + 14498816),
+    ("hash", "fwd_bf16_L65536"): 67685376 + 2786816,
+    ("attend", "fwd_bf16_L65536"): (134226176 + 32025856) + (179611136 + 497046784)
+                                   + (553658624 + 58092800),
+    ("attend", "fwdbwd_bf16_L16384"): (67116800 + 6149632) + (77871872 + 87319552)
+                                      + (138425856 + 14625024),
 }
 
 
