@@ -645,7 +645,7 @@ def run_fwd_bwd(args, w, world):
             "ms_fwd": round(fwd / steps, 4), "ms_bwd": round(bwd / steps, 4), "steps": steps,
             "config": workload_config(w),
             # the backward call (G = dO . O, key scales, the tensor-core kernel,
-            # the cast) against HBM with the survey's algorithmic bytes
+            # the cast) against HBM with the algorithmic bytes of stage_work
             "roofline_bwd": roofline_of(w, "bwd", bwd / steps, peaks, peak_kind,
                                         TRAFFIC.get(("bwd", w.name)))}
 
