@@ -42,10 +42,13 @@ def all_gather_heads(local: torch.Tensor, B: int, H: int, world: int, rank: int,
                      group=None) -> torch.Tensor:
     """Reassembles [B, H, ...] from every rank's [1, h1 - h0, ...] slice.
     Slices are padded to the largest one so that one all_gather of equal
-    sizes serves (NCCL and gloo both take it)."""
+    sizes serves (NCCL and gloo both take it).  A world of one rank holds
+    every head already and needs no process group."""
+    tail = tuple(local.shape[2:])
+    if world == 1:
+        return local.reshape((B, H) + tail)
     import torch.distributed as dist
     per = -(-(B * H) // world)
-    tail = tuple(local.shape[2:])
     pad = torch.zeros((per,) + tail, dtype=local.dtype, device=local.device)
     pad[:local.shape[1]] = local[0]
     bufs = [torch.empty_like(pad) for _ in range(world)]

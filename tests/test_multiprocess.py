@@ -146,3 +146,19 @@ def test_two_rank_head_shards_reassemble_the_one_rank_result(tmp_path, oracle):
     flat = ref["O"].reshape(1, 6, 256, 64)
     assert torch.equal(got[0]["O"], flat[:, 0:3])
     assert torch.equal(got[1]["O"], flat[:, 3:6])
+
+
+def test_one_rank_gather_needs_no_process_group(oracle):
+    """A world of one rank holds every head: the gather returns the forward's
+    O and lse in [B, H, ...] shape without touching torch.distributed."""
+    import torch
+    import torch.distributed as dist
+    from lsh_attention_long_b200 import workloads as W
+    from lsh_attention_long_b200.shard import forward_sharded
+    assert not dist.is_initialized()
+    inp = W.make_random(2, 3, 256, 64, 16, 2, torch.float32, seed=17)
+    out = forward_sharded(inp["Q"], inp["V"], inp["rot"], 16, 64, True, 1, 0,
+                          forward=_oracle_forward, gather=True)
+    ref = _oracle_forward(inp["Q"], inp["V"], inp["rot"], 16, 64, True)
+    assert torch.equal(out["O_full"], ref["O"])
+    assert torch.equal(out["lse_full"], ref["lse"])
