@@ -211,6 +211,56 @@ __device__ __forceinline__ void drain_dv(uint32_t region, bool v1, bool v2, floa
   }
 }
 
+// Per token, before the backward: G = dO . O, the key scale log2(e)/(|q|
+// sqrt(d)) (0 for a zero row) and zeroed fp32 gradient rows.  Eight threads
+// per token: 16 bytes of each input row, 32 bytes of each gradient row.
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ Q,
+                                const __nv_bfloat16* __restrict__ O,
+                                const __nv_bfloat16* __restrict__ dO, size_t n_tok,
+                                float* __restrict__ G, float* __restrict__ rn,
+                                float* __restrict__ dq_acc, float* __restrict__ dv_acc) {
+  const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t tok = g >> 3;
+  const int k = (int)(g & 7) * 8;
+  const bool in = tok < n_tok;
+  float ssq = 0.f, dot = 0.f;
+  if (in) {
+    float x[8], y[8];
+    load8(Q + tok * kHeadDim + k, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ssq = fmaf(x[e], x[e], ssq);
+    load8(O + tok * kHeadDim + k, x);
+    load8(dO + tok * kHeadDim + k, y);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dot = fmaf(x[e], y[e], dot);
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    store8(dq_acc + tok * kHeadDim + k, z);
+    store8(dv_acc + tok * kHeadDim + k, z);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  if (in && k == 0) {
+    rn[tok] = ssq > 0.f ? rsqrtf(ssq) * (0.125f * kLog2e) : 0.f;
+    G[tok] = dot;
+  }
+}
+
+// dQ and dV from the fp32 gradient rows, eight consecutive values per thread.
+template <typename OutT>
+__global__ void bwd_cast_kernel(const float* __restrict__ dq_acc, const float* __restrict__ dv_acc,
+                                size_t n, OutT* __restrict__ dQ, OutT* __restrict__ dV) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  float x[8];
+  load8(dq_acc + i, x);
+  store8(dQ + i, x);
+  load8(dv_acc + i, x);
+  store8(dV + i, x);
+}
+
 __global__ void __launch_bounds__(kBwThreads, 1) attend_bwd_tc_kernel(AttnBwdTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);

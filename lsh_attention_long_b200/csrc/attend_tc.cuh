@@ -276,24 +276,6 @@ __device__ __noinline__ float exact_row_max(uint32_t region, int qc, const uint3
   return mx2 == -INFINITY ? 0.f : mx2;
 }
 
-// log2(e) / (|q| sqrt(d)) per token (0 for a zero row): the key
-// normalisation and score scale, in the log2 units the softmax uses.
-__global__ void key_scale_kernel(const __nv_bfloat16* __restrict__ Q, size_t n_tok,
-                                 float* __restrict__ rn) {
-  const size_t tok = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (tok >= n_tok) return;
-  float ssq = 0.f;
-#pragma unroll
-  for (int k = 0; k < kHeadDim; k += 8) {
-    float x[8];
-    load8(Q + tok * kHeadDim + k, x);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ssq = fmaf(x[e], x[e], ssq);
-  }
-  rn[tok] = ssq > 0.f ? rsqrtf(ssq) * (0.125f * kLog2e) : 0.f;
-}
-
-
 // Per token, before the forward: the key scale log2(e)/(|q| sqrt(d)) (0 for a
 // zero row) and the value row in fp16 for the P.V product.  Eight threads
 // per token, 16 bytes of q and of v each.

@@ -437,15 +437,14 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
   float* dk = reinterpret_cast<float*>(reinterpret_cast<char*>(dv) + acc_bytes);
   // the tensor-core kernel projects dkhat into dq itself: no dk accumulator
   const bool tc_path = attend_tc_supported(D);
-  if (cudaMemsetAsync(dq, 0, (tc_path ? 2 : 3) * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
   const T* q = static_cast<const T*>(Q);
   const unsigned tb = (unsigned)((D.n_tok + 255) / 256);
-  lsh::bwd_dot_kernel<T><<<tb, 256, 0, st>>>(static_cast<const T*>(O), static_cast<const T*>(dO),
-                                             D.n_tok, G);
-  if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
+  const unsigned tb8 = (unsigned)((D.n_tok * 8 + 255) / 256);  // eight threads per token
   if (tc_path) {
-    lsh::key_scale_kernel<<<tb, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(Q), D.n_tok,
-                                              rn);
+    // G, key scales and zeroed dq, dv rows in one pass
+    lsh::bwd_prep_kernel<<<tb8, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(O),
+        reinterpret_cast<const __nv_bfloat16*>(dO), D.n_tok, G, rn, dq, dv);
     if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
     lsh::AttnBwdTcArgs b;
     b.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
@@ -473,6 +472,10 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
     const unsigned grid = (unsigned)(b.total_tiles < sms ? b.total_tiles : sms);
     lsh::attend_bwd_tc_kernel<<<grid, lsh::kBwThreads, smem, st>>>(b);
   } else {
+    if (cudaMemsetAsync(dq, 0, 3 * acc_bytes, st) != cudaSuccess) return LSH_ERR_CUDA;
+    lsh::bwd_dot_kernel<T><<<tb, 256, 0, st>>>(static_cast<const T*>(O),
+                                               static_cast<const T*>(dO), D.n_tok, G);
+    if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
     const size_t smem = lsh::simt_bwd_smem_bytes(a.chunk, a.W);
     lsh_status s0 = allow_smem(lsh::attend_bwd_simt_kernel<T>, smem);
     if (s0 != LSH_OK) return s0;
@@ -482,13 +485,22 @@ lsh_status attend_bwd_launch(const Dims& D, const void* Q, const void* V, const 
         1.f / (float)D.R, dq, dk, dv);
   }
   if (last_launch() != LSH_OK) return LSH_ERR_CUDA;
-  if (f32_out)
-    lsh::bwd_finalize_kernel<T, float><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv,
-                                                           D.n_tok, static_cast<float*>(dQ),
+  if (tc_path) {  // the tensor-core kernel has already projected dkhat into dq
+    const size_t n = D.n_tok * kHeadDim;
+    if (f32_out)
+      lsh::bwd_cast_kernel<float><<<tb8, 256, 0, st>>>(dq, dv, n, static_cast<float*>(dQ),
+                                                       static_cast<float*>(dV));
+    else
+      lsh::bwd_cast_kernel<T><<<tb8, 256, 0, st>>>(dq, dv, n, static_cast<T*>(dQ),
+                                                   static_cast<T*>(dV));
+  } else if (f32_out) {
+    lsh::bwd_finalize_kernel<T, float><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok,
+                                                           static_cast<float*>(dQ),
                                                            static_cast<float*>(dV));
-  else
-    lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, tc_path ? nullptr : dk, dv, D.n_tok,
-                                                    static_cast<T*>(dQ), static_cast<T*>(dV));
+  } else {
+    lsh::bwd_finalize_kernel<T><<<tb, 256, 0, st>>>(q, dq, dk, dv, D.n_tok, static_cast<T*>(dQ),
+                                                    static_cast<T*>(dV));
+  }
   return last_launch();
 }
 
