@@ -146,6 +146,13 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // Launched as a programmatic dependent of the previous grid in the stream,
+  // this CTA may have got here while that grid still runs: every global
+  // access below waits for it to complete and for its writes to be visible.
+  // Then the next grid may start its own set-up (it can only take SMs this
+  // grid has left: each CTA holds most of an SM's shared memory).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t tmem = S.tmem_base;
   const int n_n = g.N / kGmBN;
   const int n_units = (g.M / kGmBM) * n_n * g.k_splits;

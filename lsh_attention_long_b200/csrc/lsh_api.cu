@@ -861,8 +861,20 @@ lsh_status gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const lsh::
   if (s0 != LSH_OK) return s0;
   const int units = (g.M / lsh::kGmBM) * (g.N / lsh::kGmBN) * g.k_splits;
   const int sms = num_sms();
-  lsh::gemm_tc_kernel<<<(unsigned)(units < sms ? units : sms), lsh::kGmThreads, smem, st>>>(ma, mb,
-                                                                                          g);
+  // programmatic dependent launch: the grid may be scheduled while the
+  // previous one in the stream finishes; the kernel waits for it
+  // (griddepcontrol.wait) before touching global memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(units < sms ? units : sms));
+  cfg.blockDim = dim3(lsh::kGmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lsh::gemm_tc_kernel, ma, mb, g) != cudaSuccess) return LSH_ERR_CUDA;
   return last_launch();
 }
 
