@@ -81,4 +81,16 @@ __device__ __forceinline__ void store8(float* p, const float* v) {
   *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// Programmatic dependent launch.  A grid launched with the programmatic
+// stream serialization attribute may start while the previous grid in its
+// stream still runs; grid_dep_wait() blocks until that grid has completed
+// and its memory writes are visible (a no-op for a grid launched without
+// the attribute), so it comes before a kernel's first global access.
+// grid_dep_launch() lets the next grid in the stream be scheduled (once
+// every CTA of this grid has called it or exited).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace lsh

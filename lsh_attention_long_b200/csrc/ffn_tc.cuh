@@ -151,8 +151,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   // access below waits for it to complete and for its writes to be visible.
   // Then the next grid may start its own set-up (it can only take SMs this
   // grid has left: each CTA holds most of an SM's shared memory).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_dep_wait();
+  grid_dep_launch();
   const uint32_t tmem = S.tmem_base;
   const int n_n = g.N / kGmBN;
   const int n_units = (g.M / kGmBM) * n_n * g.k_splits;
