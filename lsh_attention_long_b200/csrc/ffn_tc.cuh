@@ -62,6 +62,10 @@ struct GemmArgs {
   const float* R;    // kEpiAddF32: [M][ldr], or NULL (C32 = acc)
   int ldr;
   long long wait_limit;
+  // 1: the operands this launch loads are not written by the previous grid
+  // in the stream (only its stores must follow that grid), so loads and MMAs
+  // start at once and the epilogue waits; 0: every global access waits
+  int late_wait;
 };
 
 constexpr int kGmStageOutBytes = 4 * 32 * 128;  // per epilogue warp: 32 rows of 128 B
@@ -147,11 +151,12 @@ __global__ void __launch_bounds__(kGmThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   // Launched as a programmatic dependent of the previous grid in the stream,
-  // this CTA may have got here while that grid still runs: every global
-  // access below waits for it to complete and for its writes to be visible.
-  // Then the next grid may start its own set-up (it can only take SMs this
-  // grid has left: each CTA holds most of an SM's shared memory).
-  grid_dep_wait();
+  // this CTA may have got here while that grid still runs: global accesses
+  // wait for it to complete and for its writes to be visible (all of them,
+  // or with late_wait only the epilogue's).  Then the next grid may start its
+  // own set-up (it can only take SMs this grid has left: each CTA holds most
+  // of an SM's shared memory).
+  if (!g.late_wait) grid_dep_wait();
   grid_dep_launch();
   const uint32_t tmem = S.tmem_base;
   const int n_n = g.N / kGmBN;
@@ -246,6 +251,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    if (g.late_wait) grid_dep_wait();
     // Each thread owns one output row (its TMEM lane) and works 32 columns
     // at a time.  Per-row operands (mask, residual) are loaded before the
     // TMEM load they are combined with; the bias of the tile sits in shared

@@ -922,6 +922,11 @@ lsh_status lsh_ffn_forward(int32_t tokens, int32_t d_model, int32_t d_ff, int32_
     g1.bias = static_cast<const __nv_bfloat16*>(b1);
     g1.relu = 1;
     g1.C = H; g1.ldc = d_ff;
+    // after the first chunk, the grid before this one is the previous
+    // chunk's second product, which reads H but writes nothing this product
+    // loads (X and W1 were complete before the first chunk's wait returned):
+    // only the stores into H must wait for it
+    g1.late_wait = c0 > 0 ? 1 : 0;
     s = gemm_launch(mx, mw1, g1, st);
     if (s != LSH_OK) return s;
     // Y[c0 : c0+n] = H W2^T + b2
