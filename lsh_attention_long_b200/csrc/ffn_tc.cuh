@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 // gradients): thread x of block (y) sums its column over a slab of rows.
 __global__ void colsum_add_kernel(const __nv_bfloat16* __restrict__ a, int rows, int cols,
                                   int rows_per_block, float* __restrict__ out) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   const int r0 = blockIdx.y * rows_per_block;

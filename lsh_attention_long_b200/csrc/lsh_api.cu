@@ -67,6 +67,27 @@ inline lsh_status last_launch() {
   return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }
 
+// Launches a kernel as a programmatic dependent of the previous grid in the
+// stream: it may be scheduled while that grid finishes, and waits for it
+// (grid_dep_wait) before the global accesses that depend on it.
+template <typename... KArgs, typename... Args>
+lsh_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  return last_launch();
+}
+
 // Opt a kernel into more than 48 KB of dynamic shared memory.
 template <typename K>
 lsh_status allow_smem(K kernel, size_t bytes) {
@@ -861,21 +882,8 @@ lsh_status gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const lsh::
   if (s0 != LSH_OK) return s0;
   const int units = (g.M / lsh::kGmBM) * (g.N / lsh::kGmBN) * g.k_splits;
   const int sms = num_sms();
-  // programmatic dependent launch: the grid may be scheduled while the
-  // previous one in the stream finishes; the kernel waits for it
-  // (griddepcontrol.wait) before touching global memory
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(units < sms ? units : sms));
-  cfg.blockDim = dim3(lsh::kGmThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lsh::gemm_tc_kernel, ma, mb, g) != cudaSuccess) return LSH_ERR_CUDA;
-  return last_launch();
+  return launch_pdl(lsh::gemm_tc_kernel, dim3((unsigned)(units < sms ? units : sms)),
+                    dim3(lsh::kGmThreads), smem, st, ma, mb, g);
 }
 
 // K ranges per output tile for a weight-gradient product: enough work units
@@ -979,6 +987,12 @@ lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32
       !bf16_map(&mdy_mn, dY, T, D, 64) || !bf16_map(&mh_mn, H, C, F, 64) ||
       !bf16_map(&mda_mn, dA, C, F, 64) || !bf16_map(&mx_mn, X, T, D, 64))
     return LSH_ERR_CUDA;
+  // Every launch below is a programmatic dependent of the one before.  A
+  // grid completes only after its wait has returned, so when a grid is
+  // launched every grid two or more launches back has completed, and a grid
+  // whose loads read only inputs or such grids' outputs may load and multiply
+  // at once and wait in its epilogue (late_wait).  Only dX = R + dA W1 loads
+  // what its immediate predecessor writes.
   for (int c0 = 0; c0 < tokens; c0 += chunk) {
     const int n = tokens - c0 < chunk ? tokens - c0 : chunk;
     // H = max(0, X W1^T + b1), recomputed for the chunk
@@ -987,6 +1001,7 @@ lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32
     g1.bias = static_cast<const __nv_bfloat16*>(b1);
     g1.relu = 1;
     g1.C = H; g1.ldc = d_ff;
+    g1.late_wait = c0 > 0 ? 1 : 0;  // its stores into H wait for the last chunk's readers
     if ((s = gemm_launch(mx, mw1, g1, st)) != LSH_OK) return s;
     // dA = (dY W2) where H > 0: the gradient at the pre-activation
     lsh::GemmArgs g2 = gemm_args(n, d_ff, d_model, lsh::kEpiMask);
@@ -994,6 +1009,7 @@ lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32
     g2.b_mn = 1;  // W2 [d_model][d_ff] is [K][N]
     g2.mask = H; g2.ldm = d_ff;
     g2.C = dA; g2.ldc = d_ff;
+    g2.late_wait = 1;  // loads dY and W2; its epilogue reads the mask H
     if ((s = gemm_launch(mdy, mw2_mn, g2, st)) != LSH_OK) return s;
     // dX = R + dA W1
     lsh::GemmArgs g3 = gemm_args(n, d_model, d_ff, lsh::kEpiAddF32);
@@ -1006,20 +1022,25 @@ lsh_status lsh_ffn_backward(int32_t tokens, int32_t d_model, int32_t d_ff, int32
     g4.a_mn = 1; g4.b_mn = 1; g4.a_row0 = c0;
     g4.k_splits = k_splits_for((d_model / lsh::kGmBM) * (d_ff / lsh::kGmBN), n);
     g4.C32 = dW2; g4.ldc32 = d_ff;
+    g4.late_wait = 1;  // loads dY and H (two launches back)
     if ((s = gemm_launch(mdy_mn, mh_mn, g4, st)) != LSH_OK) return s;
     lsh::GemmArgs g5 = gemm_args(d_ff, d_model, n, lsh::kEpiAtomicF32);
     g5.a_mn = 1; g5.b_mn = 1; g5.b_row0 = c0;
     g5.k_splits = k_splits_for((d_ff / lsh::kGmBM) * (d_model / lsh::kGmBN), n);
     g5.C32 = dW1; g5.ldc32 = d_model;
+    g5.late_wait = 1;  // loads dA (three launches back) and X
     if ((s = gemm_launch(mda_mn, mx_mn, g5, st)) != LSH_OK) return s;
     // db2 += column sums of dY, db1 += column sums of dA
     const int rpb = 256;
     const dim3 gb2((unsigned)((d_model + 255) / 256), (unsigned)((n + rpb - 1) / rpb));
-    lsh::colsum_add_kernel<<<gb2, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dY) + (size_t)c0 * d_model, n, d_model, rpb, db2);
+    if ((s = launch_pdl(lsh::colsum_add_kernel, gb2, dim3(256), 0, st,
+                        static_cast<const __nv_bfloat16*>(dY) + (size_t)c0 * d_model, n,
+                        d_model, rpb, db2)) != LSH_OK)
+      return s;
     const dim3 gb1((unsigned)((d_ff + 255) / 256), (unsigned)((n + rpb - 1) / rpb));
-    lsh::colsum_add_kernel<<<gb1, 256, 0, st>>>(dA, n, d_ff, rpb, db1);
-    if ((s = last_launch()) != LSH_OK) return s;
+    if ((s = launch_pdl(lsh::colsum_add_kernel, gb1, dim3(256), 0, st,
+                        static_cast<const __nv_bfloat16*>(dA), n, d_ff, rpb, db1)) != LSH_OK)
+      return s;
   }
   return LSH_OK;
 }
