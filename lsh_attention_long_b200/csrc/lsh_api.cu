@@ -317,12 +317,20 @@ lsh_status attend_tc_launch(const Dims& D, const void* Q, const void* V, const u
   a.n_chunks = D.L / 64;
   a.causal = D.causal;
   a.n_tiles = (a.n_chunks + 1) / 2;
-  a.tpi = a.n_tiles < 4 ? a.n_tiles : 4;
-  a.ipr = (a.n_tiles + a.tpi - 1) / a.tpi;
   // items head by head, every round of a head before the next head: tiles
   // do not depend on one another, so the CTAs in flight share one or a few
   // heads' q and v rows, which stay in L2 across the rounds
   const int sms = num_sms();
+  // tiles per item: a run of consecutive tiles shares window chunks, so
+  // eight beat four unless they lengthen the tail (items go to CTAs
+  // round-robin; the busiest CTA runs ceil(items / CTAs) of them)
+  const auto busiest = [&](int t) {
+    const long long items = (long long)D.R * a.BH * ((a.n_tiles + t - 1) / t);
+    return (items + sms - 1) / sms * t;
+  };
+  a.tpi = busiest(8) <= busiest(4) ? 8 : 4;
+  if (a.tpi > a.n_tiles) a.tpi = a.n_tiles;
+  a.ipr = (a.n_tiles + a.tpi - 1) / a.tpi;
   a.heads_per_block = 1;
   a.n_items = (long long)a.R * a.BH * a.ipr;
   a.wait_limit = g_wait_limit;
