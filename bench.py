@@ -771,11 +771,11 @@ def run_recall(args):
 # attend_tc_kernel + combine16_kernel.  Each is from one capture of the
 # workload's timed step (profiles/launches_fwd_bf16_L65536.md).
 TRAFFIC = {
-    ("hash", "fwd_bf16_L65536"): 67685376 + 2786816,
-    ("attend", "fwd_bf16_L65536"): (134226176 + 32025856) + (179611136 + 497046784)
-                                   + (553658624 + 58092800),
-    ("attend", "fwdbwd_bf16_L16384"): (67116800 + 6149632) + (77871872 + 87319552)
-                                      + (138425856 + 14625024),
+    ("hash", "fwd_bf16_L65536"): 67661824 + 2908928,
+    ("attend", "fwd_bf16_L65536"): (134232576 + 31965440) + (182373888 + 497529344)
+                                   + (553657856 + 57975808),
+    ("attend", "fwdbwd_bf16_L16384"): (67115264 + 6037504) + (77978368 + 85642240)
+                                      + (138419712 + 14423552),
 }
 
 
