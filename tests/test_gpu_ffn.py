@@ -136,3 +136,34 @@ def test_ffn_backward_at_full_size(oracle, parity_record):
                           "max_abs": {"dX": err, "db2": err_db2}, "tol": TOL})
     assert err <= TOL
     assert err_db2 <= TOL * scale
+
+
+def test_back_to_back_chunks_are_ordered():
+    """Consecutive GEMM launches overlap their set-up with the previous
+    product's last tiles, and a later chunk's hidden product loads and
+    multiplies before the previous output product has finished.  Repeated
+    runs of eight chunks, with one workspace reused and nothing in between,
+    must give bit-identical outputs (forward Y, backward dX: neither is
+    accumulated with atomics), so no chunk reads or overwrites the hidden
+    activation out of order."""
+    inp = W.ffn_inputs(1024, 512, 2048, seed=21, backward=True)
+    t = {k: v.cuda() for k, v in inp.items()}
+    ws = L.ffn_workspace(1024, 512, 2048, 128, t["X"].device)
+    first = None
+    for _ in range(20):
+        Y = L.lsh_ffn_forward(t["X"], t["W1"], t["b1"], t["W2"], t["b2"], 128, ws=ws)
+        if first is None:
+            first = Y.clone()
+        else:
+            assert torch.equal(Y, first)
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
+    dX0 = None
+    for _ in range(10):
+        dX, _ = L.lsh_ffn_backward(t["X"], t["W1"], t["b1"], t["W2"], t["dY"], 128)
+        if dX0 is None:
+            dX0 = dX.clone()
+        else:
+            assert torch.equal(dX, dX0)
+    torch.cuda.synchronize()
+    assert L.lsh_device_status() == 0
